@@ -1,0 +1,136 @@
+"""Router: block pooling, pooled block softmax, cumulative-mass tiers (oracle).
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).
+
+"Triage" (zhuanzhiai paper page, abstract) routes every tile from block
+statistics; "HierPAS" (conference listing, abstract) estimates the attention
+pattern cheaply and gives progressively reduced precision to less critical
+regions; "APT" (Lattice paper summary) selects and assigns precision with two
+thresholds on attention probability (APDT).  The pooled-mass router restates
+these at tile level:
+
+1. Blocks.  Query block i holds rows [i*Bq, min(N, (i+1)*Bq)); key block j
+   holds keys [j*Bk, min(N, (j+1)*Bk)) and has n_j keys (ragged tails keep
+   their real size).
+2. Pooling.  qbar_i, kbar_j, vbar_j are fp64 means of the bf16 rows; the skip
+   tier uses their bf16 (round to nearest even) copies.
+3. Pooled mass.  sbar_ij = qbar_i . kbar_j * scale; M_ij = n_j exp(sbar_ij -
+   max_j sbar_ij) / sum_j (.)  (each block weighted by its key count, as the
+   skip tier weights block j by n_j).
+4. Tiers.  Sort j by (-M_ij, j); C_r is the exclusive prefix sum of the sorted
+   masses; the tile at rank r takes the most precise tier t whose threshold
+   tau_t satisfies C_r < tau_t, else it is skipped (the tile that crosses a
+   threshold is kept: the smallest set covering tau).  Then every key block
+   whose token range meets query block i's range is made full.
+5. Flags.  A tile is flagged when |C_r - tau_t| <= 1e-5 tau_t for some t, or
+   when it and a sort neighbour have |M - M'| <= 1e-5 max(M, M') and got
+   different tiers from the prefix rule: only there may a GPU router differ.
+6. Lists.  Per row: full blocks ascending, then residual, then low, then skip.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from .formats import bf16_rne
+
+TIER_SKIP, TIER_LOW, TIER_RES, TIER_FULL = 0, 1, 2, 3
+FLAG_REL = 1e-5
+
+
+def block_ranges(N: int, block: int):
+    return [(b * block, min(N, (b + 1) * block)) for b in range(-(-N // block))]
+
+
+def pool_means(X: np.ndarray, block: int):
+    """fp64 means of each block of rows, and the row counts n_j."""
+    rngs = block_ranges(X.shape[0], block)
+    means = np.stack([X[a:b].mean(axis=0) for a, b in rngs])
+    counts = np.array([b - a for a, b in rngs], dtype=np.int64)
+    return means, counts
+
+
+def pooled_mass(qbar: np.ndarray, kbar: np.ndarray, n_k: np.ndarray, scale: float):
+    """M [nQb, nKb]: n_j-weighted softmax over key blocks of pooled logits."""
+    s = (qbar @ kbar.T) * scale
+    w = n_k[None, :] * np.exp(s - s.max(axis=1, keepdims=True))
+    return w / w.sum(axis=1, keepdims=True)
+
+
+def diag_blocks(i: int, block_q: int, block_k: int, N: int):
+    """Key blocks whose token range intersects query block i's token range."""
+    a, b = i * block_q, min(N, (i + 1) * block_q)
+    return list(range(a // block_k, (b - 1) // block_k + 1))
+
+
+def tier_codes_for(tau) -> list:
+    """Tier of each threshold, most precise first: (full, low) or (full, res, low)."""
+    if len(tau) == 2:
+        return [TIER_FULL, TIER_LOW]
+    if len(tau) == 3:
+        return [TIER_FULL, TIER_RES, TIER_LOW]
+    if len(tau) == 1:
+        return [TIER_FULL]
+    raise ValueError("1 to 3 thresholds")
+
+
+def assign_tiers(M_row: np.ndarray, tau, diag=()):
+    """Tiers (uint8 [nKb]) and flags (bool [nKb]) of one query-block row."""
+    n = M_row.shape[0]
+    j = np.arange(n)
+    order = np.lexsort((j, -M_row))                  # primary -M, secondary j
+    Ms = M_row[order]
+    C = np.concatenate([[0.0], np.cumsum(Ms)[:-1]])  # exclusive prefix
+    codes = tier_codes_for(tau)
+    tier_sorted = np.full(n, TIER_SKIP, dtype=np.uint8)
+    for t in reversed(range(len(tau))):              # most precise tier wins
+        tier_sorted[C < tau[t]] = codes[t]
+    flag_sorted = np.zeros(n, dtype=bool)
+    for t in range(len(tau)):
+        flag_sorted |= np.abs(C - tau[t]) <= FLAG_REL * tau[t]
+    if n > 1:
+        near = np.abs(Ms[1:] - Ms[:-1]) <= FLAG_REL * np.maximum(Ms[1:], Ms[:-1])
+        diff = tier_sorted[1:] != tier_sorted[:-1]
+        pair = near & diff
+        flag_sorted[1:] |= pair
+        flag_sorted[:-1] |= pair
+    tiers = np.empty(n, dtype=np.uint8)
+    flags = np.empty(n, dtype=bool)
+    tiers[order] = tier_sorted
+    flags[order] = flag_sorted
+    for jj in diag:
+        tiers[jj] = TIER_FULL
+    return tiers, flags
+
+
+def row_lists(tiers_row: np.ndarray):
+    """counts [full, res, low, skip] and the key-block list in that order, each ascending."""
+    groups = [np.nonzero(tiers_row == t)[0] for t in (TIER_FULL, TIER_RES, TIER_LOW, TIER_SKIP)]
+    counts = np.array([len(g) for g in groups], dtype=np.int32)
+    return counts, np.concatenate(groups).astype(np.int32)
+
+
+def route_head(Qh, Kh, Vh, tau, block_q: int, block_k: int, scale: float = 0.0,
+               keep_diag_full: bool = True) -> dict:
+    """Router output for one head (fp64 values of bf16 Q, K, V [N, d])."""
+    N, d = Qh.shape
+    if scale == 0.0:
+        scale = 1.0 / math.sqrt(d)
+    qbar, _ = pool_means(Qh, block_q)
+    kbar, n_k = pool_means(Kh, block_k)
+    vbar, _ = pool_means(Vh, block_k)
+    M = pooled_mass(qbar, kbar, n_k, scale)
+    nqb, nkb = M.shape
+    tiers = np.empty((nqb, nkb), dtype=np.uint8)
+    flags = np.empty((nqb, nkb), dtype=bool)
+    counts = np.empty((nqb, 4), dtype=np.int32)
+    lists = np.empty((nqb, nkb), dtype=np.int32)
+    for i in range(nqb):
+        diag = diag_blocks(i, block_q, block_k, N) if keep_diag_full else ()
+        tiers[i], flags[i] = assign_tiers(M[i], tau, diag)
+        counts[i], lists[i] = row_lists(tiers[i])
+    return {"qbar": qbar, "kbar": kbar, "vbar": vbar, "n_k": n_k, "M": M,
+            "kbar_b": bf16_rne(kbar), "vbar_b": bf16_rne(vbar), "scale": scale,
+            "tiers": tiers, "flags": flags, "counts": counts, "lists": lists}
