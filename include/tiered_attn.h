@@ -1,0 +1,181 @@
+/*
+ * tiered_attn.h -- C ABI of the tiered-precision block-sparse attention library
+ * for video diffusion transformers (libtiered_attn.so, sm_100a).
+ *
+ * The method.  Self-attention over the tokens of a video latent is split into
+ * (query-block, key-block) tiles.  A router working from cheap block statistics
+ * (pooled block means of Q and K) assigns every tile one of four tiers:
+ *   full      computed in bf16;
+ *   low       computed in a reduced precision (FP8 e4m3, or NVFP4: e2m1 values
+ *             with a ue4m3 scale per 16 elements);
+ *   residual  NVFP4 with a second NVFP4 term for x - dequant(x);
+ *   skip      replaced by its block means: block j of n_j keys adds
+ *             n_j * exp(q . kbar_j * scale) to the softmax denominator and that
+ *             weight times vbar_j to the numerator.
+ * All tiers are then folded into one flash-style online-softmax pass.
+ * Sources: "Triage" (zhuanzhiai paper page, abstract: skip by block means,
+ * skim in NVFP4, refine with an NVFP4 residual, router from block statistics,
+ * one fused pass); "HierPAS" (conference listing, abstract: progressively
+ * reduced precision for less critical regions, cheap pattern estimate);
+ * "APT" (Lattice paper summary: two thresholds on attention probability
+ * choose selection and precision).  The pooled-mass thresholds below are the
+ * tile-level form of those two thresholds.
+ *
+ * Conventions shared by every entry point.
+ *  - Tensors Q, K, V, O are bf16, logically [B, H, N, d], innermost dimension
+ *    contiguous; the element strides of the B, H and N dimensions are given in
+ *    ta_params.  Base pointers must be 16-byte aligned and stride_n * 2 bytes a
+ *    multiple of 16.
+ *  - Pointers named *_dev are device pointers; *_host are host pointers (pinned
+ *    memory gives asynchronous copies).  The caller owns and allocates every
+ *    buffer, including the workspace; the library allocates no memory and keeps
+ *    no state between calls (besides cached driver entry points).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously on it; only the calls documented as
+ *    synchronising wait for the device.
+ *  - Every call validates its arguments on the host first and returns a
+ *    ta_status without launching anything when they are invalid.  Launch
+ *    failures return TA_ERR_CUDA.  Errors found by a kernel (a bounded wait that
+ *    ran out) are written to the workspace's status word and read back with
+ *    tiered_attn_get_status().
+ */
+#ifndef TIERED_ATTN_H
+#define TIERED_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TA_OK = 0,
+  TA_ERR_INVALID_ARG = -1,   /* bad params, null or misaligned pointer        */
+  TA_ERR_UNSUPPORTED = -2,   /* valid but not built (e.g. d not in {64,128})  */
+  TA_ERR_WORKSPACE = -3,     /* workspace too small                           */
+  TA_ERR_CUDA = -4,          /* a CUDA runtime / driver call failed           */
+  TA_ERR_TIMEOUT = -5        /* a kernel's bounded wait ran out (device side) */
+} ta_status;
+
+typedef enum {
+  TA_LOW_NONE = 0,           /* two tiers only: full and skip                 */
+  TA_LOW_FP8_E4M3 = 1,       /* low tier in FP8 e4m3, one power-of-two scale per tile */
+  TA_LOW_NVFP4 = 2,          /* low tier in NVFP4 (e2m1 + ue4m3 scale per 16)  */
+  TA_LOW_NVFP4_RES = 3       /* NVFP4 low tier plus an NVFP4+residual tier    */
+} ta_low_format;
+
+/* Tier codes stored in the tier map. */
+enum { TA_TIER_SKIP = 0, TA_TIER_LOW = 1, TA_TIER_RES = 2, TA_TIER_FULL = 3 };
+
+typedef struct {
+  int32_t B, H, N, d;        /* batch, heads, tokens, head dim (d in {64,128}) */
+  int32_t block_q, block_k;  /* tile rows / keys, each in {64,128}            */
+  int32_t low;               /* ta_low_format                                 */
+  int32_t n_thresholds;      /* 1 (full only), 2 (full, low), 3 (full, res, low) */
+  double  tau[3];            /* ascending cumulative-mass thresholds          */
+  int32_t keep_diag_full;    /* 1: key blocks meeting the query block's token
+                                range are always full                          */
+  int32_t p_offset_log2;     /* o in P' = 2^o exp(s - m): lifts P' into the
+                                FP8 / FP4 grids; cancels in O (0..15)          */
+  float   softmax_scale;     /* 0 selects 1/sqrt(d)                           */
+  int32_t debug_flags;       /* test hooks, 0 in normal use (see TA_DEBUG_*)  */
+  int64_t stride_b, stride_h, stride_n;  /* element strides of Q, K, V, O     */
+} ta_params;
+
+/* Test hook: the attention producer never loads the first K tile, so the
+ * kernel's bounded wait runs out and the status word reports TA_ERR_TIMEOUT. */
+#define TA_DEBUG_DROP_FIRST_K 1
+
+/* Device pointers into a planned workspace (see tiered_attn_plan_views).
+ * BH = B*H, nQb = ceil(N/block_q), nKb = ceil(N/block_k), Np = 16*ceil(N/16).
+ * Pointers of data the configured low format does not produce are NULL. */
+typedef struct {
+  int32_t* status;           /* int32[4]: [0] ta_status of the last kernel error */
+  double*  qbar;             /* f64 [BH, nQb, d]  block means of Q            */
+  double*  kbar;             /* f64 [BH, nKb, d]  block means of K            */
+  uint16_t* kbar_b;          /* bf16 [BH, nKb, d] round-to-nearest-even of kbar */
+  uint16_t* vbar_b;          /* bf16 [BH, nKb, d] same for V                  */
+  int32_t* n_k;              /* int32 [nKb] keys per key block                */
+  double*  logits;           /* f64 [BH, nQb, nKb] pooled logits * scale      */
+  double*  mass;             /* f64 [BH, nQb, nKb] pooled block mass M        */
+  uint8_t* tier_map;         /* u8  [BH, nQb, nKb] TA_TIER_* per tile          */
+  int32_t* row_counts;       /* i32 [BH, nQb, 4] tiles per tier: full, res, low, skip */
+  int32_t* row_lists;        /* i32 [BH, nQb, nKb] key blocks: full ascending,
+                                then res, low, skip (each ascending)           */
+  /* FP8 copies: codes u8 [BH, N, d] (row-major like the input), scales f32
+   * per tile [BH, nQb] for Q and [BH, nKb] for K and V.
+   * NVFP4 copies: Q, K codes packed two per byte along d, u8 [BH, N, d/2]
+   * (element 2c in the low nibble), scales ue4m3 u8 [BH, N, d/16];
+   * V codes transposed and packed along tokens, u8 [BH, d, Np/2], scales
+   * u8 [BH, Np/16, d] (groups of 16 tokens from token 0, zero past N). */
+  uint8_t* q_codes; uint8_t* k_codes; uint8_t* v_codes;
+  void*    q_scales; void* k_scales; void* v_scales;
+  /* residual NVFP4 copies (TA_LOW_NVFP4_RES), same layouts as above */
+  uint8_t* rq_codes; uint8_t* rk_codes; uint8_t* rv_codes;
+  uint8_t* rq_scales; uint8_t* rk_scales; uint8_t* rv_scales;
+  /* bf16 [BH, N, d] dequantised values of the low copies (exact in bf16) */
+  uint16_t* dq; uint16_t* dk; uint16_t* dv;
+  /* bf16 [BH, N, d] dequantised residual copies (TA_LOW_NVFP4_RES) */
+  uint16_t* drq; uint16_t* drk; uint16_t* drv;
+} ta_plan_views;
+
+/* Bytes of workspace that tiered_attn_plan / tiered_attn_forward need for
+ * `p`; 0 when `p` is invalid or unsupported.  Host only, no device access. */
+size_t tiered_attn_workspace_bytes(const ta_params* p);
+
+/* Router + quantiser ("Triage" abstract: the router predicts from block
+ * statistics; NVFP4 skim / refine copies).  Reads Q, K, V once: block means of
+ * Q, K, V (fp64), the low-precision copies of Q, K, V and their dequantised
+ * bf16 values; then the pooled logits, the n_j-weighted pooled block softmax M,
+ * the tiers by exclusive cumulative mass in (-M, j) order (most precise tier t
+ * with prefix < tau[t], else skip; diagonal blocks forced full when
+ * keep_diag_full), and the per-row tile lists.  Three kernel launches on
+ * `stream`.  ws_dev must hold tiered_attn_workspace_bytes(p) bytes, 256-byte
+ * aligned; its previous contents are overwritten (the status word is reset).
+ * Returns TA_OK when the launches were enqueued. */
+ta_status tiered_attn_plan(const ta_params* p, const void* Q_dev, const void* K_dev,
+                           const void* V_dev, void* ws_dev, size_t ws_bytes, void* stream);
+
+/* Fused tiered attention over a planned workspace ("Triage" abstract: all
+ * tiers in a single pass).  O_dev receives bf16 [B, H, N, d] with the strides of
+ * `p`.  Reads the plan in ws_dev and writes only its status word, so one plan
+ * serves any number of forwards over the same Q, K, V.  One kernel launch. */
+ta_status tiered_attn_forward(const ta_params* p, const void* Q_dev, const void* K_dev,
+                              const void* V_dev, void* ws_dev, size_t ws_bytes,
+                              void* O_dev, void* stream);
+
+/* Whole layer from host memory: copies Q, K, V (host, [B,H,N,d] with the
+ * strides of `p`) into the caller's device buffers, plans, runs the forward and
+ * copies O back to O_host, all enqueued on `stream` (one cudaMemcpyAsync per
+ * tensor).  Does not synchronise: the caller synchronises `stream` before
+ * reading O_host. */
+ta_status tiered_attn_layer_from_host(const ta_params* p, const void* Q_host, const void* K_host,
+                                      const void* V_host, void* O_host, void* Q_dev, void* K_dev,
+                                      void* V_dev, void* O_dev, void* ws_dev, size_t ws_bytes,
+                                      void* stream);
+
+/* Fills `out` with device pointers into ws_dev for workspace layout `p`.  Host
+ * only.  TA_ERR_INVALID_ARG for a null argument or invalid `p`. */
+ta_status tiered_attn_plan_views(const ta_params* p, void* ws_dev, ta_plan_views* out);
+
+/* Synchronises `stream`, reads the status word of ws_dev and returns it
+ * (TA_OK, or the first device-side error such as TA_ERR_TIMEOUT). */
+ta_status tiered_attn_get_status(const void* ws_dev, void* stream);
+
+/* Test entry points: each launches one stage of tiered_attn_plan alone. */
+ta_status tiered_attn_prep(const ta_params* p, const void* Q_dev, const void* K_dev,
+                           const void* V_dev, void* ws_dev, size_t ws_bytes, void* stream);
+ta_status tiered_attn_route(const ta_params* p, void* ws_dev, size_t ws_bytes, void* stream);
+
+/* Static description of a status code. */
+const char* tiered_attn_status_string(ta_status s);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t tiered_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TIERED_ATTN_H */

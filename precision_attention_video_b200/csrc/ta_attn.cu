@@ -1,0 +1,485 @@
+// ta_attn.cu -- the fused one-pass tiered attention kernel (sm_100a).
+//
+// "Triage" (zhuanzhiai paper page, abstract) runs all tiers of a query block
+// in a single fused pass: full tiles in bf16, low tiles in reduced precision,
+// and skipped tiles replaced by their block means, so that block j of n_j keys
+// adds n_j exp(q . kbar_j * scale) to the softmax denominator and that weight
+// times vbar_j to the numerator.  One CTA owns one (head, query block) and
+// walks the block's compacted tile list (full ascending, low ascending, then
+// the skipped blocks) with an online softmax:
+//
+//   warp 4      producer: TMA loads of the kept K / V tiles (bf16, or the
+//               dequantised low copies) into a two-stage ring; for skipped
+//               blocks it gathers up to BK pooled rows kbar_b / vbar_b into a
+//               "pseudo-key" tile, so a skip chunk costs one tile of MMA for
+//               up to BK skipped blocks and never touches their K / V;
+//   warp 5      MMA issuer: tcgen05.mma kind::f16, S = Q K^T into a double-
+//               buffered TMEM accumulator, O += P V into a TMEM accumulator;
+//               completion is signalled with tcgen05.commit on mbarriers;
+//   warps 0-3   softmax: thread r owns TMEM lane r (query row r): loads its S
+//               row, keeps the running max m and sum l, forms
+//               P' = 2^o exp(s - m'), rounds it as the tile's tier demands
+//               (bf16; e4m3; NVFP4 per 16 keys), rescales O in TMEM when m
+//               grows, and writes P' to shared memory as the A operand of PV.
+//               The epilogue writes O = acc / l in bf16.
+//
+// Low tiles run through the same bf16 tensor-core path on the exact bf16
+// values of their dequantised FP8 / NVFP4 operands and of the quantised P'
+// (every FP8 and NVFP4 value is exactly representable in bf16), so the
+// products equal those of the low-precision operands up to fp32 accumulation
+// order.  All waits are bounded: a wait that runs out sets the CTA's abort
+// flag and the workspace status word, every role leaves its loop, in-flight
+// copies and MMAs are drained (bounded), and TMEM is freed before return.
+#include "ta_common.cuh"
+#include "ta_kernels.cuh"
+
+namespace ta {
+namespace {
+
+constexpr int kThreads = 192;  // 4 softmax warps + producer + MMA
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+
+enum TileKind { KIND_FULL = 0, KIND_LOW = 1, KIND_SKIP = 2 };
+
+struct RowPlan {
+  int n_full, n_res, n_low, n_skip;
+  int T;             // number of tiles (skip blocks chunked by BK)
+  const int* list;   // this row's list
+};
+
+template <int BK>
+__device__ __forceinline__ void tile_of(const RowPlan& rp, int t, int& kind, int& first) {
+  if (t < rp.n_full) {
+    kind = KIND_FULL;
+    first = t;
+  } else if (t < rp.n_full + rp.n_low) {
+    kind = KIND_LOW;
+    first = rp.n_full + rp.n_res + (t - rp.n_full);
+  } else {
+    kind = KIND_SKIP;
+    first = rp.n_full + rp.n_res + rp.n_low + (t - rp.n_full - rp.n_low) * BK;
+  }
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Shared-memory layout (offsets from a 1024-aligned base).
+template <int D, int BK>
+struct Smem {
+  static constexpr int kQ = 128 * D * 2;      // one query tile, 128 rows
+  static constexpr int kKV = BK * D * 2;      // one K or V tile
+  static constexpr int kP = 128 * BK * 2;     // P tile
+  static constexpr int oQ = 0;
+  static constexpr int oDQ = oQ + kQ;
+  static constexpr int oK0 = oDQ + kQ;
+  static constexpr int oV0 = oK0 + kKV;
+  static constexpr int oK1 = oV0 + kKV;
+  static constexpr int oV1 = oK1 + kKV;
+  static constexpr int oP = oV1 + kKV;
+  static constexpr int oBar = oP + kP;
+  static constexpr int kBars = 16;
+  static constexpr int oMisc = oBar + kBars * 8;
+  static constexpr int kTotal = oMisc + 64;
+  static constexpr int kAlloc = kTotal + 1024;  // alignment slack
+  static constexpr uint32_t kTmemCols = (2 * BK + D) <= 256 ? 256u : 512u;
+};
+
+enum {
+  BAR_Q = 0, BAR_K0 = 1, BAR_K1 = 2, BAR_V0 = 3, BAR_V1 = 4, BAR_E0 = 5, BAR_E1 = 6,
+  BAR_S0 = 7, BAR_S1 = 8, BAR_P = 9, BAR_O = 10, BAR_DRAIN = 11
+};
+
+template <int D, int BK>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmQ,
+                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
+                const __grid_constant__ CUtensorMap tmDV) {
+  using L = Smem<D, BK>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::oBar);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oMisc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::oMisc + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int qb = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int q0 = qb * a.bq;
+  const int64_t row_id = (int64_t)bh * a.nQb + qb;
+
+  RowPlan rp;
+  rp.n_full = a.row_counts[row_id * 4 + 0];
+  rp.n_res = a.row_counts[row_id * 4 + 1];
+  rp.n_low = a.row_counts[row_id * 4 + 2];
+  rp.n_skip = a.row_counts[row_id * 4 + 3];
+  rp.list = a.row_lists + row_id * a.nKb;
+  rp.T = rp.n_full + rp.n_low + (rp.n_skip + BK - 1) / BK;
+  const bool has_low = rp.n_low > 0;
+
+  AbortCtx ctx{abort_flag, a.status};
+
+  // ---- set-up: barriers, zero padding rows, TMEM ----
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(&bars[BAR_Q], 1);
+    mbar_init(&bars[BAR_K0], 1);
+    mbar_init(&bars[BAR_K1], 1);
+    mbar_init(&bars[BAR_V0], 1);
+    mbar_init(&bars[BAR_V1], 1);
+    mbar_init(&bars[BAR_E0], 1);
+    mbar_init(&bars[BAR_E1], 1);
+    mbar_init(&bars[BAR_S0], 1);
+    mbar_init(&bars[BAR_S1], 1);
+    mbar_init(&bars[BAR_P], a.bq);
+    mbar_init(&bars[BAR_O], 1);
+    mbar_init(&bars[BAR_DRAIN], 1);
+    fence_mbar_init();
+  }
+  if (warp < 4) {
+    // Rows >= bq of the query tiles and of P stay zero for the whole kernel.
+    const int r = threadIdx.x;
+    if (r >= a.bq) {
+      for (int c = 0; c < (D * 2) / 16; ++c) {
+        const int box = c / 8, ch = c % 8;
+        const uint32_t off = box * (128 * 128) + r * 128 + ((ch ^ (r & 7)) * 16);
+        *reinterpret_cast<uint4*>(sm + L::oQ + off) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sm + L::oDQ + off) = make_uint4(0, 0, 0, 0);
+      }
+      for (int c = 0; c < (BK * 2) / 16; ++c) {
+        const int box = c / 8, ch = c % 8;
+        const uint32_t off = box * (128 * 128) + r * 128 + ((ch ^ (r & 7)) * 16);
+        *reinterpret_cast<uint4*>(sm + L::oP + off) = make_uint4(0, 0, 0, 0);
+      }
+      fence_proxy_async_smem();
+    }
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS0 = tmem, tS1 = tmem + BK, tO = tmem + 2 * BK;
+
+  bool aborted = false;
+
+  if (warp == kProducerWarp) {
+    // ===================== producer =====================
+    int kf_issued[2] = {0, 0}, vf_issued[2] = {0, 0};
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const uint32_t qbytes = (uint32_t)a.bq * D * 2;
+      mbar_arrive_expect_tx(&bars[BAR_Q], has_low ? 2 * qbytes : qbytes);
+      for (int x = 0; x < D / 64; ++x) {
+        tma_load_4d(sm + L::oQ + x * (128 * 128), &tmQ, &bars[BAR_Q], x * 64, q0, h, b);
+        if (has_low)
+          tma_load_4d(sm + L::oDQ + x * (128 * 128), &tmDQ, &bars[BAR_Q], x * 64, q0, h, b);
+      }
+    }
+    const __nv_bfloat16* kbar = a.kbar_b + (int64_t)bh * a.nKb * D;
+    const __nv_bfloat16* vbar = a.vbar_b + (int64_t)bh * a.nKb * D;
+    for (int t = 0; t < rp.T; ++t) {
+      const int s = t & 1;
+      if (t >= 2) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&bars[BAR_E0 + s], ((t >> 1) - 1) & 1, ctx, 1);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { aborted = true; break; }
+      }
+      int kind, first;
+      tile_of<BK>(rp, t, kind, first);
+      unsigned char* kst = sm + (s ? L::oK1 : L::oK0);
+      unsigned char* vst = sm + (s ? L::oV1 : L::oV0);
+      if (kind != KIND_SKIP) {
+        if (lane == 0) {
+          const int j = rp.list[first];
+          const CUtensorMap* mk = (kind == KIND_LOW) ? &tmDK : &tmK;
+          const CUtensorMap* mv = (kind == KIND_LOW) ? &tmDV : &tmV;
+          const bool drop = (t == 0) && (a.debug_flags & TA_DEBUG_DROP_FIRST_K);
+          if (!drop) {
+            mbar_arrive_expect_tx(&bars[BAR_K0 + s], BK * D * 2);
+            for (int x = 0; x < D / 64; ++x)
+              tma_load_4d(kst + x * (BK * 128), mk, &bars[BAR_K0 + s], x * 64, j * BK, h, b);
+            kf_issued[s]++;
+          }
+          mbar_arrive_expect_tx(&bars[BAR_V0 + s], BK * D * 2);
+          for (int x = 0; x < D / 64; ++x)
+            tma_load_4d(vst + x * (BK * 128), mv, &bars[BAR_V0 + s], x * 64, j * BK, h, b);
+          vf_issued[s]++;
+        }
+      } else {
+        // gather pooled rows of the skipped blocks into a pseudo K / V tile
+        const int cnt = min(BK, rp.n_skip - (first - rp.n_full - rp.n_res - rp.n_low));
+        for (int e = lane; e < BK * (D / 8); e += 32) {
+          const int c = e / (D / 8), ch = e % (D / 8);
+          uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+          if (c < cnt) {
+            const int j = rp.list[first + c];
+            kv = *reinterpret_cast<const uint4*>(kbar + (int64_t)j * D + ch * 8);
+            vv = *reinterpret_cast<const uint4*>(vbar + (int64_t)j * D + ch * 8);
+          }
+          const uint32_t off = (ch >> 3) * (BK * 128) + c * 128 + (((ch & 7) ^ (c & 7)) * 16);
+          *reinterpret_cast<uint4*>(kst + off) = kv;
+          *reinterpret_cast<uint4*>(vst + off) = vv;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bars[BAR_K0 + s]);
+          mbar_arrive(&bars[BAR_V0 + s]);
+          kf_issued[s]++;
+          vf_issued[s]++;
+        }
+      }
+    }
+    if (aborted && lane == 0) {
+      // let copies already in flight land before the CTA goes away
+      for (int s = 0; s < 2; ++s) {
+        if (kf_issued[s] > 0) mbar_wait_drain(&bars[BAR_K0 + s], (kf_issued[s] - 1) & 1);
+        if (vf_issued[s] > 0) mbar_wait_drain(&bars[BAR_V0 + s], (vf_issued[s] - 1) & 1);
+      }
+      mbar_wait_drain(&bars[BAR_Q], 0);
+    }
+  } else if (warp == kMmaWarp) {
+    // ===================== MMA issuer =====================
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16(128, BK, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, D, true);
+      const uint32_t sQ = smem_u32(sm + L::oQ), sDQ = smem_u32(sm + L::oDQ);
+      const uint32_t sP = smem_u32(sm + L::oP);
+      auto issue_s = [&](int t) -> bool {
+        const int s = t & 1;
+        if (!mbar_wait(&bars[BAR_K0 + s], (t >> 1) & 1, ctx, 2)) return false;
+        tc_fence_after();
+        int kind, first;
+        tile_of<BK>(rp, t, kind, first);
+        const uint32_t aq = (kind == KIND_LOW) ? sDQ : sQ;
+        const uint32_t sk = smem_u32(sm + (s ? L::oK1 : L::oK0));
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(aq + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sk + (kk >> 2) * (BK * 128) + (kk & 3) * 32, 16, 1024);
+          mma_f16_ss(s ? tS1 : tS0, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bars[BAR_S0 + s]);
+        return true;
+      };
+      bool ok = mbar_wait(&bars[BAR_Q], 0, ctx, 3);
+      if (ok) {
+        tc_fence_after();
+        ok = issue_s(0);
+      }
+      for (int t = 0; ok && t < rp.T; ++t) {
+        const int s = t & 1;
+        if (t + 1 < rp.T && !issue_s(t + 1)) { ok = false; break; }
+        if (!mbar_wait(&bars[BAR_P], t & 1, ctx, 4)) { ok = false; break; }
+        if (!mbar_wait(&bars[BAR_V0 + s], (t >> 1) & 1, ctx, 5)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sv = smem_u32(sm + (s ? L::oV1 : L::oV0));
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(sP + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sv + kk * 16 * 128, BK * 128, 1024);
+          mma_f16_ss(tO, ad, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&bars[BAR_O]);
+        tc_commit(&bars[BAR_E0 + s]);
+      }
+      if (!ok) {
+        aborted = true;
+        tc_commit(&bars[BAR_DRAIN]);
+        mbar_wait_drain(&bars[BAR_DRAIN], 0);
+      }
+    }
+  } else if (threadIdx.x < a.bq) {
+    // ===================== softmax warps =====================
+    const int r = threadIdx.x;  // query row within the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const float o_off = (float)a.p_offset;
+    float m = -INFINITY, l = 0.0f;
+    for (int t = 0; t < rp.T; ++t) {
+      const int s = t & 1;
+      bool ok = mbar_wait(&bars[BAR_S0 + s], (t >> 1) & 1, ctx, 6);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) { aborted = true; break; }
+      tc_fence_after();
+      int kind, first;
+      tile_of<BK>(rp, t, kind, first);
+      int nvalid;
+      if (kind == KIND_SKIP) {
+        nvalid = min(BK, rp.n_skip - (first - rp.n_full - rp.n_res - rp.n_low));
+      } else {
+        nvalid = min(BK, a.N - rp.list[first] * BK);
+      }
+      float x[BK];
+#pragma unroll
+      for (int c0 = 0; c0 < BK; c0 += 32) {
+        uint32_t raw[32];
+        tmem_ld32((s ? tS1 : tS0) + lane_off + c0, raw);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[c0 + c] = __uint_as_float(raw[c]) * a.scale_log2;
+      }
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BK; ++c) {
+        if (c >= nvalid) x[c] = -INFINITY;
+        tmax = fmaxf(tmax, x[c]);
+      }
+      const float m_new = fmaxf(m, tmax);
+      const float alpha = fast_exp2(m - m_new);  // 0 on the first tile
+      float rowsum = 0.0f;
+#pragma unroll
+      for (int c = 0; c < BK; ++c) {
+        x[c] = fast_exp2(x[c] - m_new + o_off);
+      }
+      if (kind == KIND_SKIP) {
+#pragma unroll
+        for (int c = 0; c < BK; ++c) {
+          if (c < nvalid) {
+            const int j = rp.list[first + c];
+            x[c] *= (float)min(BK, a.N - j * BK);
+          }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < BK; ++c) rowsum += x[c];
+      l = l * alpha + rowsum;
+      m = m_new;
+
+      // round P' as the tier demands, into bf16 pairs
+      uint32_t p[BK / 2];
+      if (kind == KIND_LOW && a.low == TA_LOW_FP8_E4M3) {
+#pragma unroll
+        for (int c = 0; c < BK; c += 2) {
+          const float2 f = e4m3x2_to_float2(cvt_e4m3x2(x[c], x[c + 1]));
+          p[c / 2] = pack_bf16(f.x, f.y);
+        }
+      } else if (kind == KIND_LOW) {
+#pragma unroll
+        for (int g = 0; g < BK; g += 16) {
+          float amax = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) amax = fmaxf(amax, x[g + i]);
+          const uint32_t scc = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xFFu;
+          const float sc = e4m3_to_float(scc);
+          const float inv = (sc > 0.0f) ? __frcp_rn(sc) : 0.0f;
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            const uint32_t cc = cvt_e2m1x2(__fmul_rn(x[g + i], inv), __fmul_rn(x[g + i + 1], inv));
+            p[(g + i) / 2] = pack_bf16(e2m1_value(cc & 0xFu) * sc, e2m1_value(cc >> 4) * sc);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < BK; c += 2) p[c / 2] = pack_bf16(x[c], x[c + 1]);
+      }
+
+      // PV of the previous tile must be done before P and O are touched
+      if (t > 0) {
+        bool ok2 = mbar_wait(&bars[BAR_O], (t - 1) & 1, ctx, 7);
+        ok2 = __all_sync(0xffffffffu, ok2);
+        if (!ok2) { aborted = true; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t raw[32];
+            tmem_ld32(tO + lane_off + c0, raw);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * alpha);
+            tmem_st32(tO + lane_off + c0, raw);
+          }
+          tmem_wait_st();
+        }
+      }
+      // P row -> shared memory, K-major, 128-byte swizzle
+#pragma unroll
+      for (int ch = 0; ch < BK / 8; ++ch) {
+        const uint32_t off = (ch >> 3) * (128 * 128) + r * 128 + (((ch & 7) ^ (r & 7)) * 16);
+        *reinterpret_cast<uint4*>(sm + L::oP + off) =
+            make_uint4(p[ch * 4 + 0], p[ch * 4 + 1], p[ch * 4 + 2], p[ch * 4 + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars[BAR_P]);
+    }
+    if (!aborted) {
+      bool ok = mbar_wait(&bars[BAR_O], (rp.T - 1) & 1, ctx, 8);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.0f / l;
+        const bool valid = (q0 + r) < a.N;
+        __nv_bfloat16* orow = a.O + (int64_t)b * a.sb + (int64_t)h * a.sh + (int64_t)(q0 + r) * a.sn;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t raw[32];
+          tmem_ld32(tO + lane_off + c0, raw);
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2)
+            w[c / 2] = pack_bf16(__uint_as_float(raw[c]) * inv_l, __uint_as_float(raw[c + 1]) * inv_l);
+          if (valid) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              *reinterpret_cast<uint4*>(orow + c0 + v * 8) =
+                  make_uint4(w[v * 4 + 0], w[v * 4 + 1], w[v * 4 + 2], w[v * 4 + 3]);
+          }
+        }
+      } else {
+        aborted = true;
+      }
+    }
+  }
+
+  // ---- teardown ----
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, L::kTmemCols);
+}
+
+template <int D, int BK>
+cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
+  using L = Smem<D, BK>;
+  auto k = attn_kernel<D, BK>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.nQb, a.B * a.H);
+  k<<<grid, kThreads, L::kAlloc, s>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5]);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int attn_smem_bytes(int d, int bk) {
+  if (d == 64 && bk == 64) return Smem<64, 64>::kAlloc;
+  if (d == 64 && bk == 128) return Smem<64, 128>::kAlloc;
+  if (d == 128 && bk == 64) return Smem<128, 64>::kAlloc;
+  return Smem<128, 128>::kAlloc;
+}
+
+cudaError_t launch_attn(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
+  if (a.d == 64 && a.bk == 64) return launch_d<64, 64>(a, maps, s);
+  if (a.d == 64 && a.bk == 128) return launch_d<64, 128>(a, maps, s);
+  if (a.d == 128 && a.bk == 64) return launch_d<128, 64>(a, maps, s);
+  return launch_d<128, 128>(a, maps, s);
+}
+
+}  // namespace ta

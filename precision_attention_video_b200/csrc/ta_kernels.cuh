@@ -1,0 +1,66 @@
+// ta_kernels.cuh -- argument blocks and launchers of the tiered-attention
+// kernels (router / quantiser / fused attention), shared by the C ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tiered_attn.h"
+
+namespace ta {
+
+// Everything the plan stage reads and writes (device pointers into the
+// workspace; null where the low format does not produce the array).
+struct PlanArgs {
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  int64_t sb, sh, sn;           // element strides of Q, K, V
+  int B, H, N, d, bq, bk, low;  // shape, tiles, ta_low_format
+  int R;                        // rows per prep chunk = max(bq, bk)
+  int nQb, nKb, Np;             // ceil(N/bq), ceil(N/bk), 16*ceil(N/16)
+  int n_tau;
+  double tau[3];
+  int keep_diag;
+  double scale;                 // softmax scale (fp64 in the router)
+  int* status;
+  double* qbar;
+  double* kbar;
+  __nv_bfloat16* kbar_b;
+  __nv_bfloat16* vbar_b;
+  int* n_k;
+  double* logits;
+  double* mass;
+  uint8_t* tier_map;
+  int* row_counts;
+  int* row_lists;
+  uint8_t *q_codes, *k_codes, *v_codes;
+  void *q_scales, *k_scales, *v_scales;
+  uint8_t *rq_codes, *rk_codes, *rv_codes;
+  uint8_t *rq_scales, *rk_scales, *rv_scales;
+  __nv_bfloat16 *dq, *dk, *dv, *drq, *drk, *drv;
+};
+
+// Fused attention arguments.
+struct AttnArgs {
+  int B, H, N, d, bq, bk, low;
+  int nQb, nKb;
+  int64_t sb, sh, sn;           // element strides of O
+  float scale_log2;             // softmax_scale * log2(e)
+  int p_offset;                 // o of P' = 2^o exp(s - m)
+  int debug_flags;
+  int* status;
+  const __nv_bfloat16* kbar_b;  // skip pseudo-keys [BH, nKb, d]
+  const __nv_bfloat16* vbar_b;
+  const int* row_counts;
+  const int* row_lists;
+  __nv_bfloat16* O;
+};
+
+cudaError_t launch_prep(const PlanArgs& a, cudaStream_t s);
+cudaError_t launch_route(const PlanArgs& a, cudaStream_t s);
+cudaError_t launch_attn(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s);
+
+}  // namespace ta

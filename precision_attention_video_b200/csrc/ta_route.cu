@@ -1,0 +1,223 @@
+// ta_route.cu -- the router: pooled block logits, pooled block softmax,
+// cumulative-mass tiers and compacted per-row tile lists.
+//
+// "Triage" (zhuanzhiai paper page, abstract) predicts each tile's treatment
+// from block statistics; "HierPAS" (conference listing, abstract) estimates the
+// attention pattern cheaply and keeps precision where the mass is; "APT"
+// (Lattice paper summary, APDT) turns attention probability into selection and
+// precision with two thresholds.  Per head and query block i:
+//   sbar_ij = (qbar_i . kbar_j) * scale,
+//   M_ij    = n_j exp(sbar_ij - max_j sbar_ij) / sum_j (.),
+//   sort j by (-M_ij, j); C_r = exclusive prefix sum of the sorted masses;
+//   tier(rank r) = the most precise tier t with C_r < tau_t, else skip;
+//   key blocks meeting query block i's token range become full;
+//   list = full blocks ascending, then residual, low, skip (each ascending).
+// The router runs in fp64 end to end (means, logits, exp, prefix), so its
+// cumulative masses agree with an fp64 evaluation to ~1e-15 relative and the
+// tier map only depends on the ordering rule, not on rounding.
+#include "ta_common.cuh"
+#include "ta_kernels.cuh"
+
+namespace ta {
+namespace {
+
+// ---------------------------------------------------------------------------
+// Pooled logits: logits[bh, i, j] = scale * sum_c qbar[bh, i, c] kbar[bh, j, c]
+// 32 x 32 output tile per CTA, 2 x 2 per thread, d staged 32 at a time.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) logits_kernel(const PlanArgs a) {
+  __shared__ double qs[32][33];
+  __shared__ double ks[32][33];
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  const int bh = blockIdx.z, i0 = blockIdx.x * 32, j0 = blockIdx.y * 32;
+  const int D = a.d;
+  const double* qb = a.qbar + (int64_t)bh * a.nQb * D;
+  const double* kb = a.kbar + (int64_t)bh * a.nKb * D;
+  double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    for (int e = tid; e < 32 * 32; e += 256) {
+      const int r = e / 32, c = e % 32;
+      qs[r][c] = (i0 + r < a.nQb) ? qb[(int64_t)(i0 + r) * D + c0 + c] : 0.0;
+      ks[r][c] = (j0 + r < a.nKb) ? kb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < 32; ++c) {
+      const double q0 = qs[ty * 2][c], q1 = qs[ty * 2 + 1][c];
+      const double k0 = ks[tx * 2][c], k1 = ks[tx * 2 + 1][c];
+      acc[0][0] += q0 * k0;
+      acc[0][1] += q0 * k1;
+      acc[1][0] += q1 * k0;
+      acc[1][1] += q1 * k1;
+    }
+    __syncthreads();
+  }
+  for (int u = 0; u < 2; ++u)
+    for (int v = 0; v < 2; ++v) {
+      const int i = i0 + ty * 2 + u, j = j0 + tx * 2 + v;
+      if (i < a.nQb && j < a.nKb) a.logits[((int64_t)bh * a.nQb + i) * a.nKb + j] = acc[u][v] * a.scale;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Per-row routing, one warp per (bh, query block).
+// ---------------------------------------------------------------------------
+constexpr int kRouteWarps = 8;
+
+__device__ __forceinline__ bool before(double ka, int ia, double kb, int ib) {
+  return (ka > kb) || (ka == kb && ia < ib);
+}
+
+__device__ __forceinline__ double warp_max(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs a, int sortn) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  double* key = reinterpret_cast<double*>(smem_raw) + (size_t)warp * sortn;
+  int* idx = reinterpret_cast<int*>(reinterpret_cast<double*>(smem_raw) + (size_t)kRouteWarps * sortn) +
+             (size_t)warp * sortn;
+  uint8_t* tier = reinterpret_cast<uint8_t*>(reinterpret_cast<int*>(reinterpret_cast<double*>(smem_raw) +
+                                                                    (size_t)kRouteWarps * sortn) +
+                                             (size_t)kRouteWarps * sortn) +
+                  (size_t)warp * sortn;
+
+  const int64_t g = (int64_t)blockIdx.x * kRouteWarps + warp;  // global row
+  const int64_t nrows = (int64_t)a.B * a.H * a.nQb;
+  if (g >= nrows) return;
+  const int i = (int)(g % a.nQb);
+  const int nKb = a.nKb;
+  const double* lrow = a.logits + g * nKb;
+
+  // pooled block softmax weighted by key counts
+  double mx = -INFINITY;
+  for (int j = lane; j < nKb; j += 32) mx = fmax(mx, lrow[j]);
+  mx = warp_max(mx);
+  double part = 0.0;
+  for (int j = lane; j < nKb; j += 32) {
+    const int nj = min(a.bk, a.N - j * a.bk);
+    const double w = (double)nj * exp(lrow[j] - mx);
+    key[j] = w;
+    part += w;
+  }
+  const double total = warp_sum(part);
+  for (int j = lane; j < sortn; j += 32) {
+    if (j < nKb) {
+      const double m = key[j] / total;
+      key[j] = m;
+      idx[j] = j;
+      a.mass[g * nKb + j] = m;
+    } else {
+      key[j] = -1.0;
+      idx[j] = 0x7fffffff - (sortn - j);
+    }
+  }
+  __syncwarp();
+
+  // bitonic sort into (-M, j) order
+  for (int k = 2; k <= sortn; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int t = lane; t < sortn; t += 32) {
+        const int u = t ^ jj;
+        if (u > t) {
+          const double kt = key[t], ku = key[u];
+          const int it = idx[t], iu = idx[u];
+          const bool up = (t & k) == 0;
+          const bool sw = up ? before(ku, iu, kt, it) : before(kt, it, ku, iu);
+          if (sw) {
+            key[t] = ku;
+            key[u] = kt;
+            idx[t] = iu;
+            idx[u] = it;
+          }
+        }
+      }
+      __syncwarp();
+    }
+  }
+
+  // exclusive prefix of the sorted masses, then tiers by rank
+  const int per = sortn / 32;
+  double lsum = 0.0;
+  for (int r = lane * per; r < (lane + 1) * per; ++r) lsum += fmax(key[r], 0.0);
+  double incl = lsum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  double C = incl - lsum;
+  int codes[3];
+  if (a.n_tau == 1) {
+    codes[0] = TA_TIER_FULL;
+  } else if (a.n_tau == 2) {
+    codes[0] = TA_TIER_FULL;
+    codes[1] = TA_TIER_LOW;
+  } else {
+    codes[0] = TA_TIER_FULL;
+    codes[1] = TA_TIER_RES;
+    codes[2] = TA_TIER_LOW;
+  }
+  for (int r = lane * per; r < (lane + 1) * per; ++r) {
+    const int j = idx[r];
+    if (j < nKb) {
+      int t = TA_TIER_SKIP;
+      for (int q = a.n_tau - 1; q >= 0; --q)
+        if (C < a.tau[q]) t = codes[q];
+      tier[j] = (uint8_t)t;
+    }
+    C += fmax(key[r], 0.0);
+  }
+  __syncwarp();
+  if (a.keep_diag && lane == 0) {
+    const int r0 = i * a.bq, r1 = min(a.N, (i + 1) * a.bq);
+    for (int j = r0 / a.bk; j <= (r1 - 1) / a.bk; ++j) tier[j] = TA_TIER_FULL;
+  }
+  __syncwarp();
+
+  // tier map row, counts and the compacted list
+  for (int j = lane; j < nKb; j += 32) a.tier_map[g * nKb + j] = tier[j];
+  const int order[4] = {TA_TIER_FULL, TA_TIER_RES, TA_TIER_LOW, TA_TIER_SKIP};
+  int base = 0;
+  for (int q = 0; q < 4; ++q) {
+    const int t = order[q];
+    int cnt = 0;
+    for (int j0 = 0; j0 < nKb; j0 += 32) {
+      const int j = j0 + lane;
+      const bool p = (j < nKb) && tier[j] == t;
+      const unsigned bal = __ballot_sync(0xffffffffu, p);
+      if (p) a.row_lists[g * nKb + base + cnt + __popc(bal & ((1u << lane) - 1u))] = j;
+      cnt += __popc(bal);
+    }
+    if (lane == 0) a.row_counts[g * 4 + q] = cnt;
+    base += cnt;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_route(const PlanArgs& a, cudaStream_t s) {
+  dim3 g1((a.nQb + 31) / 32, (a.nKb + 31) / 32, a.B * a.H);
+  logits_kernel<<<g1, 256, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  int sortn = 32;
+  while (sortn < a.nKb) sortn <<= 1;
+  const size_t smem = (size_t)kRouteWarps * sortn * (sizeof(double) + sizeof(int) + 1);
+  e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t rows = (int64_t)a.B * a.H * a.nQb;
+  dim3 g2((unsigned)((rows + kRouteWarps - 1) / kRouteWarps));
+  route_kernel<<<g2, kRouteWarps * 32, smem, s>>>(a, sortn);
+  return cudaGetLastError();
+}
+
+}  // namespace ta

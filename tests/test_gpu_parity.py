@@ -1,0 +1,137 @@
+"""GPU parity: the CUDA path through the C ABI against the oracle.
+
+Plan stage: block means (fp64) and their bf16 copies bit-exact; FP8 / NVFP4
+(+residual) codes, scales and dequantised values bit-exact; pooled logits and
+masses to fp64 rounding; the tier map bit-exact except on oracle-flagged tiles;
+the row lists consistent with the tier map.  Forward: O within rel-L2 1e-2 and
+max-abs 2e-2 of the oracle run on the same inputs with the same rounding rules
+(rows whose tier map matches the oracle's).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import (assert_out_close, check_lists, compare_tiers, inputs, oracle_head,
+                         run_gpu, to64, unpack_fp4)
+from oracle import quant as Qz
+
+pytestmark = pytest.mark.gpu
+
+
+def _plan_parity(cfg, Q, K, V, views, heads):
+    nkb = cfg.n_kb
+    n_k = views["n_k"].numpy()
+    np.testing.assert_array_equal(n_k, [min(cfg.block_k, cfg.N - j * cfg.block_k) for j in range(nkb)])
+    for (b, h) in heads:
+        bh = b * cfg.H + h
+        rt, qt, _ = oracle_head(cfg, Q, K, V, b, h, qblocks=[])
+        np.testing.assert_array_equal(views["qbar"][bh].numpy(), rt["qbar"])
+        np.testing.assert_array_equal(views["kbar"][bh].numpy(), rt["kbar"])
+        np.testing.assert_array_equal(to64(views["kbar_b"][bh]), rt["kbar_b"])
+        np.testing.assert_array_equal(to64(views["vbar_b"][bh]), rt["vbar_b"])
+        np.testing.assert_allclose(views["logits"][bh].numpy(), (rt["qbar"] @ rt["kbar"].T) * rt["scale"],
+                                   rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(views["mass"][bh].numpy(), rt["M"], rtol=1e-10, atol=1e-15)
+        tiers = views["tier_map"][bh].numpy()
+        compare_tiers(tiers, rt)
+        check_lists(tiers, views["row_counts"][bh].numpy(), views["row_lists"][bh].numpy())
+        if cfg.low == Qz.LOW_FP8:
+            for t in "qkv":
+                np.testing.assert_array_equal(views[f"{t}_codes"][bh].numpy(), qt[f"{t}_codes"])
+                np.testing.assert_array_equal(views[f"{t}_scales"][bh].numpy().astype(np.float64), qt[f"{t}_scale"])
+                np.testing.assert_array_equal(to64(views[f"d{t}"][bh]), qt[f"d{t}"][:cfg.N])
+        elif cfg.low in (Qz.LOW_NVFP4, Qz.LOW_NVFP4_RES):
+            pres = ["", "r"] if cfg.low == Qz.LOW_NVFP4_RES else [""]
+            for pre in pres:
+                for t in "qk":
+                    np.testing.assert_array_equal(unpack_fp4(views[f"{pre}{t}_codes"][bh].numpy()),
+                                                  qt[f"{pre}{t}_codes"])
+                    np.testing.assert_array_equal(views[f"{pre}{t}_scales"][bh].numpy(), qt[f"{pre}{t}_sc"])
+                vt = unpack_fp4(views[f"{pre}v_codes"][bh].numpy()).T
+                np.testing.assert_array_equal(vt, qt[f"{pre}v_codes"])
+                np.testing.assert_array_equal(views[f"{pre}v_scales"][bh].numpy(), qt[f"{pre}v_sc"])
+            for t in "qkv":
+                np.testing.assert_array_equal(to64(views[f"d{t}"][bh]), qt[f"d{t}"][:cfg.N])
+            if cfg.low == Qz.LOW_NVFP4_RES:
+                for t, key in (("q", "rq"), ("k", "rk"), ("v", "rv")):
+                    np.testing.assert_array_equal(to64(views[f"dr{t}"][bh]), qt[key][:cfg.N])
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_plan_parity_fp8(cuda_ok, name):
+    cfg, Q, K, V = inputs(name)
+    _, views, _, st = run_gpu(cfg, Q, K, V, forward=False)
+    assert st == 0
+    heads = [(0, h) for h in range(cfg.H)]
+    _plan_parity(cfg, Q, K, V, views, heads)
+
+
+def test_plan_parity_nvfp4_ragged(cuda_ok):
+    # 480p tile / format settings on a smaller ragged grid (N = 3*10*21 = 630 = 4*128 + 118)
+    cfg, Q, K, V = inputs("480p", grid=(3, 10, 21), H=3)
+    _, views, _, st = run_gpu(cfg, Q, K, V, forward=False)
+    assert st == 0
+    _plan_parity(cfg, Q, K, V, views, [(0, h) for h in range(cfg.H)])
+
+
+def test_plan_parity_nvfp4_residual_ragged(cuda_ok):
+    cfg, Q, K, V = inputs("720p", grid=(3, 9, 20), H=2)   # N = 540 = 4*128 + 28
+    _, views, _, st = run_gpu(cfg, Q, K, V, forward=False)
+    assert st == 0
+    _plan_parity(cfg, Q, K, V, views, [(0, h) for h in range(cfg.H)])
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_forward_parity_fp8(cuda_ok, name):
+    cfg, Q, K, V = inputs(name)
+    _, views, O, st = run_gpu(cfg, Q, K, V)
+    assert st == 0
+    heads = [(0, h) for h in range(cfg.H)] if cfg.H <= 2 else [(0, 0), (0, cfg.H // 2), (0, cfg.H - 1)]
+    for (b, h) in heads:
+        bh = b * cfg.H + h
+        rt, qt, Oref = oracle_head(cfg, Q, K, V, b, h)
+        _, rows = compare_tiers(views["tier_map"][bh].numpy(), rt)
+        Og = to64(O[b, h])
+        for i in rows:  # a flagged tile differs: compare only rows routed alike
+            Oref[i * cfg.block_q:(i + 1) * cfg.block_q] = np.nan
+        assert_out_close(Og, Oref, f"{name} head {h}")
+
+
+def test_forward_parity_nvfp4_ragged(cuda_ok):
+    cfg, Q, K, V = inputs("480p", grid=(3, 10, 21), H=3)
+    _, views, O, st = run_gpu(cfg, Q, K, V)
+    assert st == 0
+    for h in range(cfg.H):
+        rt, qt, Oref = oracle_head(cfg, Q, K, V, 0, h)
+        _, rows = compare_tiers(views["tier_map"][h].numpy(), rt)
+        for i in rows:
+            Oref[i * cfg.block_q:(i + 1) * cfg.block_q] = np.nan
+        assert_out_close(to64(O[0, h]), Oref, f"nvfp4 head {h}")
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_all_full_matches_oracle_and_sdpa(cuda_ok, name):
+    cfg, Q, K, V = inputs(name)
+    _, views, O, st = run_gpu(cfg, Q, K, V, tau=(2.0, 2.0))
+    assert st == 0
+    assert (views["tier_map"].numpy() == 3).all()
+    for h in range(min(cfg.H, 2)):
+        _, _, Oref = oracle_head(cfg, Q, K, V, 0, h, tau=(2.0, 2.0))
+        assert_out_close(to64(O[0, h]), Oref, f"all-full head {h}")
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q.cuda().float(), K.cuda().float(), V.cuda().float()).cpu()
+    rel = (O.float() - ref).norm() / ref.norm()
+    assert rel < 1e-2
+
+
+def test_skip_only_rows(cuda_ok):
+    # thresholds 0: only the diagonal stays (full), every other tile is a skip
+    cfg, Q, K, V = inputs("tiny")
+    _, views, O, st = run_gpu(cfg, Q, K, V, tau=(0.0, 0.0))
+    assert st == 0
+    t = views["tier_map"].numpy()
+    assert ((t == 3) | (t == 0)).all() and (t == 0).any()
+    for h in range(cfg.H):
+        rt, _, Oref = oracle_head(cfg, Q, K, V, 0, h, tau=(0.0, 0.0))
+        assert_out_close(to64(O[0, h]), Oref, f"skip-only head {h}")
