@@ -1,0 +1,370 @@
+"""Benchmark of the tiered-precision video-DiT attention layer on B200.
+
+One step = one full attention layer of the 480p-video-like workload
+(B=1, H=40, N=32760 tokens from a 21x30x52 latent grid, d=128, 128x128 tiles,
+NVFP4 low tier, cumulative-mass thresholds 0.6 / 0.9): tiered_attn_plan
+(pooling, quantisation, routing) followed by tiered_attn_forward, on inputs
+already resident in HBM.  The metric is dense-equivalent attention TFLOPS,
+4*B*H*N^2*d / (plan + forward time); ms per layer and the attention kernel's
+fraction of tensor-pipe peak for the FLOPs it executes are reported beside it.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With --gpus N > 1 (launched by torchrun) each rank runs an independent
+replica of the layer on its own GPU (the heads of a layer need no exchange);
+`value` is the work of all ranks divided by the slowest rank's time.
+--impl reference times the CPU oracle (fp64, software FP8/NVFP4 rounding) on
+the host cores on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from latent_gen import get_config, make_qkv  # noqa: E402
+
+WORKLOAD = "480p"
+METRIC = "dense-equiv attention TFLOPS & ms/layer @32760 tok; % tensor-pipe peak"
+UNIT = "TFLOPS"
+L2_BYTES = 126 * 2 ** 20
+
+# DRAM traffic of one tiered_attn_forward launch on this workload, from the ncu
+# capture summarised in profiles/ (dram__bytes_read.sum + dram__bytes_write.sum);
+# valid only for the kernel source it was measured on.
+ATTN_TRAFFIC = {"source_sha1": None, "bytes_per_launch": None}
+
+
+def _env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def attn_source_sha1():
+    p = os.path.join(ROOT, "precision_attention_video_b200", "csrc", "ta_attn.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def algorithmic_attn_flops(cfg, counts: np.ndarray, lists: np.ndarray):
+    """FLOPs the tiered forward is defined to execute: 4*|q_i|*|k_j|*d per kept
+    tile and 4*|q_i|*d per skipped block, with real (ragged) block sizes."""
+    N, d, bq, bk = cfg.N, cfg.d, cfg.block_q, cfg.block_k
+    nqb, nkb = cfg.n_qb, cfg.n_kb
+    qrows = np.array([min(bq, N - i * bq) for i in range(nqb)], dtype=np.float64)
+    kcols = np.array([min(bk, N - j * bk) for j in range(nkb)], dtype=np.float64)
+    BH = counts.shape[0]
+    kept_cols = np.zeros((BH, nqb))
+    n_skip = counts[..., 3].astype(np.float64)
+    for bh in range(BH):
+        for i in range(nqb):
+            nk = int(counts[bh, i, :3].sum())
+            kept_cols[bh, i] = kcols[lists[bh, i, :nk]].sum()
+    kept = 4.0 * d * (kept_cols * qrows[None, :]).sum()
+    skip = 4.0 * d * (n_skip * qrows[None, :]).sum()
+    return kept, skip
+
+
+def workload(args):
+    cfg = get_config(WORKLOAD)
+    if args.heads:
+        cfg = cfg.with_(H=args.heads)
+    return cfg
+
+
+def run_gpu_arm(args, rank, world, local_rank):
+    import precision_attention_video_b200 as pav
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = workload(args)
+    Q, K, V = make_qkv(cfg)
+    p = pav.params_for(cfg)
+    Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+    O = torch.empty_like(Qd)
+    ws = pav.alloc_workspace(p, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        pav.plan(p, Qd, Kd, Vd, ws, stream)
+        pav.forward(p, Qd, Kd, Vd, ws, O, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = pav.get_status(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {pav.status_string(st)}")
+
+    views = pav.plan_views(p, ws)
+    counts = views["row_counts"].cpu().numpy()
+    lists = views["row_lists"].cpu().numpy()
+    tiers = views["tier_map"].cpu().numpy()
+    kept_flops, skip_flops = algorithmic_attn_flops(cfg, counts, lists)
+
+    # timed region: K whole steps, events around each forward for the roofline
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clk:
+        t0.record(stream)
+        for a, b, c in ev:
+            a.record(stream)
+            pav.plan(p, Qd, Kd, Vd, ws, stream)
+            b.record(stream)
+            pav.forward(p, Qd, Kd, Vd, ws, O, stream)
+            c.record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = t0.elapsed_time(t1)
+    plan_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    fwd_ms = [b.elapsed_time(c) for _, b, c in ev]
+    st = pav.get_status(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {pav.status_string(st)}")
+
+    # end to end through the public C ABI from pinned host buffers
+    Qh, Kh, Vh = Q.pin_memory(), K.pin_memory(), V.pin_memory()
+    Oh = torch.empty_like(Q).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    pav.layer_from_host(p, Qh, Kh, Vh, Oh, Qd, Kd, Vd, O, ws, stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        pav.layer_from_host(p, Qh, Kh, Vh, Oh, Qd, Kd, Vd, O, ws, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    res = {
+        "total_ms": total_ms, "plan_ms": plan_ms, "fwd_ms": fwd_ms, "e2e_ms": e2e_ms,
+        "clocks": clk.summary(), "kept_flops": kept_flops, "skip_flops": skip_flops,
+        "tier_frac": {n: float((tiers == t).mean()) for n, t in
+                      (("full", 3), ("res", 2), ("low", 1), ("skip", 0))},
+        "h2d": 3 * Q.numel() * Q.element_size(), "d2h": O.numel() * O.element_size(),
+    }
+    return cfg, res
+
+
+def cpu_baseline(cfg, budget_s: float = 20.0, threads: int = 0):
+    """The oracle, as it stands, on a bounded sample of the workload: whole
+    heads are routed and quantised, then query blocks of those heads (spread
+    over the sequence) are attended until the time budget is used.  The unit
+    is dense-equivalent TFLOPS of the query rows attended; input generation is
+    not timed."""
+    import oracle
+    from latent_gen.generator import make_head
+    from oracle import quant as Qz
+    from oracle import route as Rt
+
+    cores = threads or len(os.sched_getaffinity(0))
+    rows, heads, spent = 0, 0, 0.0
+    nqb = cfg.n_qb
+    order = [(i * 17) % nqb for i in range(nqb)]
+    while spent < budget_s and heads < cfg.H:
+        q, k, v = make_head(cfg, 0, heads)
+        Qh, Kh, Vh = (torch.from_numpy(x).to(torch.bfloat16).double().numpy() for x in (q, k, v))
+        t = time.time()
+        rt = Rt.route_head(Qh, Kh, Vh, cfg.tau, cfg.block_q, cfg.block_k)
+        qt = Qz.quantize_head(Qh, Kh, Vh, cfg.low, cfg.block_q, cfg.block_k)
+        spent += time.time() - t
+        done = 0
+        while done < nqb and spent < budget_s:
+            blocks = order[done:done + cores]
+            t = time.time()
+            oracle.tiered_attention_head(Qh, Kh, Vh, rt, qt, cfg.low, cfg.block_q, cfg.block_k,
+                                         cfg.p_offset_log2, rt["scale"], False, blocks,
+                                         threads=cores)
+            spent += time.time() - t
+            rows += sum(min(cfg.block_q, cfg.N - i * cfg.block_q) for i in blocks)
+            done += len(blocks)
+        heads += 1
+    flops = 4.0 * rows * cfg.N * cfg.d
+    return {"value": flops / spent / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{heads} head(s) of the workload routed and quantised in full, {rows} of "
+                      f"{cfg.B * cfg.H * cfg.N} query rows attended; {spent:.1f} s of oracle time"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (smaller profiling cases)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = _env_int("WORLD_SIZE", 1)
+    rank = _env_int("RANK", 0)
+    local_rank = _env_int("LOCAL_RANK", 0)
+    cfg = workload(args)
+    config = {"workload": "480p-video-like tiered attention layer", "B": cfg.B, "H": cfg.H,
+              "N": cfg.N, "d": cfg.d, "grid_txyx": list(cfg.grid),
+              "tile": [cfg.block_q, cfg.block_k], "low_tier": "nvfp4", "tau": list(cfg.tau),
+              "logit_std": cfg.logit_std, "l2": "inputs larger than L2 (Q+K+V 1.0 GB per GPU)",
+              "parallelism": f"replicas x{args.gpus}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        t = time.time()
+        per = []
+        for _ in range(args.steps):
+            per.append(cpu_baseline(cfg, budget_s=max(5.0, 120.0 / max(1, args.steps))))
+        v = statistics.median([x["value"] for x in per])
+        ms = 4.0 * cfg.B * cfg.H * cfg.N ** 2 * cfg.d / (v * 1e12) * 1e3
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": v, "unit": UNIT, "cores": per[0]["cores"],
+                                 "kind": "oracle", "sample": per[0]["sample"]},
+                "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                "wall_s": time.time() - t}
+        print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    cfg, r = run_gpu_arm(args, rank, world, local_rank)
+
+    dense = 4.0 * cfg.B * cfg.H * float(cfg.N) ** 2 * cfg.d
+    step_ms = r["total_ms"] / args.steps
+    fwd_ms = statistics.mean(r["fwd_ms"])
+    if world > 1:
+        t = torch.tensor([step_ms, fwd_ms, r["e2e_ms"]], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        step_ms, fwd_ms, e2e_ms = t.tolist()
+    else:
+        e2e_ms = r["e2e_ms"]
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    executed = r["kept_flops"] + r["skip_flops"]
+    achieved = executed / (fwd_ms * 1e-3) / 1e12
+    traffic = None
+    if ATTN_TRAFFIC["source_sha1"] == attn_source_sha1():
+        traffic = ATTN_TRAFFIC["bytes_per_launch"]
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": world * dense / (step_ms * 1e-3) / 1e12, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config,
+            "ms_plan": statistics.mean(r["plan_ms"]), "ms_forward": fwd_ms,
+            "tier_frac": r["tier_frac"],
+            "roofline": {"kernel": "tiered_attn_forward (attn_kernel<128,128>)", "bound": "tensor",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16_tflops_sustained (MEASURED_PEAKS.json)"
+                         if peak_src == "measured" else "fallback 1.4 PFLOP/s sustained",
+                         "flops_per_launch": executed},
+            "e2e": {"value": world * dense / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": 4 * args.steps,
+            "clocks": r["clocks"],
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(cfg)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
