@@ -168,6 +168,32 @@ ta_status tiered_attn_prep(const ta_params* p, const void* Q_dev, const void* K_
                            const void* V_dev, void* ws_dev, size_t ws_bytes, void* stream);
 ta_status tiered_attn_route(const ta_params* p, void* ws_dev, size_t ws_bytes, void* stream);
 
+/* Router that allocates nothing (the pages have no counterpart: this is a
+ * deployment variant of tiered_attn_plan's routing stage).
+ *
+ * For callers that cannot allocate device memory: code running inside a host
+ * framework that owns all of the GPU's memory (a plugin with a fixed budget),
+ * or a latency-critical path where cudaMalloc would synchronise the device.
+ * From Q, K, V it writes the tier map (u8 [B*H, nQb, nKb]), the per-row tier
+ * counts (i32 [B*H, nQb, 4]) and the per-row lists (i32 [B*H, nQb, nKb]) into
+ * caller buffers, exactly as tiered_attn_plan does; it makes no low-precision
+ * copies.  Its intermediate block means, pooled logits and masses live in one
+ * fixed array of TA_ROUTE_NOALLOC_SCRATCH_BYTES in the library's device memory,
+ * which every GPU that loads the library holds until the process exits.
+ *  - Problems whose intermediates exceed that size (about B*H*nQb*nKb*16 +
+ *    B*H*(nQb+nKb)*d*8 + B*H*nKb*d*4 bytes) return TA_ERR_WORKSPACE.
+ *  - The first call on a device looks up the array's device address (with that
+ *    device current); make that first call before any stream capture.
+ *  - All calls share the one array: calls whose work overlaps on the GPU (two
+ *    streams, or two threads) race and corrupt each other's results.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * Output pointers must be device pointers; Q, K, V 16-byte aligned. */
+#define TA_ROUTE_NOALLOC_SCRATCH_BYTES (16u << 20)
+ta_status tiered_attn_route_noalloc(const ta_params* p, const void* Q_dev, const void* K_dev,
+                                    const void* V_dev, uint8_t* tier_map_dev,
+                                    int32_t* row_counts_dev, int32_t* row_lists_dev,
+                                    void* stream);
+
 /* Static description of a status code. */
 const char* tiered_attn_status_string(ta_status s);
 

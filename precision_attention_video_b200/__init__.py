@@ -11,6 +11,7 @@ from .binding import (  # noqa: F401
     TA_LOW_NONE, TA_LOW_FP8_E4M3, TA_LOW_NVFP4, TA_LOW_NVFP4_RES,
     TA_TIER_SKIP, TA_TIER_LOW, TA_TIER_RES, TA_TIER_FULL, TA_DEBUG_DROP_FIRST_K,
     TieredAttnError, alloc_workspace, forward, get_status, layer_from_host, make_params,
-    params_for, plan, plan_views, prep, route, status_string, version, workspace_bytes,
+    params_for, plan, plan_views, prep, route, route_noalloc, status_string, version,
+    workspace_bytes,
 )
 from .binding import LIB_PATH  # noqa: F401

@@ -70,6 +70,7 @@ def _load():
         "tiered_attn_get_status": (st, [vp, vp]),
         "tiered_attn_prep": (st, [P, vp, vp, vp, vp, sz, vp]),
         "tiered_attn_route": (st, [P, vp, sz, vp]),
+        "tiered_attn_route_noalloc": (st, [P, vp, vp, vp, vp, vp, vp, vp]),
         "tiered_attn_status_string": (ctypes.c_char_p, [st]),
         "tiered_attn_version": (ctypes.c_int32, []),
     }
@@ -162,6 +163,14 @@ def prep(p, Q, K, V, ws, stream=None) -> None:
 def route(p, ws, stream=None) -> None:
     _check("tiered_attn_route", _lib.tiered_attn_route(
         ctypes.byref(p), ws.data_ptr(), ws.numel(), _stream(stream)))
+
+
+def route_noalloc(p: ta_params, Q, K, V, tier_map, row_counts, row_lists, stream=None) -> None:
+    """Tier map, row counts and row lists without any workspace: the router's
+    intermediates live in the library's fixed device array (see the header)."""
+    _check("tiered_attn_route_noalloc", _lib.tiered_attn_route_noalloc(
+        ctypes.byref(p), Q.data_ptr(), K.data_ptr(), V.data_ptr(), tier_map.data_ptr(),
+        row_counts.data_ptr(), row_lists.data_ptr(), _stream(stream)))
 
 
 def forward(p: ta_params, Q, K, V, ws, O, stream=None) -> None:
