@@ -8,16 +8,19 @@
 // walks the block's compacted tile list (full ascending, low ascending, then
 // the skipped blocks) with an online softmax:
 //
-//   warp 4      producer: TMA loads of the kept K / V tiles (bf16, or the
+//   warp 8      producer: TMA loads of the kept K / V tiles (bf16, or the
 //               dequantised low copies) into a two-stage ring; for skipped
 //               blocks it gathers up to BK pooled rows kbar_b / vbar_b into a
 //               "pseudo-key" tile, so a skip chunk costs one tile of MMA for
 //               up to BK skipped blocks and never touches their K / V;
-//   warp 5      MMA issuer: tcgen05.mma kind::f16, S = Q K^T into a double-
+//   warp 9      MMA issuer: tcgen05.mma kind::f16, S = Q K^T into a double-
 //               buffered TMEM accumulator, O += P V into a TMEM accumulator;
 //               completion is signalled with tcgen05.commit on mbarriers;
-//   warps 0-3   softmax: thread r owns TMEM lane r (query row r): loads its S
-//               row, keeps the running max m and sum l, forms
+//   warps 0-7   softmax: warps w and w+4 share TMEM lanes 32w..32w+31 (query
+//               rows) and split each row's columns in halves; the pair swaps
+//               its half-row maxima through shared memory and a 64-thread
+//               named barrier.  Each thread loads its half S row, keeps the
+//               running max m and its half of the sum l, forms
 //               P' = 2^o exp(s - m'), rounds it as the tile's tier demands
 //               (bf16; e4m3; NVFP4 per 16 keys), rescales O in TMEM when m
 //               grows, and writes P' to shared memory as the A operand of PV.
@@ -36,9 +39,10 @@
 namespace ta {
 namespace {
 
-constexpr int kThreads = 192;  // 4 softmax warps + producer + MMA
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kSoftmaxWarps = 8;  // warp w: rows 32*(w%4).., column half w/4
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
 
 enum TileKind { KIND_FULL = 0, KIND_LOW = 1, KIND_SKIP = 2 };
 
@@ -73,6 +77,32 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Named barrier over `count` threads that also ANDs a predicate across them:
+// the warps of a softmax pair leave their loop together or not at all.
+__device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)pred), "r"(id), "r"(count)
+      : "memory");
+  return out != 0;
+}
+
+// Two e2m1 codes (low nibble first) to f16x2 (exact).
+__device__ __forceinline__ __half2 e2m1x2_to_half2(uint32_t codes) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
+      : "=r"(r)
+      : "r"(codes));
+  return *reinterpret_cast<__half2*>(&r);
+}
+
 // Shared-memory layout (offsets from a 1024-aligned base).
 template <int D, int BK>
 struct Smem {
@@ -89,8 +119,9 @@ struct Smem {
   static constexpr int oBar = oP + kP;
   static constexpr int kBars = 16;
   static constexpr int oMisc = oBar + kBars * 8;
-  static constexpr int kTotal = oMisc + 64;
-  static constexpr int kAlloc = kTotal + 1024;  // alignment slack
+  static constexpr int oXchg = oMisc + 64;  // float [2 slots][2 halves][128 rows]
+  static constexpr int kTotal = oXchg + 2 * 2 * 128 * 4;
+  static constexpr int kAlloc = kTotal;  // the base is checked for 1024-byte alignment
   static constexpr uint32_t kTmemCols = (2 * BK + D) <= 256 ? 256u : 512u;
 };
 
@@ -107,8 +138,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tmDV) {
   using L = Smem<D, BK>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* sm = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* sm = smem_raw;
+  if (smem_u32(sm) & 1023u) {
+    // the 128-byte-swizzled tiles need a 1024-byte-aligned base: refuse cleanly
+    if (threadIdx.x == 0 && a.status) atomicCAS(a.status + ST_CODE, 0, (int)TA_ERR_UNSUPPORTED);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::oBar);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::oMisc);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::oMisc + 4);
@@ -142,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[BAR_E1], 1);
     mbar_init(&bars[BAR_S0], 1);
     mbar_init(&bars[BAR_S1], 1);
-    mbar_init(&bars[BAR_P], a.bq);
+    mbar_init(&bars[BAR_P], 2 * a.bq);  // both column halves of every live row
     mbar_init(&bars[BAR_O], 1);
     mbar_init(&bars[BAR_DRAIN], 1);
     fence_mbar_init();
@@ -226,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         // gather pooled rows of the skipped blocks into a pseudo K / V tile
         const int cnt = min(BK, rp.n_skip - (first - rp.n_full - rp.n_res - rp.n_low));
+#pragma unroll 8
         for (int e = lane; e < BK * (D / 8); e += 32) {
           const int c = e / (D / 8), ch = e % (D / 8);
           uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
@@ -307,18 +343,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_drain(&bars[BAR_DRAIN], 0);
       }
     }
-  } else if (threadIdx.x < a.bq) {
+  } else if (warp < kSoftmaxWarps && (warp & 3) * 32 < a.bq) {
     // ===================== softmax warps =====================
-    const int r = threadIdx.x;  // query row within the tile == TMEM lane
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    constexpr int HB = BK / 2;              // columns per half row
+    constexpr int HD = D / 2;               // O columns per half row
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;      // query row within the tile == TMEM lane
+    const int pair_bar = 1 + quarter;       // named barrier of warps quarter, quarter+4
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    float* xchg = reinterpret_cast<float*>(sm + L::oXchg);  // [slot][half][row]
+    const float c2 = a.scale_log2;           // S -> log2 units
     const float o_off = (float)a.p_offset;
-    float m = -INFINITY, l = 0.0f;
+    float m = -INFINITY, l = 0.0f;           // running max (raw S units), half row sum
     for (int t = 0; t < rp.T; ++t) {
       const int s = t & 1;
       bool ok = mbar_wait(&bars[BAR_S0 + s], (t >> 1) & 1, ctx, 6);
       ok = __all_sync(0xffffffffu, ok);
-      if (!ok) { aborted = true; break; }
-      tc_fence_after();
       int kind, first;
       tile_of<BK>(rp, t, kind, first);
       int nvalid;
@@ -327,93 +367,109 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         nvalid = min(BK, a.N - rp.list[first] * BK);
       }
-      float x[BK];
-#pragma unroll
-      for (int c0 = 0; c0 < BK; c0 += 32) {
-        uint32_t raw[32];
-        tmem_ld32((s ? tS1 : tS0) + lane_off + c0, raw);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[c0 + c] = __uint_as_float(raw[c]) * a.scale_log2;
-      }
+      const int nv = min(max(nvalid - half * HB, 0), HB);  // valid columns of this half
+      float x[HB];
       float tmax = -INFINITY;
+      if (ok) {
+        tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < BK; ++c) {
-        if (c >= nvalid) x[c] = -INFINITY;
-        tmax = fmaxf(tmax, x[c]);
+        for (int c0 = 0; c0 < HB; c0 += 32) {
+          uint32_t raw[32];
+          tmem_ld32((s ? tS1 : tS0) + lane_off + half * HB + c0, raw);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c0 + c] = __uint_as_float(raw[c]);
+        }
+        if (nv == HB) {
+#pragma unroll
+          for (int c = 0; c < HB; ++c) tmax = fmaxf(tmax, x[c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < HB; ++c) {
+            if (c >= nv) x[c] = -INFINITY;
+            tmax = fmaxf(tmax, x[c]);
+          }
+        }
+        xchg[(s * 2 + half) * 128 + r] = tmax;
       }
-      const float m_new = fmaxf(m, tmax);
-      const float alpha = fast_exp2(m - m_new);  // 0 on the first tile
+      // swap half-row maxima with the partner warp; leave together on abort
+      ok = bar_and(pair_bar, 64, ok);
+      if (!ok) { aborted = true; break; }
+      const float m_new = fmaxf(m, fmaxf(tmax, xchg[(s * 2 + (half ^ 1)) * 128 + r]));
+      const float alpha = fast_exp2((m - m_new) * c2);  // 0 on the first tile
+      const float mc = m_new * c2 - o_off;              // P' = 2^(s*c2 - mc)
       float rowsum = 0.0f;
 #pragma unroll
-      for (int c = 0; c < BK; ++c) {
-        x[c] = fast_exp2(x[c] - m_new + o_off);
-      }
+      for (int c = 0; c < HB; ++c) x[c] = fast_exp2(fmaf(x[c], c2, -mc));
       if (kind == KIND_SKIP) {
 #pragma unroll
-        for (int c = 0; c < BK; ++c) {
-          if (c < nvalid) {
-            const int j = rp.list[first + c];
+        for (int c = 0; c < HB; ++c) {
+          if (c < nv) {
+            const int j = rp.list[first + half * HB + c];
             x[c] *= (float)min(BK, a.N - j * BK);
           }
         }
       }
 #pragma unroll
-      for (int c = 0; c < BK; ++c) rowsum += x[c];
+      for (int c = 0; c < HB; ++c) rowsum += x[c];
       l = l * alpha + rowsum;
       m = m_new;
 
       // round P' as the tier demands, into bf16 pairs
-      uint32_t p[BK / 2];
+      uint32_t p[HB / 2];
       if (kind == KIND_LOW && a.low == TA_LOW_FP8_E4M3) {
 #pragma unroll
-        for (int c = 0; c < BK; c += 2) {
+        for (int c = 0; c < HB; c += 2) {
           const float2 f = e4m3x2_to_float2(cvt_e4m3x2(x[c], x[c + 1]));
           p[c / 2] = pack_bf16(f.x, f.y);
         }
       } else if (kind == KIND_LOW) {
 #pragma unroll
-        for (int g = 0; g < BK; g += 16) {
+        for (int g = 0; g < HB; g += 16) {
           float amax = 0.0f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) amax = fmaxf(amax, x[g + i]);
           const uint32_t scc = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xFFu;
           const float sc = e4m3_to_float(scc);
           const float inv = (sc > 0.0f) ? __frcp_rn(sc) : 0.0f;
+          const __half2 sc2 = __float2half2_rn(sc);  // exact: a ue4m3 value
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
             const uint32_t cc = cvt_e2m1x2(__fmul_rn(x[g + i], inv), __fmul_rn(x[g + i + 1], inv));
-            p[(g + i) / 2] = pack_bf16(e2m1_value(cc & 0xFu) * sc, e2m1_value(cc >> 4) * sc);
+            const float2 f = __half22float2(__hmul2(e2m1x2_to_half2(cc), sc2));  // exact
+            p[(g + i) / 2] = pack_bf16(f.x, f.y);
           }
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < BK; c += 2) p[c / 2] = pack_bf16(x[c], x[c + 1]);
+        for (int c = 0; c < HB; c += 2) p[c / 2] = pack_bf16(x[c], x[c + 1]);
       }
 
       // PV of the previous tile must be done before P and O are touched
       if (t > 0) {
         bool ok2 = mbar_wait(&bars[BAR_O], (t - 1) & 1, ctx, 7);
         ok2 = __all_sync(0xffffffffu, ok2);
+        ok2 = bar_and(pair_bar, 64, ok2);
         if (!ok2) { aborted = true; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
+          for (int c0 = 0; c0 < HD; c0 += 32) {
             uint32_t raw[32];
-            tmem_ld32(tO + lane_off + c0, raw);
+            tmem_ld32(tO + lane_off + half * HD + c0, raw);
 #pragma unroll
             for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * alpha);
-            tmem_st32(tO + lane_off + c0, raw);
+            tmem_st32(tO + lane_off + half * HD + c0, raw);
           }
           tmem_wait_st();
         }
       }
-      // P row -> shared memory, K-major, 128-byte swizzle
+      // this half of the P row -> shared memory, K-major, 128-byte swizzle
 #pragma unroll
-      for (int ch = 0; ch < BK / 8; ++ch) {
+      for (int q = 0; q < HB / 8; ++q) {
+        const int ch = half * (HB / 8) + q;    // 16-byte chunk index within the row
         const uint32_t off = (ch >> 3) * (128 * 128) + r * 128 + (((ch & 7) ^ (r & 7)) * 16);
         *reinterpret_cast<uint4*>(sm + L::oP + off) =
-            make_uint4(p[ch * 4 + 0], p[ch * 4 + 1], p[ch * 4 + 2], p[ch * 4 + 3]);
+            make_uint4(p[q * 4 + 0], p[q * 4 + 1], p[q * 4 + 2], p[q * 4 + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -422,15 +478,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!aborted) {
       bool ok = mbar_wait(&bars[BAR_O], (rp.T - 1) & 1, ctx, 8);
       ok = __all_sync(0xffffffffu, ok);
+      // row sums go to the slot the last tile did not use (free since the
+      // pair's barrier of tile T-1)
+      const int ls = rp.T & 1;
+      xchg[(ls * 2 + half) * 128 + r] = l;
+      ok = bar_and(pair_bar, 64, ok);
       if (ok) {
         tc_fence_after();
-        const float inv_l = 1.0f / l;
+        const float inv_l = 1.0f / (l + xchg[(ls * 2 + (half ^ 1)) * 128 + r]);
         const bool valid = (q0 + r) < a.N;
-        __nv_bfloat16* orow = a.O + (int64_t)b * a.sb + (int64_t)h * a.sh + (int64_t)(q0 + r) * a.sn;
+        __nv_bfloat16* orow = a.O + (int64_t)b * a.sb + (int64_t)h * a.sh + (int64_t)(q0 + r) * a.sn +
+                              half * HD;
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = 0; c0 < HD; c0 += 32) {
           uint32_t raw[32];
-          tmem_ld32(tO + lane_off + c0, raw);
+          tmem_ld32(tO + lane_off + half * HD + c0, raw);
           uint32_t w[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2)
