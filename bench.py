@@ -128,22 +128,26 @@ class ClockSampler:
 
 
 def algorithmic_attn_flops(cfg, counts: np.ndarray, lists: np.ndarray):
-    """FLOPs the tiered forward is defined to execute: 4*|q_i|*|k_j|*d per kept
-    tile and 4*|q_i|*d per skipped block, with real (ragged) block sizes."""
+    """FLOPs the tiered forward is defined to execute, by tier: 4*|q_i|*|k_j|*d
+    per full / residual / low tile and 4*|q_i|*d per skipped block, with real
+    (ragged) block sizes.  Returns (full, low, skip)."""
     N, d, bq, bk = cfg.N, cfg.d, cfg.block_q, cfg.block_k
     nqb, nkb = cfg.n_qb, cfg.n_kb
     qrows = np.array([min(bq, N - i * bq) for i in range(nqb)], dtype=np.float64)
     kcols = np.array([min(bk, N - j * bk) for j in range(nkb)], dtype=np.float64)
     BH = counts.shape[0]
-    kept_cols = np.zeros((BH, nqb))
+    full_cols = np.zeros((BH, nqb))
+    low_cols = np.zeros((BH, nqb))
     n_skip = counts[..., 3].astype(np.float64)
     for bh in range(BH):
         for i in range(nqb):
-            nk = int(counts[bh, i, :3].sum())
-            kept_cols[bh, i] = kcols[lists[bh, i, :nk]].sum()
-    kept = 4.0 * d * (kept_cols * qrows[None, :]).sum()
+            nf, nr, nl = (int(x) for x in counts[bh, i, :3])
+            full_cols[bh, i] = kcols[lists[bh, i, :nf + nr]].sum()
+            low_cols[bh, i] = kcols[lists[bh, i, nf + nr:nf + nr + nl]].sum()
+    full = 4.0 * d * (full_cols * qrows[None, :]).sum()
+    low = 4.0 * d * (low_cols * qrows[None, :]).sum()
     skip = 4.0 * d * (n_skip * qrows[None, :]).sum()
-    return kept, skip
+    return full, low, skip
 
 
 def workload(args):
@@ -181,7 +185,7 @@ def run_gpu_arm(args, rank, world, local_rank):
     counts = views["row_counts"].cpu().numpy()
     lists = views["row_lists"].cpu().numpy()
     tiers = views["tier_map"].cpu().numpy()
-    kept_flops, skip_flops = algorithmic_attn_flops(cfg, counts, lists)
+    full_flops, low_flops, skip_flops = algorithmic_attn_flops(cfg, counts, lists)
 
     # timed region: K whole steps, events around each forward for the roofline
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -227,7 +231,8 @@ def run_gpu_arm(args, rank, world, local_rank):
 
     res = {
         "total_ms": total_ms, "plan_ms": plan_ms, "fwd_ms": fwd_ms, "e2e_ms": e2e_ms,
-        "clocks": clk.summary(), "kept_flops": kept_flops, "skip_flops": skip_flops,
+        "clocks": clk.summary(), "full_flops": full_flops, "low_flops": low_flops,
+        "skip_flops": skip_flops,
         "tier_frac": {n: float((tiers == t).mean()) for n, t in
                       (("full", 3), ("res", 2), ("low", 1), ("skip", 0))},
         "h2d": 3 * Q.numel() * Q.element_size(), "d2h": O.numel() * O.element_size(),
@@ -331,8 +336,14 @@ def main():
     else:
         e2e_ms = r["e2e_ms"]
     peaks, peak_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    executed = r["kept_flops"] + r["skip_flops"]
+    p_bf16 = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    # full tiles and skip chunks run on the bf16 pipe; NVFP4 low tiles on the
+    # FP4 pipe, whose peak is taken as 4x the measured bf16 one (nominal ratio).
+    # FP8 low tiles (other workloads) run on bf16 images, at the bf16 peak.
+    p_low = 4.0 * p_bf16 if cfg.low == 2 else p_bf16
+    executed = r["full_flops"] + r["low_flops"] + r["skip_flops"]
+    t_min = (r["full_flops"] + r["skip_flops"]) / (p_bf16 * 1e12) + r["low_flops"] / (p_low * 1e12)
+    peak = executed / t_min / 1e12          # blended tensor peak of this launch's FLOP mix
     achieved = executed / (fwd_ms * 1e-3) / 1e12
     traffic = None
     if ATTN_TRAFFIC["source_sha1"] == attn_source_sha1():
@@ -349,9 +360,12 @@ def main():
             "roofline": {"kernel": "tiered_attn_forward (attn_kernel<128,128>)", "bound": "tensor",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"{peak_src} bf16_tflops_sustained (MEASURED_PEAKS.json)"
-                         if peak_src == "measured" else "fallback 1.4 PFLOP/s sustained",
-                         "flops_per_launch": executed},
+                         "peak_source": (f"blend of {peak_src} bf16_tflops_sustained "
+                                         f"{p_bf16:.1f} and nvfp4 = 4x that, weighted by "
+                                         "the launch's FLOPs per tier"),
+                         "flops_per_launch": executed,
+                         "flops_by_tier": {"full": r["full_flops"], "low": r["low_flops"],
+                                           "skip": r["skip_flops"]}},
             "e2e": {"value": world * dense / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                     "ms_per_step": e2e_ms},

@@ -114,7 +114,9 @@ typedef struct {
   /* residual NVFP4 copies (TA_LOW_NVFP4_RES), same layouts as above */
   uint8_t* rq_codes; uint8_t* rk_codes; uint8_t* rv_codes;
   uint8_t* rq_scales; uint8_t* rk_scales; uint8_t* rv_scales;
-  /* bf16 [BH, N, d] dequantised values of the low copies (exact in bf16) */
+  /* bf16 [BH, N, d] dequantised values of the low copies (exact in bf16);
+   * present for the FP8 and residual formats, whose tiles read them (NVFP4
+   * tiles run on the packed codes and scales directly) */
   uint16_t* dq; uint16_t* dk; uint16_t* dv;
   /* bf16 [BH, N, d] dequantised residual copies (TA_LOW_NVFP4_RES) */
   uint16_t* drq; uint16_t* drk; uint16_t* drv;
@@ -126,8 +128,8 @@ size_t tiered_attn_workspace_bytes(const ta_params* p);
 
 /* Router + quantiser ("Triage" abstract: the router predicts from block
  * statistics; NVFP4 skim / refine copies).  Reads Q, K, V once: block means of
- * Q, K, V (fp64), the low-precision copies of Q, K, V and their dequantised
- * bf16 values; then the pooled logits, the n_j-weighted pooled block softmax M,
+ * Q, K, V (fp64), the low-precision copies of Q, K, V (and, for FP8 and the
+ * residual format, their dequantised bf16 values); then the pooled logits, the n_j-weighted pooled block softmax M,
  * the tiers by exclusive cumulative mass in (-M, j) order (most precise tier t
  * with prefix < tau[t], else skip; diagonal blocks forced full when
  * keep_diag_full), and the per-row tile lists.  Three kernel launches on

@@ -112,7 +112,9 @@ Layout layout_of(const ta_params* p) {
       }
     }
   }
-  if (p->low != TA_LOW_NONE) {
+  // bf16 images of the low copies: the FP8 tier and the residual tier read
+  // them; NVFP4 tiles run natively on the packed codes
+  if (p->low == TA_LOW_FP8_E4M3 || p->low == TA_LOW_NVFP4_RES) {
     L.dq = take(tok * 2);
     L.dk = take(tok * 2);
     L.dv = take(tok * 2);
@@ -217,6 +219,21 @@ EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(f);
   });
   return fn;
+}
+
+// Byte tensor [BH, rows, inner] (contiguous), box = 64 bytes x box_rows,
+// 64-byte swizzle: the packed NVFP4 copies.
+bool make_map_fp4(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int64_t inner,
+                  int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)inner, (cuuint64_t)(inner * rows)};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // bf16 tensor [B, H, N, d] (element strides sb, sh, sn), box = 64 x rows, 128B swizzle.
@@ -332,6 +349,9 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
     return st;
   if ((st = check_ws(p, ws, ws_bytes)) != TA_OK) return st;
   if (p->low == TA_LOW_NVFP4_RES) return TA_ERR_UNSUPPORTED;
+  // native NVFP4 tiles are built for d = 128 with 128 x 128 tiles
+  if (p->low == TA_LOW_NVFP4 && (p->d != 128 || p->block_q != 128 || p->block_k != 128))
+    return TA_ERR_UNSUPPORTED;
   const Shape s = shape_of(p);
   const Layout L = layout_of(p);
   ta::AttnArgs a;
@@ -357,6 +377,10 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
   a.row_counts = at<int>(ws, L.row_counts);
   a.row_lists = at<int>(ws, L.row_lists);
   a.O = static_cast<__nv_bfloat16*>(O);
+  a.Np = (int)s.Np;
+  a.q_sf = p->low == TA_LOW_NVFP4 ? at<uint8_t>(ws, L.q_scales) : nullptr;
+  a.k_sf = p->low == TA_LOW_NVFP4 ? at<uint8_t>(ws, L.k_scales) : nullptr;
+  a.v_sf = p->low == TA_LOW_NVFP4 ? at<uint8_t>(ws, L.v_scales) : nullptr;
 
   CUtensorMap maps[6];
   const int64_t cb = (int64_t)p->H * p->N * p->d, ch = (int64_t)p->N * p->d, cn = p->d;
@@ -365,7 +389,12 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
             make_map(&maps[2], V, p->B, p->H, p->N, p->d, p->stride_b, p->stride_h, p->stride_n, p->block_k);
   // the dequantised copies are contiguous [B*H, N, d]; without a low tier they
   // alias the bf16 inputs (never read)
-  if (L.dq != kAbsent) {
+  if (p->low == TA_LOW_NVFP4) {
+    const int64_t BH = (int64_t)p->B * p->H;
+    ok = ok && make_map_fp4(&maps[3], at<void>(ws, L.q_codes), BH, p->N, p->d / 2, p->block_q) &&
+         make_map_fp4(&maps[4], at<void>(ws, L.k_codes), BH, p->N, p->d / 2, p->block_k) &&
+         make_map_fp4(&maps[5], at<void>(ws, L.v_codes), BH, p->d, s.Np / 2, p->d);
+  } else if (L.dq != kAbsent) {
     const void* dq = at<void>(ws, L.dq);
     const void* dk = at<void>(ws, L.dk);
     const void* dv = at<void>(ws, L.dv);

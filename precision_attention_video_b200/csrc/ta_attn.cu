@@ -130,13 +130,47 @@ enum {
   BAR_S0 = 7, BAR_S1 = 8, BAR_P = 9, BAR_O = 10, BAR_DRAIN = 11
 };
 
+// TMEM columns of the NVFP4 scale factors (4 columns per 64-element K chunk,
+// 2 chunks per operand), after S0, S1 and O.
 template <int D, int BK>
+struct TmemSf {
+  static constexpr uint32_t kSfaQ = 2 * BK + D;
+  static constexpr uint32_t kSfbK0 = kSfaQ + 8, kSfbK1 = kSfaQ + 16;
+  static constexpr uint32_t kSfbV0 = kSfaQ + 24, kSfbV1 = kSfaQ + 32;
+  static constexpr uint32_t kSfaP = kSfaQ + 40;  // last block ends at kSfaQ + 48 <= 512
+};
+
+// NVFP4 tiles in shared memory: codes [rows][64 B] with 64-byte swizzle, then
+// the two [32][16 B] scale-factor blocks at +kFp4Sf.
+constexpr int kFp4Sf = 128 * 64;
+
+// Gather the ue4m3 scales of `nrows` rows (row-major, 8 bytes = 8 groups of 16
+// along d = 128) into the two [32][16 B] blocks at `dst`: row 32*m1 + m0 of K
+// chunk c (groups 4c..4c+3) at dst + c*512 + m0*16 + m1*4.  Rows past
+// `nrows` get zero scales.
+__device__ __forceinline__ void gather_row_sf(unsigned char* dst, const uint8_t* src, int nrows,
+                                              int lane) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = lane * 4 + i;
+    uint2 v = make_uint2(0u, 0u);
+    if (rr < nrows) v = *reinterpret_cast<const uint2*>(src + (int64_t)rr * 8);
+    const int off = (rr & 31) * 16 + (rr >> 5) * 4;
+    *reinterpret_cast<uint32_t*>(dst + off) = v.x;
+    *reinterpret_cast<uint32_t*>(dst + 512 + off) = v.y;
+  }
+}
+
+template <int D, int BK, bool FP4>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmQ,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
                 const __grid_constant__ CUtensorMap tmDV) {
   using L = Smem<D, BK>;
+  using TS = TmemSf<D, BK>;
+  static_assert(!FP4 || (D == 128 && BK == 128), "native NVFP4 tiles need d = 128, 128-key tiles");
+  constexpr uint32_t kTmemCols = FP4 ? 512u : L::kTmemCols;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw;
   if (smem_u32(sm) & 1023u) {
@@ -201,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -215,16 +249,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp) {
     // ===================== producer =====================
     int kf_issued[2] = {0, 0}, vf_issued[2] = {0, 0};
+    if (FP4 && has_low) {
+      // scales of the NVFP4 query copy, ready for tcgen05.cp
+      gather_row_sf(sm + L::oDQ + kFp4Sf, a.q_sf + ((int64_t)bh * a.N + q0) * 8,
+                    min(128, a.N - q0), lane);
+      fence_proxy_async_smem();
+      __syncwarp();
+    }
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       const uint32_t qbytes = (uint32_t)a.bq * D * 2;
-      mbar_arrive_expect_tx(&bars[BAR_Q], has_low ? 2 * qbytes : qbytes);
-      for (int x = 0; x < D / 64; ++x) {
+      const uint32_t lbytes = FP4 ? (uint32_t)a.bq * 64 : qbytes;
+      mbar_arrive_expect_tx(&bars[BAR_Q], has_low ? qbytes + lbytes : qbytes);
+      for (int x = 0; x < D / 64; ++x)
         tma_load_4d(sm + L::oQ + x * (128 * 128), &tmQ, &bars[BAR_Q], x * 64, q0, h, b);
-        if (has_low)
-          tma_load_4d(sm + L::oDQ + x * (128 * 128), &tmDQ, &bars[BAR_Q], x * 64, q0, h, b);
+      if (has_low) {
+        if (FP4) {
+          tma_load_3d(sm + L::oDQ, &tmDQ, &bars[BAR_Q], 0, q0, bh);
+        } else {
+          for (int x = 0; x < D / 64; ++x)
+            tma_load_4d(sm + L::oDQ + x * (128 * 128), &tmDQ, &bars[BAR_Q], x * 64, q0, h, b);
+        }
       }
     }
     const __nv_bfloat16* kbar = a.kbar_b + (int64_t)bh * a.nKb * D;
@@ -241,7 +288,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       tile_of<BK>(rp, t, kind, first);
       unsigned char* kst = sm + (s ? L::oK1 : L::oK0);
       unsigned char* vst = sm + (s ? L::oV1 : L::oV0);
-      if (kind != KIND_SKIP) {
+      if (FP4 && kind == KIND_LOW) {
+        const int j = rp.list[first];
+        // K scales (rows of the key tile) and V scales (groups of 16 keys of
+        // each d row) into the stage, in the tcgen05.cp block layout
+        gather_row_sf(kst + kFp4Sf, a.k_sf + ((int64_t)bh * a.N + j * BK) * 8,
+                      min(BK, a.N - j * BK), lane);
+        const int ng = a.Np / 16;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int g = j * 8 + c * 4 + k;   // group of 16 keys
+            uint32_t w = 0u;
+            if (g < ng) w = *reinterpret_cast<const uint32_t*>(a.v_sf + ((int64_t)bh * ng + g) * D + lane * 4);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int m = lane * 4 + i;        // d row of V^T
+              vst[kFp4Sf + c * 512 + (m & 31) * 16 + (m >> 5) * 4 + k] = (unsigned char)(w >> (8 * i));
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const bool drop = (t == 0) && (a.debug_flags & TA_DEBUG_DROP_FIRST_K);
+          if (!drop) {
+            mbar_arrive_expect_tx(&bars[BAR_K0 + s], BK * 64);
+            tma_load_3d(kst, &tmDK, &bars[BAR_K0 + s], 0, j * BK, bh);
+            kf_issued[s]++;
+          }
+          mbar_arrive_expect_tx(&bars[BAR_V0 + s], D * 64);
+          tma_load_3d(vst, &tmDV, &bars[BAR_V0 + s], j * 64, 0, bh);
+          vf_issued[s]++;
+        }
+      } else if (kind != KIND_SKIP) {
         if (lane == 0) {
           const int j = rp.list[first];
           const CUtensorMap* mk = (kind == KIND_LOW) ? &tmDK : &tmK;
@@ -307,11 +388,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tile_of<BK>(rp, t, kind, first);
         const uint32_t aq = (kind == KIND_LOW) ? sDQ : sQ;
         const uint32_t sk = smem_u32(sm + (s ? L::oK1 : L::oK0));
+        if (FP4 && kind == KIND_LOW) {
+          const uint32_t sfb = tmem + (s ? TS::kSfbK1 : TS::kSfbK0);
+          tc_cp_sf(sfb, smem_desc_rows16(sk + kFp4Sf));
+          tc_cp_sf(sfb + 4, smem_desc_rows16(sk + kFp4Sf + 512));
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(aq + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sk + (kk >> 2) * (BK * 128) + (kk & 3) * 32, 16, 1024);
-          mma_f16_ss(s ? tS1 : tS0, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 2; ++kk)
+            mma_nvfp4_ss(s ? tS1 : tS0, smem_desc_sw64(aq + kk * 32), smem_desc_sw64(sk + kk * 32),
+                         idesc_nvfp4(128, BK), tmem + TS::kSfaQ + kk * 4, sfb + kk * 4,
+                         kk > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(aq + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sk + (kk >> 2) * (BK * 128) + (kk & 3) * 32, 16, 1024);
+            mma_f16_ss(s ? tS1 : tS0, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          }
         }
         tc_commit(&bars[BAR_S0 + s]);
         return true;
@@ -319,6 +411,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(&bars[BAR_Q], 0, ctx, 3);
       if (ok) {
         tc_fence_after();
+        if (FP4 && has_low) {
+          tc_cp_sf(tmem + TS::kSfaQ, smem_desc_rows16(sDQ + kFp4Sf));
+          tc_cp_sf(tmem + TS::kSfaQ + 4, smem_desc_rows16(sDQ + kFp4Sf + 512));
+        }
         ok = issue_s(0);
       }
       for (int t = 0; ok && t < rp.T; ++t) {
@@ -328,11 +424,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&bars[BAR_V0 + s], (t >> 1) & 1, ctx, 5)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sv = smem_u32(sm + (s ? L::oV1 : L::oV0));
+        int kind_t, first_t;
+        tile_of<BK>(rp, t, kind_t, first_t);
+        if (FP4 && kind_t == KIND_LOW) {
+          const uint32_t sfb = tmem + (s ? TS::kSfbV1 : TS::kSfbV0);
+          tc_cp_sf(tmem + TS::kSfaP, smem_desc_rows16(sP + kFp4Sf));
+          tc_cp_sf(tmem + TS::kSfaP + 4, smem_desc_rows16(sP + kFp4Sf + 512));
+          tc_cp_sf(sfb, smem_desc_rows16(sv + kFp4Sf));
+          tc_cp_sf(sfb + 4, smem_desc_rows16(sv + kFp4Sf + 512));
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(sP + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sv + kk * 16 * 128, BK * 128, 1024);
-          mma_f16_ss(tO, ad, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 2; ++kk)
+            mma_nvfp4_ss(tO, smem_desc_sw64(sP + kk * 32), smem_desc_sw64(sv + kk * 32),
+                         idesc_nvfp4(128, D), tmem + TS::kSfaP + kk * 4, sfb + kk * 4,
+                         (t > 0 || kk > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(sP + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sv + kk * 16 * 128, BK * 128, 1024);
+            mma_f16_ss(tO, ad, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         tc_commit(&bars[BAR_O]);
         tc_commit(&bars[BAR_E0 + s]);
@@ -414,9 +525,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       l = l * alpha + rowsum;
       m = m_new;
 
-      // round P' as the tier demands, into bf16 pairs
+      // round P' as the tier demands, into bf16 pairs (or NVFP4 codes)
       uint32_t p[HB / 2];
-      if (kind == KIND_LOW && a.low == TA_LOW_FP8_E4M3) {
+      if (FP4 && kind == KIND_LOW) {
+        // codes of this half row (64 keys = one MMA K chunk) packed in p[0..7],
+        // ue4m3 scales of its 4 groups in p[8]
+        uint32_t scw = 0u;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float amax = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) amax = fmaxf(amax, x[g * 16 + i]);
+          const uint32_t scc = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xFFu;
+          const float sc = e4m3_to_float(scc);
+          const float inv = (sc > 0.0f) ? __frcp_rn(sc) : 0.0f;
+          scw |= scc << (8 * g);
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            uint32_t word = 0u;
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+              const int c = g * 16 + w * 8 + i;
+              word |= cvt_e2m1x2(__fmul_rn(x[c], inv), __fmul_rn(x[c + 1], inv)) << (4 * i);
+            }
+            p[g * 2 + w] = word;
+          }
+        }
+        p[8] = scw;
+      } else if (kind == KIND_LOW && a.low == TA_LOW_FP8_E4M3) {
 #pragma unroll
         for (int c = 0; c < HB; c += 2) {
           const float2 f = e4m3x2_to_float2(cvt_e4m3x2(x[c], x[c + 1]));
@@ -463,13 +599,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
         }
       }
-      // this half of the P row -> shared memory, K-major, 128-byte swizzle
+      if (FP4 && kind == KIND_LOW) {
+        // NVFP4 P row half: 32 bytes of codes into the 64-byte-swizzled tile,
+        // 4 scale bytes into the scale-factor block of K chunk `half`
 #pragma unroll
-      for (int q = 0; q < HB / 8; ++q) {
-        const int ch = half * (HB / 8) + q;    // 16-byte chunk index within the row
-        const uint32_t off = (ch >> 3) * (128 * 128) + r * 128 + (((ch & 7) ^ (r & 7)) * 16);
-        *reinterpret_cast<uint4*>(sm + L::oP + off) =
-            make_uint4(p[q * 4 + 0], p[q * 4 + 1], p[q * 4 + 2], p[q * 4 + 3]);
+        for (int q = 0; q < 2; ++q) {
+          const int ch = half * 2 + q;
+          const uint32_t off = r * 64 + ((ch ^ ((r >> 1) & 3)) * 16);
+          *reinterpret_cast<uint4*>(sm + L::oP + off) =
+              make_uint4(p[q * 4 + 0], p[q * 4 + 1], p[q * 4 + 2], p[q * 4 + 3]);
+        }
+        *reinterpret_cast<uint32_t*>(sm + L::oP + kFp4Sf + half * 512 + lane * 16 + quarter * 4) = p[8];
+      } else {
+        // this half of the P row -> shared memory, K-major, 128-byte swizzle
+#pragma unroll
+        for (int q = 0; q < HB / 8; ++q) {
+          const int ch = half * (HB / 8) + q;    // 16-byte chunk index within the row
+          const uint32_t off = (ch >> 3) * (128 * 128) + r * 128 + (((ch & 7) ^ (r & 7)) * 16);
+          *reinterpret_cast<uint4*>(sm + L::oP + off) =
+              make_uint4(p[q * 4 + 0], p[q * 4 + 1], p[q * 4 + 2], p[q * 4 + 3]);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -514,13 +663,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, L::kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int D, int BK>
+template <int D, int BK, bool FP4>
 cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
   using L = Smem<D, BK>;
-  auto k = attn_kernel<D, BK>;
+  auto k = attn_kernel<D, BK, FP4>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nQb, a.B * a.H);
@@ -538,10 +687,11 @@ int attn_smem_bytes(int d, int bk) {
 }
 
 cudaError_t launch_attn(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
-  if (a.d == 64 && a.bk == 64) return launch_d<64, 64>(a, maps, s);
-  if (a.d == 64 && a.bk == 128) return launch_d<64, 128>(a, maps, s);
-  if (a.d == 128 && a.bk == 64) return launch_d<128, 64>(a, maps, s);
-  return launch_d<128, 128>(a, maps, s);
+  if (a.d == 64 && a.bk == 64) return launch_d<64, 64, false>(a, maps, s);
+  if (a.d == 64 && a.bk == 128) return launch_d<64, 128, false>(a, maps, s);
+  if (a.d == 128 && a.bk == 64) return launch_d<128, 64, false>(a, maps, s);
+  if (a.low == TA_LOW_NVFP4) return launch_d<128, 128, true>(a, maps, s);
+  return launch_d<128, 128, false>(a, maps, s);
 }
 
 }  // namespace ta

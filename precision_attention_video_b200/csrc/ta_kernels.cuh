@@ -57,6 +57,12 @@ struct AttnArgs {
   const int* row_counts;
   const int* row_lists;
   __nv_bfloat16* O;
+  // NVFP4 scales of the low copies (used by the native FP4 tile path):
+  // Q, K [BH, N, d/16]; V [BH, Np/16, d]
+  const uint8_t* q_sf;
+  const uint8_t* k_sf;
+  const uint8_t* v_sf;
+  int Np;
 };
 
 cudaError_t launch_prep(const PlanArgs& a, cudaStream_t s);

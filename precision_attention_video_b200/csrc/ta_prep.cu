@@ -250,7 +250,8 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const PlanArgs a) {
       }
     }
     __syncthreads();
-    // ---- dequantised copy, coalesced ----
+    // ---- dequantised copy, coalesced (only where a tile path reads it) ----
+    if (deq_out != nullptr)
     for (int idx = tid; idx < R * (D / 8); idx += kThreads) {
       const int r = idx / (D / 8), c8 = idx % (D / 8);
       if (r < nrows)
