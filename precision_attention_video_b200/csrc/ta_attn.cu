@@ -8,19 +8,20 @@
 // walks the block's compacted tile list (full ascending, low ascending, then
 // the skipped blocks) with an online softmax:
 //
-//   warp 8      producer: TMA loads of the kept K / V tiles (bf16, or the
+//   warp 4S     producer: TMA loads of the kept K / V tiles (bf16, or the
 //               dequantised low copies) into a two-stage ring; for skipped
 //               blocks it gathers up to BK pooled rows kbar_b / vbar_b into a
 //               "pseudo-key" tile, so a skip chunk costs one tile of MMA for
 //               up to BK skipped blocks and never touches their K / V;
-//   warp 9      MMA issuer: tcgen05.mma kind::f16, S = Q K^T into a double-
+//   warp 4S+1   MMA issuer: tcgen05.mma kind::f16, S = Q K^T into a double-
 //               buffered TMEM accumulator, O += P V into a TMEM accumulator;
 //               completion is signalled with tcgen05.commit on mbarriers;
-//   warps 0-7   softmax: warps w and w+4 share TMEM lanes 32w..32w+31 (query
-//               rows) and split each row's columns in halves; the pair swaps
-//               its half-row maxima through shared memory and a 64-thread
-//               named barrier.  Each thread loads its half S row, keeps the
-//               running max m and its half of the sum l, forms
+//   warps 0..4S-1 softmax (S = min(d, BK)/32 column parts): the S warps with
+//               equal w%4 share TMEM lanes 32(w%4).. (query rows) and split
+//               each row's columns into S parts of 32; they swap their part
+//               maxima through shared memory and a named barrier.  Each thread
+//               loads its part of an S row, keeps the running max m and its
+//               part of the sum l, forms
 //               P' = 2^o exp(s - m'), rounds it as the tile's tier demands
 //               (bf16; e4m3; NVFP4 per 16 keys), rescales O in TMEM when m
 //               grows, and writes P' to shared memory as the A operand of PV.
@@ -39,10 +40,16 @@
 namespace ta {
 namespace {
 
-constexpr int kSoftmaxWarps = 8;  // warp w: rows 32*(w%4).., column half w/4
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+// Softmax warps: warp w owns TMEM lanes 32*(w%4).. (query rows) and column
+// part w/4 of those rows; kSplit parts per row (32 columns of S and of O each).
+template <int D, int BK>
+struct Roles {
+  static constexpr int kSplit = (D < BK ? D : BK) / 32;
+  static constexpr int kSoftmaxWarps = 4 * kSplit;
+  static constexpr int kProducerWarp = kSoftmaxWarps;
+  static constexpr int kMmaWarp = kSoftmaxWarps + 1;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+};
 
 enum TileKind { KIND_FULL = 0, KIND_LOW = 1, KIND_SKIP = 2 };
 
@@ -119,8 +126,8 @@ struct Smem {
   static constexpr int oBar = oP + kP;
   static constexpr int kBars = 16;
   static constexpr int oMisc = oBar + kBars * 8;
-  static constexpr int oXchg = oMisc + 64;  // float [2 slots][2 halves][128 rows]
-  static constexpr int kTotal = oXchg + 2 * 2 * 128 * 4;
+  static constexpr int oXchg = oMisc + 64;  // float [4 parts][128 rows]
+  static constexpr int kTotal = oXchg + 4 * 128 * 4;
   static constexpr int kAlloc = kTotal;  // the base is checked for 1024-byte alignment
   static constexpr uint32_t kTmemCols = (2 * BK + D) <= 256 ? 256u : 512u;
 };
@@ -162,13 +169,16 @@ __device__ __forceinline__ void gather_row_sf(unsigned char* dst, const uint8_t*
 }
 
 template <int D, int BK, bool FP4>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
     attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmQ,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
                 const __grid_constant__ CUtensorMap tmDV) {
   using L = Smem<D, BK>;
   using TS = TmemSf<D, BK>;
+  using RL = Roles<D, BK>;
+  constexpr int kSplit = RL::kSplit, kSoftmaxWarps = RL::kSoftmaxWarps;
+  constexpr int kProducerWarp = RL::kProducerWarp, kMmaWarp = RL::kMmaWarp;
   static_assert(!FP4 || (D == 128 && BK == 128), "native NVFP4 tiles need d = 128, 128-key tiles");
   constexpr uint32_t kTmemCols = FP4 ? 512u : L::kTmemCols;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -211,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[BAR_E1], 1);
     mbar_init(&bars[BAR_S0], 1);
     mbar_init(&bars[BAR_S1], 1);
-    mbar_init(&bars[BAR_P], 2 * a.bq);  // both column halves of every live row
+    mbar_init(&bars[BAR_P], kSplit * a.bq);  // every column part of every live row
     mbar_init(&bars[BAR_O], 1);
     mbar_init(&bars[BAR_DRAIN], 1);
     fence_mbar_init();
@@ -456,16 +466,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kSoftmaxWarps && (warp & 3) * 32 < a.bq) {
     // ===================== softmax warps =====================
-    constexpr int HB = BK / 2;              // columns per half row
-    constexpr int HD = D / 2;               // O columns per half row
-    const int quarter = warp & 3, half = warp >> 2;
+    constexpr int HB = BK / kSplit;         // S columns per thread
+    constexpr int HD = D / kSplit;          // O columns per thread
+    const int quarter = warp & 3, part = warp >> 2;
     const int r = quarter * 32 + lane;      // query row within the tile == TMEM lane
-    const int pair_bar = 1 + quarter;       // named barrier of warps quarter, quarter+4
+    const int row_bar = 1 + quarter;        // named barrier of the warps sharing these rows
+    constexpr int kBarThreads = 32 * kSplit;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    float* xchg = reinterpret_cast<float*>(sm + L::oXchg);  // [slot][half][row]
+    float* xchg = reinterpret_cast<float*>(sm + L::oXchg);  // [part][row]
     const float c2 = a.scale_log2;           // S -> log2 units
     const float o_off = (float)a.p_offset;
-    float m = -INFINITY, l = 0.0f;           // running max (raw S units), half row sum
+    float m = -INFINITY, l = 0.0f;           // running max (raw S units), part row sum
     for (int t = 0; t < rp.T; ++t) {
       const int s = t & 1;
       bool ok = mbar_wait(&bars[BAR_S0 + s], (t >> 1) & 1, ctx, 6);
@@ -478,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         nvalid = min(BK, a.N - rp.list[first] * BK);
       }
-      const int nv = min(max(nvalid - half * HB, 0), HB);  // valid columns of this half
+      const int nv = min(max(nvalid - part * HB, 0), HB);  // valid columns of this part
       float x[HB];
       float tmax = -INFINITY;
       if (ok) {
@@ -486,56 +497,58 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c0 = 0; c0 < HB; c0 += 32) {
           uint32_t raw[32];
-          tmem_ld32((s ? tS1 : tS0) + lane_off + half * HB + c0, raw);
+          tmem_ld32((s ? tS1 : tS0) + lane_off + part * HB + c0, raw);
 #pragma unroll
           for (int c = 0; c < 32; ++c) x[c0 + c] = __uint_as_float(raw[c]);
         }
-        if (nv == HB) {
+        if (nv < HB) {
 #pragma unroll
-          for (int c = 0; c < HB; ++c) tmax = fmaxf(tmax, x[c]);
-        } else {
-#pragma unroll
-          for (int c = 0; c < HB; ++c) {
+          for (int c = 0; c < HB; ++c)
             if (c >= nv) x[c] = -INFINITY;
-            tmax = fmaxf(tmax, x[c]);
-          }
         }
-        xchg[(s * 2 + half) * 128 + r] = tmax;
+        float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < HB; ++c) pm[c & 3] = fmaxf(pm[c & 3], x[c]);
+        tmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+        xchg[part * 128 + r] = tmax;
       }
-      // swap half-row maxima with the partner warp; leave together on abort
-      ok = bar_and(pair_bar, 64, ok);
+      // swap part maxima with the warps sharing these rows; leave together on abort
+      ok = bar_and(row_bar, kBarThreads, ok);
       if (!ok) { aborted = true; break; }
-      const float m_new = fmaxf(m, fmaxf(tmax, xchg[(s * 2 + (half ^ 1)) * 128 + r]));
+      float m_new = m;
+#pragma unroll
+      for (int q = 0; q < kSplit; ++q) m_new = fmaxf(m_new, xchg[q * 128 + r]);
       const float alpha = fast_exp2((m - m_new) * c2);  // 0 on the first tile
       const float mc = m_new * c2 - o_off;              // P' = 2^(s*c2 - mc)
-      float rowsum = 0.0f;
 #pragma unroll
       for (int c = 0; c < HB; ++c) x[c] = fast_exp2(fmaf(x[c], c2, -mc));
       if (kind == KIND_SKIP) {
 #pragma unroll
         for (int c = 0; c < HB; ++c) {
           if (c < nv) {
-            const int j = rp.list[first + half * HB + c];
+            const int j = rp.list[first + part * HB + c];
             x[c] *= (float)min(BK, a.N - j * BK);
           }
         }
       }
+      float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int c = 0; c < HB; ++c) rowsum += x[c];
-      l = l * alpha + rowsum;
+      for (int c = 0; c < HB; ++c) ps[c & 3] += x[c];
+      l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       m = m_new;
 
       // round P' as the tier demands, into bf16 pairs (or NVFP4 codes)
       uint32_t p[HB / 2];
       if (FP4 && kind == KIND_LOW) {
-        // codes of this half row (64 keys = one MMA K chunk) packed in p[0..7],
-        // ue4m3 scales of its 4 groups in p[8]
+        // codes of this part (HB = 32 keys, half an MMA K chunk) in p[0..3],
+        // ue4m3 scales of its 2 groups in p[4]
         uint32_t scw = 0u;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          float amax = 0.0f;
+        for (int g = 0; g < HB / 16; ++g) {
+          float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-          for (int i = 0; i < 16; ++i) amax = fmaxf(amax, x[g * 16 + i]);
+          for (int i = 0; i < 16; ++i) am[i & 3] = fmaxf(am[i & 3], x[g * 16 + i]);
+          const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
           const uint32_t scc = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xFFu;
           const float sc = e4m3_to_float(scc);
           const float inv = (sc > 0.0f) ? __frcp_rn(sc) : 0.0f;
@@ -551,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             p[g * 2 + w] = word;
           }
         }
-        p[8] = scw;
+        p[HB / 8] = scw;
       } else if (kind == KIND_LOW && a.low == TA_LOW_FP8_E4M3) {
 #pragma unroll
         for (int c = 0; c < HB; c += 2) {
@@ -580,41 +593,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < HB; c += 2) p[c / 2] = pack_bf16(x[c], x[c + 1]);
       }
 
-      // PV of the previous tile must be done before P and O are touched
-      if (t > 0) {
-        bool ok2 = mbar_wait(&bars[BAR_O], (t - 1) & 1, ctx, 7);
-        ok2 = __all_sync(0xffffffffu, ok2);
-        ok2 = bar_and(pair_bar, 64, ok2);
+      // PV of the previous tile must be done before P and O are touched; the
+      // row barrier also orders this tile's reads of xchg before the next
+      // tile's writes
+      {
+        bool ok2 = true;
+        if (t > 0) {
+          ok2 = mbar_wait(&bars[BAR_O], (t - 1) & 1, ctx, 7);
+          ok2 = __all_sync(0xffffffffu, ok2);
+        }
+        ok2 = bar_and(row_bar, kBarThreads, ok2);
         if (!ok2) { aborted = true; break; }
+      }
+      if (t > 0) {
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
           for (int c0 = 0; c0 < HD; c0 += 32) {
             uint32_t raw[32];
-            tmem_ld32(tO + lane_off + half * HD + c0, raw);
+            tmem_ld32(tO + lane_off + part * HD + c0, raw);
 #pragma unroll
             for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * alpha);
-            tmem_st32(tO + lane_off + half * HD + c0, raw);
+            tmem_st32(tO + lane_off + part * HD + c0, raw);
           }
           tmem_wait_st();
         }
       }
       if (FP4 && kind == KIND_LOW) {
-        // NVFP4 P row half: 32 bytes of codes into the 64-byte-swizzled tile,
-        // 4 scale bytes into the scale-factor block of K chunk `half`
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int ch = half * 2 + q;
+        // NVFP4 P part: 16 bytes of codes into the 64-byte-swizzled tile, 2
+        // scale bytes into the scale-factor block of K chunk part/2
+        {
+          const int ch = part;
           const uint32_t off = r * 64 + ((ch ^ ((r >> 1) & 3)) * 16);
-          *reinterpret_cast<uint4*>(sm + L::oP + off) =
-              make_uint4(p[q * 4 + 0], p[q * 4 + 1], p[q * 4 + 2], p[q * 4 + 3]);
+          *reinterpret_cast<uint4*>(sm + L::oP + off) = make_uint4(p[0], p[1], p[2], p[3]);
         }
-        *reinterpret_cast<uint32_t*>(sm + L::oP + kFp4Sf + half * 512 + lane * 16 + quarter * 4) = p[8];
+        *reinterpret_cast<uint16_t*>(sm + L::oP + kFp4Sf + (part >> 1) * 512 + lane * 16 +
+                                     quarter * 4 + (part & 1) * 2) = (uint16_t)p[HB / 8];
       } else {
-        // this half of the P row -> shared memory, K-major, 128-byte swizzle
+        // this part of the P row -> shared memory, K-major, 128-byte swizzle
 #pragma unroll
         for (int q = 0; q < HB / 8; ++q) {
-          const int ch = half * (HB / 8) + q;    // 16-byte chunk index within the row
+          const int ch = part * (HB / 8) + q;    // 16-byte chunk index within the row
           const uint32_t off = (ch >> 3) * (128 * 128) + r * 128 + (((ch & 7) ^ (r & 7)) * 16);
           *reinterpret_cast<uint4*>(sm + L::oP + off) =
               make_uint4(p[q * 4 + 0], p[q * 4 + 1], p[q * 4 + 2], p[q * 4 + 3]);
@@ -627,21 +646,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!aborted) {
       bool ok = mbar_wait(&bars[BAR_O], (rp.T - 1) & 1, ctx, 8);
       ok = __all_sync(0xffffffffu, ok);
-      // row sums go to the slot the last tile did not use (free since the
-      // pair's barrier of tile T-1)
-      const int ls = rp.T & 1;
-      xchg[(ls * 2 + half) * 128 + r] = l;
-      ok = bar_and(pair_bar, 64, ok);
+      // row sums through the exchange slots: free since the last tile's second
+      // row barrier
+      xchg[part * 128 + r] = l;
+      ok = bar_and(row_bar, kBarThreads, ok);
       if (ok) {
         tc_fence_after();
-        const float inv_l = 1.0f / (l + xchg[(ls * 2 + (half ^ 1)) * 128 + r]);
+        float lt = 0.0f;
+#pragma unroll
+        for (int q = 0; q < kSplit; ++q) lt += xchg[q * 128 + r];
+        const float inv_l = 1.0f / lt;
         const bool valid = (q0 + r) < a.N;
         __nv_bfloat16* orow = a.O + (int64_t)b * a.sb + (int64_t)h * a.sh + (int64_t)(q0 + r) * a.sn +
-                              half * HD;
+                              part * HD;
 #pragma unroll
         for (int c0 = 0; c0 < HD; c0 += 32) {
           uint32_t raw[32];
-          tmem_ld32(tO + lane_off + half * HD + c0, raw);
+          tmem_ld32(tO + lane_off + part * HD + c0, raw);
           uint32_t w[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2)
@@ -673,7 +694,8 @@ cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s)
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nQb, a.B * a.H);
-  k<<<grid, kThreads, L::kAlloc, s>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5]);
+  k<<<grid, Roles<D, BK>::kThreads, L::kAlloc, s>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                   maps[5]);
   return cudaGetLastError();
 }
 
