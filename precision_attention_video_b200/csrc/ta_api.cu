@@ -8,10 +8,6 @@
 #include "ta_common.cuh"
 #include "ta_kernels.cuh"
 
-namespace ta {
-int attn_smem_bytes(int d, int bk);
-}
-
 namespace {
 
 constexpr size_t kAlign = 256;

@@ -24,7 +24,12 @@
 //               part of the sum l, forms
 //               P' = 2^o exp(s - m'), rounds it as the tile's tier demands
 //               (bf16; e4m3; NVFP4 per 16 keys), rescales O in TMEM when m
-//               grows, and writes P' to shared memory as the A operand of PV.
+//               grows, and hands P' to the PV MMA: bf16 P' is stored into the
+//               TMEM columns of its own S buffer (the A operand of a TMEM x
+//               shared-memory MMA), so the two S buffers double as two P
+//               buffers; NVFP4 P' (codes + scales) goes to one of two small
+//               shared-memory buffers.  A tile's softmax waits for the previous
+//               tile's PV only when it must rescale O.
 //               The epilogue writes O = acc / l in bf16.
 //
 // Low tiles run through the same bf16 tensor-core path on the exact bf16
@@ -111,11 +116,12 @@ __device__ __forceinline__ __half2 e2m1x2_to_half2(uint32_t codes) {
 }
 
 // Shared-memory layout (offsets from a 1024-aligned base).
-template <int D, int BK>
+template <int D, int BK, bool FP4>
 struct Smem {
   static constexpr int kQ = 128 * D * 2;      // one query tile, 128 rows
   static constexpr int kKV = BK * D * 2;      // one K or V tile
-  static constexpr int kP = 128 * BK * 2;     // P tile
+  static constexpr int kPfp4 = 128 * 64 + 1024;  // one NVFP4 P tile: codes + scales
+  static constexpr int kP = FP4 ? 2 * kPfp4 : 0;  // bf16 P lives in TMEM
   static constexpr int oQ = 0;
   static constexpr int oDQ = oQ + kQ;
   static constexpr int oK0 = oDQ + kQ;
@@ -134,7 +140,7 @@ struct Smem {
 
 enum {
   BAR_Q = 0, BAR_K0 = 1, BAR_K1 = 2, BAR_V0 = 3, BAR_V1 = 4, BAR_E0 = 5, BAR_E1 = 6,
-  BAR_S0 = 7, BAR_S1 = 8, BAR_P = 9, BAR_O = 10, BAR_DRAIN = 11
+  BAR_S0 = 7, BAR_S1 = 8, BAR_P = 9, BAR_PD0 = 10, BAR_PD1 = 11, BAR_DRAIN = 12
 };
 
 // TMEM columns of the NVFP4 scale factors (4 columns per 64-element K chunk,
@@ -144,7 +150,7 @@ struct TmemSf {
   static constexpr uint32_t kSfaQ = 2 * BK + D;
   static constexpr uint32_t kSfbK0 = kSfaQ + 8, kSfbK1 = kSfaQ + 16;
   static constexpr uint32_t kSfbV0 = kSfaQ + 24, kSfbV1 = kSfaQ + 32;
-  static constexpr uint32_t kSfaP = kSfaQ + 40;  // last block ends at kSfaQ + 48 <= 512
+  static constexpr uint32_t kSfaP0 = kSfaQ + 40, kSfaP1 = kSfaQ + 48;  // ends at +56 <= 512
 };
 
 // NVFP4 tiles in shared memory: codes [rows][64 B] with 64-byte swizzle, then
@@ -174,7 +180,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
                 const __grid_constant__ CUtensorMap tmDV) {
-  using L = Smem<D, BK>;
+  using L = Smem<D, BK, FP4>;
   using TS = TmemSf<D, BK>;
   using RL = Roles<D, BK>;
   constexpr int kSplit = RL::kSplit, kSoftmaxWarps = RL::kSoftmaxWarps;
@@ -222,12 +228,13 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
     mbar_init(&bars[BAR_S0], 1);
     mbar_init(&bars[BAR_S1], 1);
     mbar_init(&bars[BAR_P], kSplit * a.bq);  // every column part of every live row
-    mbar_init(&bars[BAR_O], 1);
+    mbar_init(&bars[BAR_PD0], 1);
+    mbar_init(&bars[BAR_PD1], 1);
     mbar_init(&bars[BAR_DRAIN], 1);
     fence_mbar_init();
   }
   if (warp < 4) {
-    // Rows >= bq of the query tiles and of P stay zero for the whole kernel.
+    // Rows >= bq of the query tiles stay zero for the whole kernel.
     const int r = threadIdx.x;
     if (r >= a.bq) {
       for (int c = 0; c < (D * 2) / 16; ++c) {
@@ -236,11 +243,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         *reinterpret_cast<uint4*>(sm + L::oQ + off) = make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(sm + L::oDQ + off) = make_uint4(0, 0, 0, 0);
       }
-      for (int c = 0; c < (BK * 2) / 16; ++c) {
-        const int box = c / 8, ch = c % 8;
-        const uint32_t off = box * (128 * 128) + r * 128 + ((ch ^ (r & 7)) * 16);
-        *reinterpret_cast<uint4*>(sm + L::oP + off) = make_uint4(0, 0, 0, 0);
-      }
+      // (rows >= bq of S, and so of the P aliased onto it, are exact zeros)
       fence_proxy_async_smem();
     }
   }
@@ -389,7 +392,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
       constexpr uint32_t idesc_qk = idesc_bf16(128, BK, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, true);
       const uint32_t sQ = smem_u32(sm + L::oQ), sDQ = smem_u32(sm + L::oDQ);
-      const uint32_t sP = smem_u32(sm + L::oP);
+      const uint32_t sP = smem_u32(sm + L::oP);  // NVFP4 P buffers
       auto issue_s = [&](int t) -> bool {
         const int s = t & 1;
         if (!mbar_wait(&bars[BAR_K0 + s], (t >> 1) & 1, ctx, 2)) return false;
@@ -438,24 +441,27 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         tile_of<BK>(rp, t, kind_t, first_t);
         if (FP4 && kind_t == KIND_LOW) {
           const uint32_t sfb = tmem + (s ? TS::kSfbV1 : TS::kSfbV0);
-          tc_cp_sf(tmem + TS::kSfaP, smem_desc_rows16(sP + kFp4Sf));
-          tc_cp_sf(tmem + TS::kSfaP + 4, smem_desc_rows16(sP + kFp4Sf + 512));
+          const uint32_t sfa = tmem + (s ? TS::kSfaP1 : TS::kSfaP0);
+          const uint32_t pb = sP + s * L::kPfp4;
+          tc_cp_sf(sfa, smem_desc_rows16(pb + kFp4Sf));
+          tc_cp_sf(sfa + 4, smem_desc_rows16(pb + kFp4Sf + 512));
           tc_cp_sf(sfb, smem_desc_rows16(sv + kFp4Sf));
           tc_cp_sf(sfb + 4, smem_desc_rows16(sv + kFp4Sf + 512));
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            mma_nvfp4_ss(tO, smem_desc_sw64(sP + kk * 32), smem_desc_sw64(sv + kk * 32),
-                         idesc_nvfp4(128, D), tmem + TS::kSfaP + kk * 4, sfb + kk * 4,
+            mma_nvfp4_ss(tO, smem_desc_sw64(pb + kk * 32), smem_desc_sw64(sv + kk * 32),
+                         idesc_nvfp4(128, D), sfa + kk * 4, sfb + kk * 4,
                          (t > 0 || kk > 0) ? 1u : 0u);
         } else {
+          // A = bf16 P' in the TMEM columns of this tile's S buffer
+          const uint32_t pa = s ? tS1 : tS0;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(sP + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
             const uint64_t bd = smem_desc_sw128(sv + kk * 16 * 128, BK * 128, 1024);
-            mma_f16_ss(tO, ad, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+            mma_f16_ts(tO, pa + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        tc_commit(&bars[BAR_O]);
+        tc_commit(&bars[BAR_PD0 + s]);
         tc_commit(&bars[BAR_E0 + s]);
       }
       if (!ok) {
@@ -593,58 +599,57 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         for (int c = 0; c < HB; c += 2) p[c / 2] = pack_bf16(x[c], x[c + 1]);
       }
 
-      // PV of the previous tile must be done before P and O are touched; the
+      // O may be rescaled only once the previous tile's PV is done; an NVFP4
+      // P buffer may be rewritten once the PV two tiles back is done.  The
       // row barrier also orders this tile's reads of xchg before the next
-      // tile's writes
+      // tile's writes, and makes the warps of a row leave together on abort.
+      const bool rescale = (t > 0) && __any_sync(0xffffffffu, alpha != 1.0f);
       {
         bool ok2 = true;
-        if (t > 0) {
-          ok2 = mbar_wait(&bars[BAR_O], (t - 1) & 1, ctx, 7);
-          ok2 = __all_sync(0xffffffffu, ok2);
-        }
+        if (FP4 && kind == KIND_LOW && t >= 2)
+          ok2 = mbar_wait(&bars[BAR_PD0 + s], ((t >> 1) - 1) & 1, ctx, 7);
+        if (rescale && ok2)
+          ok2 = mbar_wait(&bars[BAR_PD0 + (s ^ 1)], ((t - 1) >> 1) & 1, ctx, 9);
+        ok2 = __all_sync(0xffffffffu, ok2);
         ok2 = bar_and(row_bar, kBarThreads, ok2);
         if (!ok2) { aborted = true; break; }
       }
-      if (t > 0) {
+      if (rescale) {
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
-          for (int c0 = 0; c0 < HD; c0 += 32) {
-            uint32_t raw[32];
-            tmem_ld32(tO + lane_off + part * HD + c0, raw);
+        for (int c0 = 0; c0 < HD; c0 += 32) {
+          uint32_t raw[32];
+          tmem_ld32(tO + lane_off + part * HD + c0, raw);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * alpha);
-            tmem_st32(tO + lane_off + part * HD + c0, raw);
-          }
-          tmem_wait_st();
+          for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * alpha);
+          tmem_st32(tO + lane_off + part * HD + c0, raw);
         }
       }
       if (FP4 && kind == KIND_LOW) {
         // NVFP4 P part: 16 bytes of codes into the 64-byte-swizzled tile, 2
         // scale bytes into the scale-factor block of K chunk part/2
+        unsigned char* pbuf = sm + L::oP + s * L::kPfp4;
         {
           const int ch = part;
           const uint32_t off = r * 64 + ((ch ^ ((r >> 1) & 3)) * 16);
-          *reinterpret_cast<uint4*>(sm + L::oP + off) = make_uint4(p[0], p[1], p[2], p[3]);
+          *reinterpret_cast<uint4*>(pbuf + off) = make_uint4(p[0], p[1], p[2], p[3]);
         }
-        *reinterpret_cast<uint16_t*>(sm + L::oP + kFp4Sf + (part >> 1) * 512 + lane * 16 +
-                                     quarter * 4 + (part & 1) * 2) = (uint16_t)p[HB / 8];
+        *reinterpret_cast<uint16_t*>(pbuf + kFp4Sf + (part >> 1) * 512 + lane * 16 + quarter * 4 +
+                                     (part & 1) * 2) = (uint16_t)p[HB / 8];
       } else {
-        // this part of the P row -> shared memory, K-major, 128-byte swizzle
+        // bf16 P' of this part into the S buffer's first BK/2 columns (every
+        // part has loaded its S columns before the row barrier above)
 #pragma unroll
-        for (int q = 0; q < HB / 8; ++q) {
-          const int ch = part * (HB / 8) + q;    // 16-byte chunk index within the row
-          const uint32_t off = (ch >> 3) * (128 * 128) + r * 128 + (((ch & 7) ^ (r & 7)) * 16);
-          *reinterpret_cast<uint4*>(sm + L::oP + off) =
-              make_uint4(p[q * 4 + 0], p[q * 4 + 1], p[q * 4 + 2], p[q * 4 + 3]);
-        }
+        for (int q = 0; q < HB / 2; q += 16)
+          tmem_st16((s ? tS1 : tS0) + lane_off + part * (HB / 2) + q, p + q);
       }
+      tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[BAR_P]);
     }
     if (!aborted) {
-      bool ok = mbar_wait(&bars[BAR_O], (rp.T - 1) & 1, ctx, 8);
+      bool ok = mbar_wait(&bars[BAR_PD0 + ((rp.T - 1) & 1)], ((rp.T - 1) >> 1) & 1, ctx, 8);
       ok = __all_sync(0xffffffffu, ok);
       // row sums through the exchange slots: free since the last tile's second
       // row barrier
@@ -689,7 +694,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
 
 template <int D, int BK, bool FP4>
 cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
-  using L = Smem<D, BK>;
+  using L = Smem<D, BK, FP4>;
   auto k = attn_kernel<D, BK, FP4>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
@@ -700,13 +705,6 @@ cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s)
 }
 
 }  // namespace
-
-int attn_smem_bytes(int d, int bk) {
-  if (d == 64 && bk == 64) return Smem<64, 64>::kAlloc;
-  if (d == 64 && bk == 128) return Smem<64, 128>::kAlloc;
-  if (d == 128 && bk == 64) return Smem<128, 64>::kAlloc;
-  return Smem<128, 128>::kAlloc;
-}
 
 cudaError_t launch_attn(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
   if (a.d == 64 && a.bk == 64) return launch_d<64, 64, false>(a, maps, s);
