@@ -8,12 +8,14 @@
 // walks the block's compacted tile list (full ascending, low ascending, then
 // the skipped blocks) with an online softmax:
 //
-//   warp 4S     producer: TMA loads of the kept K / V tiles (bf16, or the
-//               dequantised low copies) into a two-stage ring; for skipped
-//               blocks it gathers up to BK pooled rows kbar_b / vbar_b into a
-//               "pseudo-key" tile, so a skip chunk costs one tile of MMA for
-//               up to BK skipped blocks and never touches their K / V;
-//   warp 4S+1   MMA issuer: tcgen05.mma kind::f16, S = Q K^T into a double-
+//   warps 4S, 4S+1  producers of K and of V: TMA loads of the kept tiles
+//               (bf16, or the low copies) into two two-stage rings; a K stage
+//               is released as soon as its S = Q K^T is done, a V stage after
+//               its PV.  For skipped blocks they gather up to BK pooled rows
+//               kbar_b / vbar_b into a "pseudo-key" tile, so a skip chunk costs
+//               one tile of MMA for up to BK skipped blocks and never touches
+//               their K / V;
+//   warp 4S+2   MMA issuer: tcgen05.mma kind::f16, S = Q K^T into a double-
 //               buffered TMEM accumulator, O += P V into a TMEM accumulator;
 //               completion is signalled with tcgen05.commit on mbarriers;
 //   warps 0..4S-1 softmax (S = min(d, BK)/32 column parts): the S warps with
@@ -51,9 +53,10 @@ template <int D, int BK>
 struct Roles {
   static constexpr int kSplit = (D < BK ? D : BK) / 32;
   static constexpr int kSoftmaxWarps = 4 * kSplit;
-  static constexpr int kProducerWarp = kSoftmaxWarps;
-  static constexpr int kMmaWarp = kSoftmaxWarps + 1;
-  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+  static constexpr int kProducerKWarp = kSoftmaxWarps;      // Q and K tiles
+  static constexpr int kProducerVWarp = kSoftmaxWarps + 1;  // V tiles
+  static constexpr int kMmaWarp = kSoftmaxWarps + 2;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
 };
 
 enum TileKind { KIND_FULL = 0, KIND_LOW = 1, KIND_SKIP = 2 };
@@ -139,8 +142,9 @@ struct Smem {
 };
 
 enum {
-  BAR_Q = 0, BAR_K0 = 1, BAR_K1 = 2, BAR_V0 = 3, BAR_V1 = 4, BAR_E0 = 5, BAR_E1 = 6,
-  BAR_S0 = 7, BAR_S1 = 8, BAR_P = 9, BAR_PD0 = 10, BAR_PD1 = 11, BAR_DRAIN = 12
+  BAR_Q = 0, BAR_K0 = 1, BAR_K1 = 2, BAR_V0 = 3, BAR_V1 = 4, BAR_KE0 = 5, BAR_KE1 = 6,
+  BAR_S0 = 7, BAR_S1 = 8, BAR_P = 9, BAR_PD0 = 10, BAR_PD1 = 11, BAR_DRAIN = 12,
+  BAR_VE0 = 13, BAR_VE1 = 14
 };
 
 // TMEM columns of the NVFP4 scale factors (4 columns per 64-element K chunk,
@@ -184,7 +188,8 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
   using TS = TmemSf<D, BK>;
   using RL = Roles<D, BK>;
   constexpr int kSplit = RL::kSplit, kSoftmaxWarps = RL::kSoftmaxWarps;
-  constexpr int kProducerWarp = RL::kProducerWarp, kMmaWarp = RL::kMmaWarp;
+  constexpr int kProducerKWarp = RL::kProducerKWarp, kProducerVWarp = RL::kProducerVWarp;
+  constexpr int kMmaWarp = RL::kMmaWarp;
   static_assert(!FP4 || (D == 128 && BK == 128), "native NVFP4 tiles need d = 128, 128-key tiles");
   constexpr uint32_t kTmemCols = FP4 ? 512u : L::kTmemCols;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -223,8 +228,10 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
     mbar_init(&bars[BAR_K1], 1);
     mbar_init(&bars[BAR_V0], 1);
     mbar_init(&bars[BAR_V1], 1);
-    mbar_init(&bars[BAR_E0], 1);
-    mbar_init(&bars[BAR_E1], 1);
+    mbar_init(&bars[BAR_KE0], 1);
+    mbar_init(&bars[BAR_KE1], 1);
+    mbar_init(&bars[BAR_VE0], 1);
+    mbar_init(&bars[BAR_VE1], 1);
     mbar_init(&bars[BAR_S0], 1);
     mbar_init(&bars[BAR_S1], 1);
     mbar_init(&bars[BAR_P], kSplit * a.bq);  // every column part of every live row
@@ -259,132 +266,128 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
 
   bool aborted = false;
 
-  if (warp == kProducerWarp) {
-    // ===================== producer =====================
-    int kf_issued[2] = {0, 0}, vf_issued[2] = {0, 0};
-    if (FP4 && has_low) {
-      // scales of the NVFP4 query copy, ready for tcgen05.cp
-      gather_row_sf(sm + L::oDQ + kFp4Sf, a.q_sf + ((int64_t)bh * a.N + q0) * 8,
-                    min(128, a.N - q0), lane);
-      fence_proxy_async_smem();
-      __syncwarp();
-    }
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      const uint32_t qbytes = (uint32_t)a.bq * D * 2;
-      const uint32_t lbytes = FP4 ? (uint32_t)a.bq * 64 : qbytes;
-      mbar_arrive_expect_tx(&bars[BAR_Q], has_low ? qbytes + lbytes : qbytes);
-      for (int x = 0; x < D / 64; ++x)
-        tma_load_4d(sm + L::oQ + x * (128 * 128), &tmQ, &bars[BAR_Q], x * 64, q0, h, b);
-      if (has_low) {
-        if (FP4) {
-          tma_load_3d(sm + L::oDQ, &tmDQ, &bars[BAR_Q], 0, q0, bh);
-        } else {
-          for (int x = 0; x < D / 64; ++x)
-            tma_load_4d(sm + L::oDQ + x * (128 * 128), &tmDQ, &bars[BAR_Q], x * 64, q0, h, b);
+  if (warp == kProducerKWarp || warp == kProducerVWarp) {
+    // ===================== producers (K ring / V ring) =====================
+    const bool isK = (warp == kProducerKWarp);
+    int issued[2] = {0, 0};   // loads (or gathers) signalled per stage barrier
+    uint64_t* full = &bars[isK ? BAR_K0 : BAR_V0];
+    uint64_t* empty = &bars[isK ? BAR_KE0 : BAR_VE0];
+    if (isK) {
+      if (FP4 && has_low) {
+        // scales of the NVFP4 query copy, ready for tcgen05.cp
+        gather_row_sf(sm + L::oDQ + kFp4Sf, a.q_sf + ((int64_t)bh * a.N + q0) * 8,
+                      min(128, a.N - q0), lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        const uint32_t qbytes = (uint32_t)a.bq * D * 2;
+        const uint32_t lbytes = FP4 ? (uint32_t)a.bq * 64 : qbytes;
+        mbar_arrive_expect_tx(&bars[BAR_Q], has_low ? qbytes + lbytes : qbytes);
+        for (int x = 0; x < D / 64; ++x)
+          tma_load_4d(sm + L::oQ + x * (128 * 128), &tmQ, &bars[BAR_Q], x * 64, q0, h, b);
+        if (has_low) {
+          if (FP4) {
+            tma_load_3d(sm + L::oDQ, &tmDQ, &bars[BAR_Q], 0, q0, bh);
+          } else {
+            for (int x = 0; x < D / 64; ++x)
+              tma_load_4d(sm + L::oDQ + x * (128 * 128), &tmDQ, &bars[BAR_Q], x * 64, q0, h, b);
+          }
         }
       }
+    } else if (lane == 0) {
+      tma_prefetch_desc(&tmV);
     }
-    const __nv_bfloat16* kbar = a.kbar_b + (int64_t)bh * a.nKb * D;
-    const __nv_bfloat16* vbar = a.vbar_b + (int64_t)bh * a.nKb * D;
+    // pooled rows for skip chunks: kbar_b for the K ring, vbar_b for the V ring
+    const __nv_bfloat16* pooled = (isK ? a.kbar_b : a.vbar_b) + (int64_t)bh * a.nKb * D;
     for (int t = 0; t < rp.T; ++t) {
       const int s = t & 1;
       if (t >= 2) {
         bool ok = true;
-        if (lane == 0) ok = mbar_wait(&bars[BAR_E0 + s], ((t >> 1) - 1) & 1, ctx, 1);
+        if (lane == 0) ok = mbar_wait(&empty[s], ((t >> 1) - 1) & 1, ctx, isK ? 1 : 10);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) { aborted = true; break; }
       }
       int kind, first;
       tile_of<BK>(rp, t, kind, first);
-      unsigned char* kst = sm + (s ? L::oK1 : L::oK0);
-      unsigned char* vst = sm + (s ? L::oV1 : L::oV0);
+      unsigned char* st = sm + (isK ? (s ? L::oK1 : L::oK0) : (s ? L::oV1 : L::oV0));
       if (FP4 && kind == KIND_LOW) {
         const int j = rp.list[first];
-        // K scales (rows of the key tile) and V scales (groups of 16 keys of
-        // each d row) into the stage, in the tcgen05.cp block layout
-        gather_row_sf(kst + kFp4Sf, a.k_sf + ((int64_t)bh * a.N + j * BK) * 8,
-                      min(BK, a.N - j * BK), lane);
-        const int ng = a.Np / 16;
+        if (isK) {
+          // K scales (rows of the key tile) in the tcgen05.cp block layout
+          gather_row_sf(st + kFp4Sf, a.k_sf + ((int64_t)bh * a.N + j * BK) * 8,
+                        min(BK, a.N - j * BK), lane);
+        } else {
+          // V scales: groups of 16 keys of each d row of V^T
+          const int ng = a.Np / 16;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < 2; ++c) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int g = j * 8 + c * 4 + k;   // group of 16 keys
-            uint32_t w = 0u;
-            if (g < ng) w = *reinterpret_cast<const uint32_t*>(a.v_sf + ((int64_t)bh * ng + g) * D + lane * 4);
+            for (int k = 0; k < 4; ++k) {
+              const int g = j * 8 + c * 4 + k;   // group of 16 keys
+              uint32_t w = 0u;
+              if (g < ng)
+                w = *reinterpret_cast<const uint32_t*>(a.v_sf + ((int64_t)bh * ng + g) * D + lane * 4);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int m = lane * 4 + i;        // d row of V^T
-              vst[kFp4Sf + c * 512 + (m & 31) * 16 + (m >> 5) * 4 + k] = (unsigned char)(w >> (8 * i));
+              for (int i = 0; i < 4; ++i) {
+                const int m = lane * 4 + i;        // d row of V^T
+                st[kFp4Sf + c * 512 + (m & 31) * 16 + (m >> 5) * 4 + k] = (unsigned char)(w >> (8 * i));
+              }
             }
           }
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          const bool drop = (t == 0) && (a.debug_flags & TA_DEBUG_DROP_FIRST_K);
+          const bool drop = isK && (t == 0) && (a.debug_flags & TA_DEBUG_DROP_FIRST_K);
           if (!drop) {
-            mbar_arrive_expect_tx(&bars[BAR_K0 + s], BK * 64);
-            tma_load_3d(kst, &tmDK, &bars[BAR_K0 + s], 0, j * BK, bh);
-            kf_issued[s]++;
+            mbar_arrive_expect_tx(&full[s], (isK ? BK : D) * 64);
+            if (isK)
+              tma_load_3d(st, &tmDK, &full[s], 0, j * BK, bh);
+            else
+              tma_load_3d(st, &tmDV, &full[s], j * 64, 0, bh);
+            issued[s]++;
           }
-          mbar_arrive_expect_tx(&bars[BAR_V0 + s], D * 64);
-          tma_load_3d(vst, &tmDV, &bars[BAR_V0 + s], j * 64, 0, bh);
-          vf_issued[s]++;
         }
       } else if (kind != KIND_SKIP) {
         if (lane == 0) {
           const int j = rp.list[first];
-          const CUtensorMap* mk = (kind == KIND_LOW) ? &tmDK : &tmK;
-          const CUtensorMap* mv = (kind == KIND_LOW) ? &tmDV : &tmV;
-          const bool drop = (t == 0) && (a.debug_flags & TA_DEBUG_DROP_FIRST_K);
+          const CUtensorMap* mp = isK ? ((kind == KIND_LOW) ? &tmDK : &tmK)
+                                      : ((kind == KIND_LOW) ? &tmDV : &tmV);
+          const bool drop = isK && (t == 0) && (a.debug_flags & TA_DEBUG_DROP_FIRST_K);
           if (!drop) {
-            mbar_arrive_expect_tx(&bars[BAR_K0 + s], BK * D * 2);
+            mbar_arrive_expect_tx(&full[s], BK * D * 2);
             for (int x = 0; x < D / 64; ++x)
-              tma_load_4d(kst + x * (BK * 128), mk, &bars[BAR_K0 + s], x * 64, j * BK, h, b);
-            kf_issued[s]++;
+              tma_load_4d(st + x * (BK * 128), mp, &full[s], x * 64, j * BK, h, b);
+            issued[s]++;
           }
-          mbar_arrive_expect_tx(&bars[BAR_V0 + s], BK * D * 2);
-          for (int x = 0; x < D / 64; ++x)
-            tma_load_4d(vst + x * (BK * 128), mv, &bars[BAR_V0 + s], x * 64, j * BK, h, b);
-          vf_issued[s]++;
         }
       } else {
-        // gather pooled rows of the skipped blocks into a pseudo K / V tile
+        // gather pooled rows of the skipped blocks into a pseudo K (or V) tile
         const int cnt = min(BK, rp.n_skip - (first - rp.n_full - rp.n_res - rp.n_low));
 #pragma unroll 8
         for (int e = lane; e < BK * (D / 8); e += 32) {
           const int c = e / (D / 8), ch = e % (D / 8);
-          uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
-          if (c < cnt) {
-            const int j = rp.list[first + c];
-            kv = *reinterpret_cast<const uint4*>(kbar + (int64_t)j * D + ch * 8);
-            vv = *reinterpret_cast<const uint4*>(vbar + (int64_t)j * D + ch * 8);
-          }
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (c < cnt) v = *reinterpret_cast<const uint4*>(pooled + (int64_t)rp.list[first + c] * D + ch * 8);
           const uint32_t off = (ch >> 3) * (BK * 128) + c * 128 + (((ch & 7) ^ (c & 7)) * 16);
-          *reinterpret_cast<uint4*>(kst + off) = kv;
-          *reinterpret_cast<uint4*>(vst + off) = vv;
+          *reinterpret_cast<uint4*>(st + off) = v;
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&bars[BAR_K0 + s]);
-          mbar_arrive(&bars[BAR_V0 + s]);
-          kf_issued[s]++;
-          vf_issued[s]++;
+          mbar_arrive(&full[s]);
+          issued[s]++;
         }
       }
     }
     if (aborted && lane == 0) {
       // let copies already in flight land before the CTA goes away
-      for (int s = 0; s < 2; ++s) {
-        if (kf_issued[s] > 0) mbar_wait_drain(&bars[BAR_K0 + s], (kf_issued[s] - 1) & 1);
-        if (vf_issued[s] > 0) mbar_wait_drain(&bars[BAR_V0 + s], (vf_issued[s] - 1) & 1);
-      }
-      mbar_wait_drain(&bars[BAR_Q], 0);
+      for (int s = 0; s < 2; ++s)
+        if (issued[s] > 0) mbar_wait_drain(&full[s], (issued[s] - 1) & 1);
+      if (isK) mbar_wait_drain(&bars[BAR_Q], 0);
     }
   } else if (warp == kMmaWarp) {
     // ===================== MMA issuer =====================
@@ -419,6 +422,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           }
         }
         tc_commit(&bars[BAR_S0 + s]);
+        tc_commit(&bars[BAR_KE0 + s]);   // the K stage is free once S is done
         return true;
       };
       bool ok = mbar_wait(&bars[BAR_Q], 0, ctx, 3);
@@ -462,7 +466,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           }
         }
         tc_commit(&bars[BAR_PD0 + s]);
-        tc_commit(&bars[BAR_E0 + s]);
+        tc_commit(&bars[BAR_VE0 + s]);   // the V stage is free once PV is done
       }
       if (!ok) {
         aborted = true;
