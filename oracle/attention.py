@@ -11,7 +11,8 @@ that weight times vbar_j to the numerator.  Kept tiles are computed in bf16
 Per query block i (all its rows together; every row of a block shares the
 block's tile list), in fp64, starting from m = -inf, l = 0, acc = 0:
 
-* kept tiles in list order (full ascending, then residual, then low):
+* kept tiles in list order (full, then residual, then low; within a tier by
+  descending pooled mass, lower j first on ties):
     s      = logits of the tile's real keys from the tier's operands * scale
              full: bf16 Q . bf16 K;  low: deq(Q^) . deq(K^);
              residual: deq(Q1)deq(K1) + deq(Q1)deq(K2) + deq(Q2)deq(K1)
@@ -25,13 +26,14 @@ block's tile list), in fp64, starting from m = -inf, l = 0, acc = 0:
                                        NVFP4: nvfp4_16keys(P') deq(V^);
                                        residual: P1 V1 + P1 V2 + P2 V1 with
                                        P1 = nvfp4(P'), P2 = nvfp4(fp32(P' - P1))
-* skipped blocks, as one group:
+* skipped blocks, as one group (order immaterial):
     s_j = q . bf16(kbar_j) * scale;  m' = max(m, max_j s_j); rescale
     w_j = n_j 2^o exp(s_j - m');  l += sum w_j;  acc += bf16(w_j) bf16(vbar_j)
 * O = acc / l.
 
-Readings: the tier order (full, residual, low, skip) puts the running max near
-its final value before any P' is quantised; the denominator sums P' before
+Readings: the tier order (full, residual, low, skip) and the descending-mass
+order inside a tier put the running max near its final value before any P'
+is quantised; the denominator sums P' before
 quantisation; the skipped blocks of a row enter as one group with a single
 running-max update.  ``exact=True`` turns off every rounding of P' and w (the
 operand copies stay quantised); the pins use it.

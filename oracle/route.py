@@ -25,7 +25,9 @@ these at tile level:
 5. Flags.  A tile is flagged when |C_r - tau_t| <= 1e-5 tau_t for some t, or
    when it and a sort neighbour have |M - M'| <= 1e-5 max(M, M') and got
    different tiers from the prefix rule: only there may a GPU router differ.
-6. Lists.  Per row: full blocks ascending, then residual, then low, then skip.
+6. Lists.  Per row: full blocks, then residual, then low, then skip; within a
+   tier in the sort order of step 4, so a row meets its heaviest blocks (and,
+   nearly always, its largest logits) first.
 """
 
 from __future__ import annotations
@@ -105,9 +107,12 @@ def assign_tiers(M_row: np.ndarray, tau, diag=()):
     return tiers, flags
 
 
-def row_lists(tiers_row: np.ndarray):
-    """counts [full, res, low, skip] and the key-block list in that order, each ascending."""
-    groups = [np.nonzero(tiers_row == t)[0] for t in (TIER_FULL, TIER_RES, TIER_LOW, TIER_SKIP)]
+def row_lists(tiers_row: np.ndarray, M_row: np.ndarray):
+    """counts [full, res, low, skip] and the key-block list in that tier order;
+    within a tier, blocks follow the router's (-M, j) order (largest pooled
+    mass first, lower j first among equal masses)."""
+    order = np.lexsort((np.arange(len(M_row)), -M_row))
+    groups = [order[tiers_row[order] == t] for t in (TIER_FULL, TIER_RES, TIER_LOW, TIER_SKIP)]
     counts = np.array([len(g) for g in groups], dtype=np.int32)
     return counts, np.concatenate(groups).astype(np.int32)
 
@@ -130,7 +135,7 @@ def route_head(Qh, Kh, Vh, tau, block_q: int, block_k: int, scale: float = 0.0,
     for i in range(nqb):
         diag = diag_blocks(i, block_q, block_k, N) if keep_diag_full else ()
         tiers[i], flags[i] = assign_tiers(M[i], tau, diag)
-        counts[i], lists[i] = row_lists(tiers[i])
+        counts[i], lists[i] = row_lists(tiers[i], M[i])
     return {"qbar": qbar, "kbar": kbar, "vbar": vbar, "n_k": n_k, "M": M,
             "kbar_b": bf16_rne(kbar), "vbar_b": bf16_rne(vbar), "scale": scale,
             "tiers": tiers, "flags": flags, "counts": counts, "lists": lists}

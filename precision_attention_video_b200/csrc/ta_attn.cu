@@ -5,8 +5,8 @@
 // and skipped tiles replaced by their block means, so that block j of n_j keys
 // adds n_j exp(q . kbar_j * scale) to the softmax denominator and that weight
 // times vbar_j to the numerator.  One CTA owns one (head, query block) and
-// walks the block's compacted tile list (full ascending, low ascending, then
-// the skipped blocks) with an online softmax:
+// walks the block's compacted tile list (full tiles, then low tiles, each by
+// descending pooled mass, then the skipped blocks) with an online softmax:
 //
 //   warps 4S, 4S+1  producers of K and of V: TMA loads of the kept tiles
 //               (bf16, or the low copies) into two two-stage rings; a K stage
@@ -87,9 +87,50 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, to share the exponentials with the MUFU unit:
+// x = n + f with n = round(x) (adding 1.5 * 2^23 leaves round(x) in the low
+// mantissa bits) and f in [-0.5, 0.5]; 2^f from a degree-5 polynomial fitted
+// here for relative error (max 1.8e-7 on [-0.5, 0.5], evaluated in fp32); 2^n
+// added to the exponent field.  Inputs below -125 return 0; x <= 127.
+// Every kPolyEvery-th exponential of a softmax thread uses exp2_poly (0: none).
+// Measured on this kernel: a polynomial costs more issue slots than it saves
+// on the MUFU pipe, so it is off.
+constexpr int kPolyEvery = 0;
+
+[[maybe_unused]] __device__ __forceinline__ float exp2_poly(float x) {
+  const float xc = fmaxf(x, -125.0f);
+  const float t = xc + 12582912.0f;
+  const float n = t - 12582912.0f;
+  const float f = xc - n;
+  float p = 0.0013281889259815216f;
+  p = fmaf(p, f, 0.00967559777200222f);
+  p = fmaf(p, f, 0.05550696700811386f);
+  p = fmaf(p, f, 0.24022118747234344f);
+  p = fmaf(p, f, 0.6931470036506653f);
+  p = fmaf(p, f, 1.0000001192092896f);
+  const int ni = __float_as_int(t) - 0x4B400000;
+  const float r = __int_as_float(__float_as_int(p) + (ni << 23));
+  return x < -125.0f ? 0.0f : r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Eight floats to eight e2m1 codes (RNE, satfinite) in one word, element i in
+// nibble i.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return r;
 }
 
 // Named barrier over `count` threads that also ANDs a predicate across them:
@@ -135,8 +176,9 @@ struct Smem {
   static constexpr int oBar = oP + kP;
   static constexpr int kBars = 16;
   static constexpr int oMisc = oBar + kBars * 8;
-  static constexpr int oXchg = oMisc + 64;  // float [4 parts][128 rows]
-  static constexpr int kTotal = oXchg + 4 * 128 * 4;
+  static constexpr int oXchg = oMisc + 64;           // float [2 slots][4 parts][128 rows]
+  static constexpr int oScTab = oXchg + 2 * 4 * 128 * 4;  // float2 [128]: ue4m3 value, 1/value
+  static constexpr int kTotal = oScTab + 128 * 8;
   static constexpr int kAlloc = kTotal;  // the base is checked for 1024-byte alignment
   static constexpr uint32_t kTmemCols = (2 * BK + D) <= 256 ? 256u : 512u;
 };
@@ -239,6 +281,12 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
     mbar_init(&bars[BAR_PD1], 1);
     mbar_init(&bars[BAR_DRAIN], 1);
     fence_mbar_init();
+  }
+  if (FP4 && threadIdx.x < 128) {
+    // ue4m3 code -> (value, correctly rounded reciprocal) for P' quantisation
+    const float v = (threadIdx.x == 0x7F) ? 0.0f : e4m3_to_float(threadIdx.x);
+    reinterpret_cast<float2*>(sm + L::oScTab)[threadIdx.x] =
+        make_float2(v, v > 0.0f ? __frcp_rn(v) : 0.0f);
   }
   if (warp < 4) {
     // Rows >= bq of the query tiles stay zero for the whole kernel.
@@ -483,7 +531,8 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
     const int row_bar = 1 + quarter;        // named barrier of the warps sharing these rows
     constexpr int kBarThreads = 32 * kSplit;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    float* xchg = reinterpret_cast<float*>(sm + L::oXchg);  // [part][row]
+    float* xchg = reinterpret_cast<float*>(sm + L::oXchg);  // [slot][part][row]
+    const float2* sc_tab = reinterpret_cast<const float2*>(sm + L::oScTab);
     const float c2 = a.scale_log2;           // S -> log2 units
     const float o_off = (float)a.p_offset;
     float m = -INFINITY, l = 0.0f;           // running max (raw S units), part row sum
@@ -520,18 +569,26 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < HB; ++c) pm[c & 3] = fmaxf(pm[c & 3], x[c]);
         tmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
-        xchg[part * 128 + r] = tmax;
+        xchg[(s * 4 + part) * 128 + r] = tmax;
       }
       // swap part maxima with the warps sharing these rows; leave together on abort
       ok = bar_and(row_bar, kBarThreads, ok);
       if (!ok) { aborted = true; break; }
       float m_new = m;
 #pragma unroll
-      for (int q = 0; q < kSplit; ++q) m_new = fmaxf(m_new, xchg[q * 128 + r]);
+      for (int q = 0; q < kSplit; ++q) m_new = fmaxf(m_new, xchg[(s * 4 + q) * 128 + r]);
       const float alpha = fast_exp2((m - m_new) * c2);  // 0 on the first tile
       const float mc = m_new * c2 - o_off;              // P' = 2^(s*c2 - mc)
+      if constexpr (kPolyEvery > 0) {
 #pragma unroll
-      for (int c = 0; c < HB; ++c) x[c] = fast_exp2(fmaf(x[c], c2, -mc));
+        for (int c = 0; c < HB; ++c) {
+          const float e = fmaf(x[c], c2, -mc);
+          x[c] = (c % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) ? exp2_poly(e) : fast_exp2(e);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < HB; ++c) x[c] = fast_exp2(fmaf(x[c], c2, -mc));
+      }
       if (kind == KIND_SKIP) {
 #pragma unroll
         for (int c = 0; c < HB; ++c) {
@@ -560,18 +617,14 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           for (int i = 0; i < 16; ++i) am[i & 3] = fmaxf(am[i & 3], x[g * 16 + i]);
           const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
           const uint32_t scc = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xFFu;
-          const float sc = e4m3_to_float(scc);
-          const float inv = (sc > 0.0f) ? __frcp_rn(sc) : 0.0f;
+          const float inv = sc_tab[scc].y;
           scw |= scc << (8 * g);
 #pragma unroll
           for (int w = 0; w < 2; ++w) {
-            uint32_t word = 0u;
+            float y[8];
 #pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-              const int c = g * 16 + w * 8 + i;
-              word |= cvt_e2m1x2(__fmul_rn(x[c], inv), __fmul_rn(x[c + 1], inv)) << (4 * i);
-            }
-            p[g * 2 + w] = word;
+            for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(x[g * 16 + w * 8 + i], inv);
+            p[g * 2 + w] = cvt_e2m1x8(y);
           }
         }
         p[HB / 8] = scw;
@@ -604,14 +657,16 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
       }
 
       // O may be rescaled only once the previous tile's PV is done; an NVFP4
-      // P buffer may be rewritten once the PV two tiles back is done.  The
-      // row barrier also orders this tile's reads of xchg before the next
-      // tile's writes, and makes the warps of a row leave together on abort.
+      // P buffer may be rewritten once the PV two tiles back is done.  (The
+      // maxima exchange is double-buffered: a slot is rewritten two tiles on,
+      // after every reader has passed the next tile's row barrier.)
+      // The warps sharing these rows see the same maxima, so they agree on
+      // `rescale` and on `reuse` and wait (and leave on abort) together.
       const bool rescale = (t > 0) && __any_sync(0xffffffffu, alpha != 1.0f);
-      {
+      const bool reuse = FP4 && kind == KIND_LOW && t >= 2;
+      if (rescale || reuse) {
         bool ok2 = true;
-        if (FP4 && kind == KIND_LOW && t >= 2)
-          ok2 = mbar_wait(&bars[BAR_PD0 + s], ((t >> 1) - 1) & 1, ctx, 7);
+        if (reuse) ok2 = mbar_wait(&bars[BAR_PD0 + s], ((t >> 1) - 1) & 1, ctx, 7);
         if (rescale && ok2)
           ok2 = mbar_wait(&bars[BAR_PD0 + (s ^ 1)], ((t - 1) >> 1) & 1, ctx, 9);
         ok2 = __all_sync(0xffffffffu, ok2);
@@ -648,22 +703,23 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           tmem_st16((s ? tS1 : tS0) + lane_off + part * (HB / 2) + q, p + q);
       }
       tmem_wait_st();
-      fence_proxy_async_smem();
+      if (FP4 && kind == KIND_LOW) fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[BAR_P]);
     }
     if (!aborted) {
       bool ok = mbar_wait(&bars[BAR_PD0 + ((rp.T - 1) & 1)], ((rp.T - 1) >> 1) & 1, ctx, 8);
       ok = __all_sync(0xffffffffu, ok);
-      // row sums through the exchange slots: free since the last tile's second
-      // row barrier
-      xchg[part * 128 + r] = l;
+      // row sums through the exchange slot the last tile did not use (its
+      // last readers passed the last tile's row barrier)
+      const int ls = rp.T & 1;
+      xchg[(ls * 4 + part) * 128 + r] = l;
       ok = bar_and(row_bar, kBarThreads, ok);
       if (ok) {
         tc_fence_after();
         float lt = 0.0f;
 #pragma unroll
-        for (int q = 0; q < kSplit; ++q) lt += xchg[q * 128 + r];
+        for (int q = 0; q < kSplit; ++q) lt += xchg[(ls * 4 + q) * 128 + r];
         const float inv_l = 1.0f / lt;
         const bool valid = (q0 + r) < a.N;
         __nv_bfloat16* orow = a.O + (int64_t)b * a.sb + (int64_t)h * a.sh + (int64_t)(q0 + r) * a.sn +

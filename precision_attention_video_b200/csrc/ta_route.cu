@@ -11,7 +11,8 @@
 //   sort j by (-M_ij, j); C_r = exclusive prefix sum of the sorted masses;
 //   tier(rank r) = the most precise tier t with C_r < tau_t, else skip;
 //   key blocks meeting query block i's token range become full;
-//   list = full blocks ascending, then residual, low, skip (each ascending).
+//   list = full blocks, then residual, low, skip; within a tier in (-M, j)
+//   order, so a query block meets its heaviest key blocks first.
 // The router runs in fp64 end to end (means, logits, exp, prefix), so its
 // cumulative masses agree with an fp64 evaluation to ~1e-15 relative and the
 // tier map only depends on the ordering rule, not on rounding.
@@ -183,15 +184,16 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs 
   }
   __syncwarp();
 
-  // tier map row, counts and the compacted list
+  // tier map row, counts and the compacted list: tiers in the order full,
+  // res, low, skip; within a tier the blocks keep their (-M, j) rank order
   for (int j = lane; j < nKb; j += 32) a.tier_map[g * nKb + j] = tier[j];
   const int order[4] = {TA_TIER_FULL, TA_TIER_RES, TA_TIER_LOW, TA_TIER_SKIP};
   int base = 0;
   for (int q = 0; q < 4; ++q) {
     const int t = order[q];
     int cnt = 0;
-    for (int j0 = 0; j0 < nKb; j0 += 32) {
-      const int j = j0 + lane;
+    for (int r0 = 0; r0 < sortn; r0 += 32) {
+      const int j = idx[r0 + lane];
       const bool p = (j < nKb) && tier[j] == t;
       const unsigned bal = __ballot_sync(0xffffffffu, p);
       if (p) a.row_lists[g * nKb + base + cnt + __popc(bal & ((1u << lane) - 1u))] = j;

@@ -78,13 +78,15 @@ def compare_tiers(gpu_tiers: np.ndarray, rt: dict):
     return int(diff.sum()), set(np.nonzero(diff.any(axis=1))[0].tolist())
 
 
-def check_lists(tiers: np.ndarray, counts: np.ndarray, lists: np.ndarray):
-    """Each row's list is a permutation grouped full, res, low, skip, each ascending."""
+def check_lists(tiers: np.ndarray, counts: np.ndarray, lists: np.ndarray, mass: np.ndarray):
+    """Each row's list is a permutation grouped full, res, low, skip; within a
+    tier ordered by (-M, j) of the router's (GPU) masses."""
     order = [3, 2, 1, 0]
     for i in range(tiers.shape[0]):
         pos = 0
+        rank = np.lexsort((np.arange(tiers.shape[1]), -mass[i]))
         for q, t in enumerate(order):
-            want = np.nonzero(tiers[i] == t)[0]
+            want = rank[tiers[i][rank] == t]
             assert counts[i, q] == len(want), (i, t)
             np.testing.assert_array_equal(lists[i, pos:pos + len(want)], want)
             pos += len(want)

@@ -35,7 +35,11 @@ def _plan_parity(cfg, Q, K, V, views, heads):
         np.testing.assert_allclose(views["mass"][bh].numpy(), rt["M"], rtol=1e-10, atol=1e-15)
         tiers = views["tier_map"][bh].numpy()
         compare_tiers(tiers, rt)
-        check_lists(tiers, views["row_counts"][bh].numpy(), views["row_lists"][bh].numpy())
+        check_lists(tiers, views["row_counts"][bh].numpy(), views["row_lists"][bh].numpy(),
+                    views["mass"][bh].numpy())
+        # and equal to the oracle's lists wherever the tier rows agree
+        same = (tiers == rt["tiers"]).all(axis=1)
+        np.testing.assert_array_equal(views["row_lists"][bh].numpy()[same], rt["lists"][same])
         if cfg.low == Qz.LOW_FP8:
             for t in "qkv":
                 np.testing.assert_array_equal(views[f"{t}_codes"][bh].numpy(), qt[f"{t}_codes"])

@@ -107,9 +107,11 @@ def test_flags():
 
 def test_row_lists():
     tiers = np.array([0, 3, 1, 2, 3, 0, 1], dtype=np.uint8)
-    counts, lst = R.row_lists(tiers)
+    M = np.array([0.05, 0.2, 0.1, 0.15, 0.3, 0.05, 0.15])
+    counts, lst = R.row_lists(tiers, M)
     np.testing.assert_array_equal(counts, [2, 1, 2, 2])
-    np.testing.assert_array_equal(lst, [1, 4, 3, 2, 6, 0, 5])
+    # full: 4 (0.3), 1 (0.2); res: 3; low: 6 (0.15), 2 (0.1); skip: 0, 5 (tie, lower j first)
+    np.testing.assert_array_equal(lst, [4, 1, 3, 6, 2, 0, 5])
 
 
 def test_route_head_scale_and_shapes():
