@@ -108,17 +108,12 @@ Layout layout_of(const ta_params* p) {
       }
     }
   }
-  // bf16 images of the low copies: the FP8 tier and the residual tier read
-  // them; NVFP4 tiles run natively on the packed codes
-  if (p->low == TA_LOW_FP8_E4M3 || p->low == TA_LOW_NVFP4_RES) {
+  // bf16 images of the low copies: the FP8 tier reads them; NVFP4 tiles (and
+  // their residual copies) run natively on the packed codes
+  if (p->low == TA_LOW_FP8_E4M3) {
     L.dq = take(tok * 2);
     L.dk = take(tok * 2);
     L.dv = take(tok * 2);
-  }
-  if (p->low == TA_LOW_NVFP4_RES) {
-    L.drq = take(tok * 2);
-    L.drk = take(tok * 2);
-    L.drv = take(tok * 2);
   }
   L.total = off;
   return L;
@@ -344,10 +339,9 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
       (st = check_tensor(O)))
     return st;
   if ((st = check_ws(p, ws, ws_bytes)) != TA_OK) return st;
-  if (p->low == TA_LOW_NVFP4_RES) return TA_ERR_UNSUPPORTED;
-  // native NVFP4 tiles are built for d = 128 with 128 x 128 tiles
-  if (p->low == TA_LOW_NVFP4 && (p->d != 128 || p->block_q != 128 || p->block_k != 128))
-    return TA_ERR_UNSUPPORTED;
+  // native NVFP4 (and residual) tiles are built for d = 128 with 128 x 128 tiles
+  const bool fp4 = p->low == TA_LOW_NVFP4 || p->low == TA_LOW_NVFP4_RES;
+  if (fp4 && (p->d != 128 || p->block_q != 128 || p->block_k != 128)) return TA_ERR_UNSUPPORTED;
   const Shape s = shape_of(p);
   const Layout L = layout_of(p);
   ta::AttnArgs a;
@@ -374,22 +368,34 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
   a.row_lists = at<int>(ws, L.row_lists);
   a.O = static_cast<__nv_bfloat16*>(O);
   a.Np = (int)s.Np;
-  a.q_sf = p->low == TA_LOW_NVFP4 ? at<uint8_t>(ws, L.q_scales) : nullptr;
-  a.k_sf = p->low == TA_LOW_NVFP4 ? at<uint8_t>(ws, L.k_scales) : nullptr;
-  a.v_sf = p->low == TA_LOW_NVFP4 ? at<uint8_t>(ws, L.v_scales) : nullptr;
+  a.q_sf = fp4 ? at<uint8_t>(ws, L.q_scales) : nullptr;
+  a.k_sf = fp4 ? at<uint8_t>(ws, L.k_scales) : nullptr;
+  a.v_sf = fp4 ? at<uint8_t>(ws, L.v_scales) : nullptr;
+  a.rq_sf = at<uint8_t>(ws, L.rq_scales);
+  a.rk_sf = at<uint8_t>(ws, L.rk_scales);
+  a.rv_sf = at<uint8_t>(ws, L.rv_scales);
 
-  CUtensorMap maps[6];
+  CUtensorMap maps[9];
   const int64_t cb = (int64_t)p->H * p->N * p->d, ch = (int64_t)p->N * p->d, cn = p->d;
   bool ok = make_map(&maps[0], Q, p->B, p->H, p->N, p->d, p->stride_b, p->stride_h, p->stride_n, p->block_q) &&
             make_map(&maps[1], K, p->B, p->H, p->N, p->d, p->stride_b, p->stride_h, p->stride_n, p->block_k) &&
             make_map(&maps[2], V, p->B, p->H, p->N, p->d, p->stride_b, p->stride_h, p->stride_n, p->block_k);
   // the dequantised copies are contiguous [B*H, N, d]; without a low tier they
   // alias the bf16 inputs (never read)
-  if (p->low == TA_LOW_NVFP4) {
+  if (fp4) {
     const int64_t BH = (int64_t)p->B * p->H;
     ok = ok && make_map_fp4(&maps[3], at<void>(ws, L.q_codes), BH, p->N, p->d / 2, p->block_q) &&
          make_map_fp4(&maps[4], at<void>(ws, L.k_codes), BH, p->N, p->d / 2, p->block_k) &&
          make_map_fp4(&maps[5], at<void>(ws, L.v_codes), BH, p->d, s.Np / 2, p->d);
+    if (p->low == TA_LOW_NVFP4_RES) {
+      ok = ok && make_map_fp4(&maps[6], at<void>(ws, L.rq_codes), BH, p->N, p->d / 2, p->block_q) &&
+           make_map_fp4(&maps[7], at<void>(ws, L.rk_codes), BH, p->N, p->d / 2, p->block_k) &&
+           make_map_fp4(&maps[8], at<void>(ws, L.rv_codes), BH, p->d, s.Np / 2, p->d);
+    } else {
+      maps[6] = maps[3];
+      maps[7] = maps[4];
+      maps[8] = maps[5];
+    }
   } else if (L.dq != kAbsent) {
     const void* dq = at<void>(ws, L.dq);
     const void* dk = at<void>(ws, L.dk);
@@ -401,6 +407,11 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
     maps[3] = maps[0];
     maps[4] = maps[1];
     maps[5] = maps[2];
+  }
+  if (!fp4) {
+    maps[6] = maps[3];  // residual copies: only the NVFP4 + residual format has them
+    maps[7] = maps[4];
+    maps[8] = maps[5];
   }
   if (!ok) return TA_ERR_CUDA;
   return ta::launch_attn(a, maps, static_cast<cudaStream_t>(stream)) == cudaSuccess ? TA_OK

@@ -59,7 +59,7 @@ struct Roles {
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
 };
 
-enum TileKind { KIND_FULL = 0, KIND_LOW = 1, KIND_SKIP = 2 };
+enum TileKind { KIND_FULL = 0, KIND_LOW = 1, KIND_SKIP = 2, KIND_RES = 3 };
 
 struct RowPlan {
   int n_full, n_res, n_low, n_skip;
@@ -67,17 +67,18 @@ struct RowPlan {
   const int* list;   // this row's list
 };
 
+// Tile t of a row: its kind and the position of its (first) key block in the
+// row's list.  Kept tiles come in list order (full, residual, low); skipped
+// blocks follow in chunks of BK.
 template <int BK>
 __device__ __forceinline__ void tile_of(const RowPlan& rp, int t, int& kind, int& first) {
-  if (t < rp.n_full) {
-    kind = KIND_FULL;
+  const int kept = rp.n_full + rp.n_res + rp.n_low;
+  if (t < kept) {
+    kind = t < rp.n_full ? KIND_FULL : (t < rp.n_full + rp.n_res ? KIND_RES : KIND_LOW);
     first = t;
-  } else if (t < rp.n_full + rp.n_low) {
-    kind = KIND_LOW;
-    first = rp.n_full + rp.n_res + (t - rp.n_full);
   } else {
     kind = KIND_SKIP;
-    first = rp.n_full + rp.n_res + rp.n_low + (t - rp.n_full - rp.n_low) * BK;
+    first = kept + (t - kept) * BK;
   }
 }
 
@@ -160,15 +161,17 @@ __device__ __forceinline__ __half2 e2m1x2_to_half2(uint32_t codes) {
 }
 
 // Shared-memory layout (offsets from a 1024-aligned base).
-template <int D, int BK, bool FP4>
+template <int D, int BK, bool FP4, bool RES>
 struct Smem {
+  static constexpr int NC = RES ? 2 : 1;      // NVFP4 copies per operand
   static constexpr int kQ = 128 * D * 2;      // one query tile, 128 rows
   static constexpr int kKV = BK * D * 2;      // one K or V tile
-  static constexpr int kPfp4 = 128 * 64 + 1024;  // one NVFP4 P tile: codes + scales
-  static constexpr int kP = FP4 ? 2 * kPfp4 : 0;  // bf16 P lives in TMEM
+  static constexpr int kPfp4 = 128 * 64 + 1024;  // one NVFP4 tile: codes + scales
+  static constexpr int kQlow = FP4 ? NC * kPfp4 : kQ;  // low query copies
+  static constexpr int kP = FP4 ? 2 * NC * kPfp4 : 0;  // bf16 P lives in TMEM
   static constexpr int oQ = 0;
   static constexpr int oDQ = oQ + kQ;
-  static constexpr int oK0 = oDQ + kQ;
+  static constexpr int oK0 = oDQ + kQlow;
   static constexpr int oV0 = oK0 + kKV;
   static constexpr int oK1 = oV0 + kKV;
   static constexpr int oV1 = oK1 + kKV;
@@ -191,12 +194,16 @@ enum {
 
 // TMEM columns of the NVFP4 scale factors (4 columns per 64-element K chunk,
 // 2 chunks per operand), after S0, S1 and O.
-template <int D, int BK>
+template <int D, int BK, bool RES>
 struct TmemSf {
-  static constexpr uint32_t kSfaQ = 2 * BK + D;
-  static constexpr uint32_t kSfbK0 = kSfaQ + 8, kSfbK1 = kSfaQ + 16;
-  static constexpr uint32_t kSfbV0 = kSfaQ + 24, kSfbV1 = kSfaQ + 32;
-  static constexpr uint32_t kSfaP0 = kSfaQ + 40, kSfaP1 = kSfaQ + 48;  // ends at +56 <= 512
+  static constexpr uint32_t NC = RES ? 2 : 1;   // copies (first + residual)
+  static constexpr uint32_t kBase = 2 * BK + D;
+  // query copy c; K copy c of stage s; V copy c of stage s; P copy c of buffer b
+  static constexpr __device__ uint32_t sfaQ(int c) { return kBase + 8 * c; }
+  static constexpr __device__ uint32_t sfbK(int s, int c) { return kBase + 8 * NC + 8 * (s * NC + c); }
+  static constexpr __device__ uint32_t sfbV(int s, int c) { return kBase + 24 * NC + 8 * (s * NC + c); }
+  static constexpr __device__ uint32_t sfaP(int b, int c) { return kBase + 40 * NC + 8 * (b * NC + c); }
+  static constexpr uint32_t kEnd = kBase + 56 * NC;  // <= 512 (496 with residual copies)
 };
 
 // NVFP4 tiles in shared memory: codes [rows][64 B] with 64-byte swizzle, then
@@ -220,20 +227,23 @@ __device__ __forceinline__ void gather_row_sf(unsigned char* dst, const uint8_t*
   }
 }
 
-template <int D, int BK, bool FP4>
+template <int D, int BK, bool FP4, bool RES>
 __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
     attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmQ,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
-                const __grid_constant__ CUtensorMap tmDV) {
-  using L = Smem<D, BK, FP4>;
-  using TS = TmemSf<D, BK>;
+                const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmRQ,
+                const __grid_constant__ CUtensorMap tmRK, const __grid_constant__ CUtensorMap tmRV) {
+  static_assert(!RES || FP4, "residual tiles are NVFP4 tiles");
+  using L = Smem<D, BK, FP4, RES>;
+  using TS = TmemSf<D, BK, RES>;
   using RL = Roles<D, BK>;
   constexpr int kSplit = RL::kSplit, kSoftmaxWarps = RL::kSoftmaxWarps;
   constexpr int kProducerKWarp = RL::kProducerKWarp, kProducerVWarp = RL::kProducerVWarp;
   constexpr int kMmaWarp = RL::kMmaWarp;
   static_assert(!FP4 || (D == 128 && BK == 128), "native NVFP4 tiles need d = 128, 128-key tiles");
   constexpr uint32_t kTmemCols = FP4 ? 512u : L::kTmemCols;
+  static_assert(!FP4 || TS::kEnd <= 512u, "TMEM columns");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw;
   if (smem_u32(sm) & 1023u) {
@@ -257,8 +267,9 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
   rp.n_low = a.row_counts[row_id * 4 + 2];
   rp.n_skip = a.row_counts[row_id * 4 + 3];
   rp.list = a.row_lists + row_id * a.nKb;
-  rp.T = rp.n_full + rp.n_low + (rp.n_skip + BK - 1) / BK;
-  const bool has_low = rp.n_low > 0;
+  rp.T = rp.n_full + rp.n_res + rp.n_low + (rp.n_skip + BK - 1) / BK;
+  const bool has_low = rp.n_low > 0 || rp.n_res > 0;  // tiles reading the first low copy
+  const int nq = rp.n_res > 0 ? 2 : (has_low ? 1 : 0);  // NVFP4 query copies to load
 
   AbortCtx ctx{abort_flag, a.status};
 
@@ -321,10 +332,12 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
     uint64_t* full = &bars[isK ? BAR_K0 : BAR_V0];
     uint64_t* empty = &bars[isK ? BAR_KE0 : BAR_VE0];
     if (isK) {
-      if (FP4 && has_low) {
-        // scales of the NVFP4 query copy, ready for tcgen05.cp
-        gather_row_sf(sm + L::oDQ + kFp4Sf, a.q_sf + ((int64_t)bh * a.N + q0) * 8,
-                      min(128, a.N - q0), lane);
+      if (FP4 && nq > 0) {
+        // scales of the NVFP4 query copies, ready for tcgen05.cp
+        for (int c = 0; c < nq; ++c)
+          gather_row_sf(sm + L::oDQ + c * L::kPfp4 + kFp4Sf,
+                        (c ? a.rq_sf : a.q_sf) + ((int64_t)bh * a.N + q0) * 8, min(128, a.N - q0),
+                        lane);
         fence_proxy_async_smem();
         __syncwarp();
       }
@@ -332,13 +345,14 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         const uint32_t qbytes = (uint32_t)a.bq * D * 2;
-        const uint32_t lbytes = FP4 ? (uint32_t)a.bq * 64 : qbytes;
-        mbar_arrive_expect_tx(&bars[BAR_Q], has_low ? qbytes + lbytes : qbytes);
+        const uint32_t lbytes = FP4 ? (uint32_t)(nq * a.bq * 64) : (has_low ? qbytes : 0u);
+        mbar_arrive_expect_tx(&bars[BAR_Q], qbytes + lbytes);
         for (int x = 0; x < D / 64; ++x)
           tma_load_4d(sm + L::oQ + x * (128 * 128), &tmQ, &bars[BAR_Q], x * 64, q0, h, b);
         if (has_low) {
           if (FP4) {
             tma_load_3d(sm + L::oDQ, &tmDQ, &bars[BAR_Q], 0, q0, bh);
+            if (nq > 1) tma_load_3d(sm + L::oDQ + L::kPfp4, &tmRQ, &bars[BAR_Q], 0, q0, bh);
           } else {
             for (int x = 0; x < D / 64; ++x)
               tma_load_4d(sm + L::oDQ + x * (128 * 128), &tmDQ, &bars[BAR_Q], x * 64, q0, h, b);
@@ -361,27 +375,32 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
       int kind, first;
       tile_of<BK>(rp, t, kind, first);
       unsigned char* st = sm + (isK ? (s ? L::oK1 : L::oK0) : (s ? L::oV1 : L::oV0));
-      if (FP4 && kind == KIND_LOW) {
+      if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
         const int j = rp.list[first];
-        if (isK) {
-          // K scales (rows of the key tile) in the tcgen05.cp block layout
-          gather_row_sf(st + kFp4Sf, a.k_sf + ((int64_t)bh * a.N + j * BK) * 8,
-                        min(BK, a.N - j * BK), lane);
-        } else {
-          // V scales: groups of 16 keys of each d row of V^T
-          const int ng = a.Np / 16;
+        const int ncopy = (RES && kind == KIND_RES) ? 2 : 1;   // first copy [+ residual]
+        for (int c = 0; c < ncopy; ++c) {
+          unsigned char* cst = st + c * L::kPfp4;
+          if (isK) {
+            // K scales (rows of the key tile) in the tcgen05.cp block layout
+            gather_row_sf(cst + kFp4Sf, (c ? a.rk_sf : a.k_sf) + ((int64_t)bh * a.N + j * BK) * 8,
+                          min(BK, a.N - j * BK), lane);
+          } else {
+            // V scales: groups of 16 keys of each d row of V^T
+            const uint8_t* vsf = c ? a.rv_sf : a.v_sf;
+            const int ng = a.Np / 16;
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
+            for (int kc = 0; kc < 2; ++kc) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int g = j * 8 + c * 4 + k;   // group of 16 keys
-              uint32_t w = 0u;
-              if (g < ng)
-                w = *reinterpret_cast<const uint32_t*>(a.v_sf + ((int64_t)bh * ng + g) * D + lane * 4);
+              for (int k = 0; k < 4; ++k) {
+                const int g = j * 8 + kc * 4 + k;   // group of 16 keys
+                uint32_t w = 0u;
+                if (g < ng)
+                  w = *reinterpret_cast<const uint32_t*>(vsf + ((int64_t)bh * ng + g) * D + lane * 4);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int m = lane * 4 + i;        // d row of V^T
-                st[kFp4Sf + c * 512 + (m & 31) * 16 + (m >> 5) * 4 + k] = (unsigned char)(w >> (8 * i));
+                for (int i = 0; i < 4; ++i) {
+                  const int m = lane * 4 + i;        // d row of V^T
+                  cst[kFp4Sf + kc * 512 + (m & 31) * 16 + (m >> 5) * 4 + k] = (unsigned char)(w >> (8 * i));
+                }
               }
             }
           }
@@ -391,11 +410,13 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         if (lane == 0) {
           const bool drop = isK && (t == 0) && (a.debug_flags & TA_DEBUG_DROP_FIRST_K);
           if (!drop) {
-            mbar_arrive_expect_tx(&full[s], (isK ? BK : D) * 64);
-            if (isK)
-              tma_load_3d(st, &tmDK, &full[s], 0, j * BK, bh);
-            else
-              tma_load_3d(st, &tmDV, &full[s], j * 64, 0, bh);
+            mbar_arrive_expect_tx(&full[s], ncopy * (isK ? BK : D) * 64);
+            for (int c = 0; c < ncopy; ++c) {
+              if (isK)
+                tma_load_3d(st + c * L::kPfp4, c ? &tmRK : &tmDK, &full[s], 0, j * BK, bh);
+              else
+                tma_load_3d(st + c * L::kPfp4, c ? &tmRV : &tmDV, &full[s], j * 64, 0, bh);
+            }
             issued[s]++;
           }
         }
@@ -450,17 +471,31 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         tc_fence_after();
         int kind, first;
         tile_of<BK>(rp, t, kind, first);
-        const uint32_t aq = (kind == KIND_LOW) ? sDQ : sQ;
+        const uint32_t aq = (kind == KIND_LOW || kind == KIND_RES) ? sDQ : sQ;
         const uint32_t sk = smem_u32(sm + (s ? L::oK1 : L::oK0));
-        if (FP4 && kind == KIND_LOW) {
-          const uint32_t sfb = tmem + (s ? TS::kSfbK1 : TS::kSfbK0);
-          tc_cp_sf(sfb, smem_desc_rows16(sk + kFp4Sf));
-          tc_cp_sf(sfb + 4, smem_desc_rows16(sk + kFp4Sf + 512));
+        if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
+          // NVFP4: Q1 K1 (+ Q1 K2 + Q2 K1 on residual tiles), block scales in TMEM
+          const int ncopy = (RES && kind == KIND_RES) ? 2 : 1;
+          for (int c = 0; c < ncopy; ++c) {
+            const uint32_t sfb = tmem + TS::sfbK(s, c);
+            tc_cp_sf(sfb, smem_desc_rows16(sk + c * L::kPfp4 + kFp4Sf));
+            tc_cp_sf(sfb + 4, smem_desc_rows16(sk + c * L::kPfp4 + kFp4Sf + 512));
+          }
+          const uint32_t d = s ? tS1 : tS0;
 #pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            mma_nvfp4_ss(s ? tS1 : tS0, smem_desc_sw64(aq + kk * 32), smem_desc_sw64(sk + kk * 32),
-                         idesc_nvfp4(128, BK), tmem + TS::kSfaQ + kk * 4, sfb + kk * 4,
-                         kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 2; ++kk) {
+            mma_nvfp4_ss(d, smem_desc_sw64(aq + kk * 32), smem_desc_sw64(sk + kk * 32),
+                         idesc_nvfp4(128, BK), tmem + TS::sfaQ(0) + kk * 4,
+                         tmem + TS::sfbK(s, 0) + kk * 4, kk > 0 ? 1u : 0u);
+            if (RES && kind == KIND_RES) {
+              mma_nvfp4_ss(d, smem_desc_sw64(aq + kk * 32), smem_desc_sw64(sk + L::kPfp4 + kk * 32),
+                           idesc_nvfp4(128, BK), tmem + TS::sfaQ(0) + kk * 4,
+                           tmem + TS::sfbK(s, 1) + kk * 4, 1u);
+              mma_nvfp4_ss(d, smem_desc_sw64(aq + L::kPfp4 + kk * 32), smem_desc_sw64(sk + kk * 32),
+                           idesc_nvfp4(128, BK), tmem + TS::sfaQ(1) + kk * 4,
+                           tmem + TS::sfbK(s, 0) + kk * 4, 1u);
+            }
+          }
         } else {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -476,9 +511,11 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
       bool ok = mbar_wait(&bars[BAR_Q], 0, ctx, 3);
       if (ok) {
         tc_fence_after();
-        if (FP4 && has_low) {
-          tc_cp_sf(tmem + TS::kSfaQ, smem_desc_rows16(sDQ + kFp4Sf));
-          tc_cp_sf(tmem + TS::kSfaQ + 4, smem_desc_rows16(sDQ + kFp4Sf + 512));
+        if (FP4) {
+          for (int c = 0; c < nq; ++c) {
+            tc_cp_sf(tmem + TS::sfaQ(c), smem_desc_rows16(sDQ + c * L::kPfp4 + kFp4Sf));
+            tc_cp_sf(tmem + TS::sfaQ(c) + 4, smem_desc_rows16(sDQ + c * L::kPfp4 + kFp4Sf + 512));
+          }
         }
         ok = issue_s(0);
       }
@@ -491,19 +528,31 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         const uint32_t sv = smem_u32(sm + (s ? L::oV1 : L::oV0));
         int kind_t, first_t;
         tile_of<BK>(rp, t, kind_t, first_t);
-        if (FP4 && kind_t == KIND_LOW) {
-          const uint32_t sfb = tmem + (s ? TS::kSfbV1 : TS::kSfbV0);
-          const uint32_t sfa = tmem + (s ? TS::kSfaP1 : TS::kSfaP0);
-          const uint32_t pb = sP + s * L::kPfp4;
-          tc_cp_sf(sfa, smem_desc_rows16(pb + kFp4Sf));
-          tc_cp_sf(sfa + 4, smem_desc_rows16(pb + kFp4Sf + 512));
-          tc_cp_sf(sfb, smem_desc_rows16(sv + kFp4Sf));
-          tc_cp_sf(sfb + 4, smem_desc_rows16(sv + kFp4Sf + 512));
+        if (FP4 && (kind_t == KIND_LOW || kind_t == KIND_RES)) {
+          // NVFP4: P1 V1 (+ P1 V2 + P2 V1 on residual tiles)
+          const int ncopy = (RES && kind_t == KIND_RES) ? 2 : 1;
+          const uint32_t pb = sP + s * L::NC * L::kPfp4;
+          for (int c = 0; c < ncopy; ++c) {
+            const uint32_t sfa = tmem + TS::sfaP(s, c), sfb = tmem + TS::sfbV(s, c);
+            tc_cp_sf(sfa, smem_desc_rows16(pb + c * L::kPfp4 + kFp4Sf));
+            tc_cp_sf(sfa + 4, smem_desc_rows16(pb + c * L::kPfp4 + kFp4Sf + 512));
+            tc_cp_sf(sfb, smem_desc_rows16(sv + c * L::kPfp4 + kFp4Sf));
+            tc_cp_sf(sfb + 4, smem_desc_rows16(sv + c * L::kPfp4 + kFp4Sf + 512));
+          }
 #pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
+          for (int kk = 0; kk < 2; ++kk) {
             mma_nvfp4_ss(tO, smem_desc_sw64(pb + kk * 32), smem_desc_sw64(sv + kk * 32),
-                         idesc_nvfp4(128, D), sfa + kk * 4, sfb + kk * 4,
-                         (t > 0 || kk > 0) ? 1u : 0u);
+                         idesc_nvfp4(128, D), tmem + TS::sfaP(s, 0) + kk * 4,
+                         tmem + TS::sfbV(s, 0) + kk * 4, (t > 0 || kk > 0) ? 1u : 0u);
+            if (RES && kind_t == KIND_RES) {
+              mma_nvfp4_ss(tO, smem_desc_sw64(pb + kk * 32), smem_desc_sw64(sv + L::kPfp4 + kk * 32),
+                           idesc_nvfp4(128, D), tmem + TS::sfaP(s, 0) + kk * 4,
+                           tmem + TS::sfbV(s, 1) + kk * 4, 1u);
+              mma_nvfp4_ss(tO, smem_desc_sw64(pb + L::kPfp4 + kk * 32), smem_desc_sw64(sv + kk * 32),
+                           idesc_nvfp4(128, D), tmem + TS::sfaP(s, 1) + kk * 4,
+                           tmem + TS::sfbV(s, 0) + kk * 4, 1u);
+            }
+          }
         } else {
           // A = bf16 P' in the TMEM columns of this tile's S buffer
           const uint32_t pa = s ? tS1 : tS0;
@@ -606,7 +655,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
 
       // round P' as the tier demands, into bf16 pairs (or NVFP4 codes)
       uint32_t p[HB / 2];
-      if (FP4 && kind == KIND_LOW) {
+      if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
         // codes of this part (HB = 32 keys, half an MMA K chunk) in p[0..3],
         // ue4m3 scales of its 2 groups in p[4]
         uint32_t scw = 0u;
@@ -628,6 +677,39 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           }
         }
         p[HB / 8] = scw;
+        if (RES && kind == KIND_RES) {
+          // second copy: NVFP4 of the residual fp32(P' - deq(P1)), in p[8..12]
+          uint32_t scw2 = 0u;
+#pragma unroll
+          for (int g = 0; g < HB / 16; ++g) {
+            const float sc1 = sc_tab[(scw >> (8 * g)) & 0xFFu].x;
+            float rr[16];
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+#pragma unroll
+              for (int bb = 0; bb < 4; ++bb) {
+                const float2 f = __half22float2(e2m1x2_to_half2(p[g * 2 + w] >> (8 * bb)));
+                const int c = w * 8 + 2 * bb;
+                rr[c] = __fsub_rn(x[g * 16 + c], __fmul_rn(f.x, sc1));
+                rr[c + 1] = __fsub_rn(x[g * 16 + c + 1], __fmul_rn(f.y, sc1));
+              }
+            }
+            float am = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(rr[i]));
+            const uint32_t scc2 = cvt_e4m3x2(__fdiv_rn(am, 6.0f), 0.0f) & 0xFFu;
+            const float inv2 = sc_tab[scc2].y;
+            scw2 |= scc2 << (8 * g);
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+              float y[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(rr[w * 8 + i], inv2);
+              p[8 + g * 2 + w] = cvt_e2m1x8(y);
+            }
+          }
+          p[8 + HB / 8] = scw2;
+        }
       } else if (kind == KIND_LOW && a.low == TA_LOW_FP8_E4M3) {
 #pragma unroll
         for (int c = 0; c < HB; c += 2) {
@@ -663,7 +745,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
       // The warps sharing these rows see the same maxima, so they agree on
       // `rescale` and on `reuse` and wait (and leave on abort) together.
       const bool rescale = (t > 0) && __any_sync(0xffffffffu, alpha != 1.0f);
-      const bool reuse = FP4 && kind == KIND_LOW && t >= 2;
+      const bool reuse = FP4 && (kind == KIND_LOW || kind == KIND_RES) && t >= 2;
       if (rescale || reuse) {
         bool ok2 = true;
         if (reuse) ok2 = mbar_wait(&bars[BAR_PD0 + s], ((t >> 1) - 1) & 1, ctx, 7);
@@ -684,17 +766,19 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           tmem_st32(tO + lane_off + part * HD + c0, raw);
         }
       }
-      if (FP4 && kind == KIND_LOW) {
+      if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
         // NVFP4 P part: 16 bytes of codes into the 64-byte-swizzled tile, 2
-        // scale bytes into the scale-factor block of K chunk part/2
-        unsigned char* pbuf = sm + L::oP + s * L::kPfp4;
-        {
-          const int ch = part;
-          const uint32_t off = r * 64 + ((ch ^ ((r >> 1) & 3)) * 16);
-          *reinterpret_cast<uint4*>(pbuf + off) = make_uint4(p[0], p[1], p[2], p[3]);
+        // scale bytes into the scale-factor block of K chunk part/2 (and the
+        // same for the residual copy on residual tiles)
+        unsigned char* pbuf = sm + L::oP + s * L::NC * L::kPfp4;
+        const uint32_t off = r * 64 + ((part ^ ((r >> 1) & 3)) * 16);
+        const uint32_t soff = kFp4Sf + (part >> 1) * 512 + lane * 16 + quarter * 4 + (part & 1) * 2;
+        *reinterpret_cast<uint4*>(pbuf + off) = make_uint4(p[0], p[1], p[2], p[3]);
+        *reinterpret_cast<uint16_t*>(pbuf + soff) = (uint16_t)p[HB / 8];
+        if (RES && kind == KIND_RES) {
+          *reinterpret_cast<uint4*>(pbuf + L::kPfp4 + off) = make_uint4(p[8], p[9], p[10], p[11]);
+          *reinterpret_cast<uint16_t*>(pbuf + L::kPfp4 + soff) = (uint16_t)p[8 + HB / 8];
         }
-        *reinterpret_cast<uint16_t*>(pbuf + kFp4Sf + (part >> 1) * 512 + lane * 16 + quarter * 4 +
-                                     (part & 1) * 2) = (uint16_t)p[HB / 8];
       } else {
         // bf16 P' of this part into the S buffer's first BK/2 columns (every
         // part has loaded its S columns before the row barrier above)
@@ -703,7 +787,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           tmem_st16((s ? tS1 : tS0) + lane_off + part * (HB / 2) + q, p + q);
       }
       tmem_wait_st();
-      if (FP4 && kind == KIND_LOW) fence_proxy_async_smem();
+      if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[BAR_P]);
     }
@@ -752,26 +836,27 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int D, int BK, bool FP4>
+template <int D, int BK, bool FP4, bool RES>
 cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
-  using L = Smem<D, BK, FP4>;
-  auto k = attn_kernel<D, BK, FP4>;
+  using L = Smem<D, BK, FP4, RES>;
+  auto k = attn_kernel<D, BK, FP4, RES>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nQb, a.B * a.H);
   k<<<grid, Roles<D, BK>::kThreads, L::kAlloc, s>>>(a, maps[0], maps[1], maps[2], maps[3], maps[4],
-                                                   maps[5]);
+                                                   maps[5], maps[6], maps[7], maps[8]);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attn(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
-  if (a.d == 64 && a.bk == 64) return launch_d<64, 64, false>(a, maps, s);
-  if (a.d == 64 && a.bk == 128) return launch_d<64, 128, false>(a, maps, s);
-  if (a.d == 128 && a.bk == 64) return launch_d<128, 64, false>(a, maps, s);
-  if (a.low == TA_LOW_NVFP4) return launch_d<128, 128, true>(a, maps, s);
-  return launch_d<128, 128, false>(a, maps, s);
+  if (a.d == 64 && a.bk == 64) return launch_d<64, 64, false, false>(a, maps, s);
+  if (a.d == 64 && a.bk == 128) return launch_d<64, 128, false, false>(a, maps, s);
+  if (a.d == 128 && a.bk == 64) return launch_d<128, 64, false, false>(a, maps, s);
+  if (a.low == TA_LOW_NVFP4) return launch_d<128, 128, true, false>(a, maps, s);
+  if (a.low == TA_LOW_NVFP4_RES) return launch_d<128, 128, true, true>(a, maps, s);
+  return launch_d<128, 128, false, false>(a, maps, s);
 }
 
 }  // namespace ta

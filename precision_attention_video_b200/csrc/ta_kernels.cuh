@@ -62,6 +62,10 @@ struct AttnArgs {
   const uint8_t* q_sf;
   const uint8_t* k_sf;
   const uint8_t* v_sf;
+  // scales of the residual NVFP4 copies (TA_LOW_NVFP4_RES), same layouts
+  const uint8_t* rq_sf;
+  const uint8_t* rk_sf;
+  const uint8_t* rv_sf;
   int Np;
 };
 

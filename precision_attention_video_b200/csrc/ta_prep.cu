@@ -239,8 +239,8 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const PlanArgs a) {
         }
       }
       __syncthreads();
-      if (res) {
-        __nv_bfloat16* rdeq_out = which == 0 ? a.drq : which == 1 ? a.drk : a.drv;
+      __nv_bfloat16* rdeq_out = which == 0 ? a.drq : which == 1 ? a.drk : a.drv;
+      if (res && rdeq_out != nullptr) {
         for (int idx = tid; idx < R * (D / 8); idx += kThreads) {
           const int r = idx / (D / 8), c8 = idx % (D / 8);
           if (r < nrows)
