@@ -150,11 +150,59 @@ def algorithmic_attn_flops(cfg, counts: np.ndarray, lists: np.ndarray):
     return full, low, skip
 
 
-def workload(args):
-    cfg = get_config(WORKLOAD)
+def workload(args, name=None):
+    cfg = get_config(name or args.workload)
     if args.heads:
         cfg = cfg.with_(H=args.heads)
     return cfg
+
+
+def sweep(args):
+    """Forward time of the 480p-shaped layer at every sparsity-sweep point
+    (FP8 low tier = 20 % of kept tiles) and its speedup over the all-full
+    point, one JSON line per point (not the benchmark contract line)."""
+    import precision_attention_video_b200 as pav
+
+    dev = torch.device("cuda", 0)
+    base = workload(args, "sweep0")
+    Q, K, V = make_qkv(base)
+    Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+    O = torch.empty_like(Qd)
+    dense = 4.0 * base.B * base.H * float(base.N) ** 2 * base.d
+    ref_ms = None
+    for pct in (0, 30, 50, 70, 90):
+        cfg = workload(args, f"sweep{pct}")
+        p = pav.params_for(cfg)
+        ws = pav.alloc_workspace(p, dev)
+        for _ in range(args.warmup):
+            pav.plan(p, Qd, Kd, Vd, ws)
+            pav.forward(p, Qd, Kd, Vd, ws, O)
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        fwd, pln = [], []
+        for _ in range(args.steps):
+            ev[0].record()
+            pav.plan(p, Qd, Kd, Vd, ws)
+            ev[1].record()
+            pav.forward(p, Qd, Kd, Vd, ws, O)
+            ev[2].record()
+            torch.cuda.synchronize()
+            pln.append(ev[0].elapsed_time(ev[1]))
+            fwd.append(ev[1].elapsed_time(ev[2]))
+        st = pav.get_status(ws)
+        t = pav.plan_views(p, ws)["tier_map"].cpu().numpy()
+        f = statistics.median(fwd)
+        if pct == 0:
+            ref_ms = f
+        print(json.dumps({
+            "sweep_point": pct, "tau": list(cfg.tau), "status": st,
+            "tier_frac": {"full": float((t == 3).mean()), "low": float((t == 1).mean()),
+                          "skip": float((t == 0).mean())},
+            "ms_forward": f, "ms_plan": statistics.median(pln),
+            "dense_equiv_tflops_forward": dense / (f * 1e-3) / 1e12,
+            "dense_equiv_tflops_layer": dense / ((f + statistics.median(pln)) * 1e-3) / 1e12,
+            "forward_speedup_vs_all_full": ref_ms / f}), flush=True)
+        del ws
 
 
 def run_gpu_arm(args, rank, world, local_rank):
@@ -288,17 +336,29 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (smaller profiling cases)")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="workload name (latent_gen.configs); the contract line uses 480p")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the sparsity sweep instead (one JSON line per point)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
+    if args.sweep:
+        sweep(args)
+        return
     world = _env_int("WORLD_SIZE", 1)
     rank = _env_int("RANK", 0)
     local_rank = _env_int("LOCAL_RANK", 0)
     cfg = workload(args)
-    config = {"workload": "480p-video-like tiered attention layer", "B": cfg.B, "H": cfg.H,
+    from latent_gen.configs import LOW_NAMES
+    title = {"480p": "480p-video-like tiered attention layer",
+             "720p": "720p-long-video-like tiered attention layer"}.get(
+                 cfg.name, f"{cfg.name} tiered attention layer")
+    config = {"workload": title, "B": cfg.B, "H": cfg.H,
               "N": cfg.N, "d": cfg.d, "grid_txyx": list(cfg.grid),
-              "tile": [cfg.block_q, cfg.block_k], "low_tier": "nvfp4", "tau": list(cfg.tau),
-              "logit_std": cfg.logit_std, "l2": "inputs larger than L2 (Q+K+V 1.0 GB per GPU)",
+              "tile": [cfg.block_q, cfg.block_k], "low_tier": LOW_NAMES[cfg.low], "tau": list(cfg.tau),
+              "logit_std": cfg.logit_std,
+              "l2": f"inputs larger than L2 (Q+K+V {3 * cfg.B * cfg.H * cfg.N * cfg.d * 2 / 1e9:.2f} GB per GPU)",
               "parallelism": f"replicas x{args.gpus}"}
 
     if args.impl == "reference":

@@ -56,6 +56,11 @@ ta_status validate(const ta_params* p) {
   return TA_OK;
 }
 
+// FP8 low tiles run on the FP8 tensor pipe for d = 128 with 128 x 128 tiles.
+bool native_fp8(const ta_params* p) {
+  return p->low == TA_LOW_FP8_E4M3 && p->d == 128 && p->block_q == 128 && p->block_k == 128;
+}
+
 // Workspace layout: byte offsets of every array (kAbsent when not produced).
 struct Layout {
   size_t status, n_k, qbar, kbar, kbar_b, vbar_b, logits, mass, tier_map, row_counts, row_lists;
@@ -108,9 +113,9 @@ Layout layout_of(const ta_params* p) {
       }
     }
   }
-  // bf16 images of the low copies: the FP8 tier reads them; NVFP4 tiles (and
-  // their residual copies) run natively on the packed codes
-  if (p->low == TA_LOW_FP8_E4M3) {
+  // bf16 images of the low copies: only FP8 tiles of d = 64 or 64-row tiles
+  // read them; NVFP4 (+ residual) and 128 x 128 FP8 tiles run natively on the codes
+  if (p->low == TA_LOW_FP8_E4M3 && !native_fp8(p)) {
     L.dq = take(tok * 2);
     L.dk = take(tok * 2);
     L.dv = take(tok * 2);
@@ -212,19 +217,25 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Byte tensor [BH, rows, inner] (contiguous), box = 64 bytes x box_rows,
-// 64-byte swizzle: the packed NVFP4 copies.
-bool make_map_fp4(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int64_t inner,
-                  int box_rows) {
+// Byte tensor [BH, rows, inner] (contiguous), box = box_inner bytes x
+// box_rows: the packed NVFP4 copies (64-byte boxes, 64-byte swizzle) and the
+// FP8 copies (128-byte boxes, 128-byte swizzle).
+bool make_map_u8(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int64_t inner,
+                 int box_rows, int box_inner) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)inner, (cuuint64_t)(inner * rows)};
-  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE,
+            box_inner == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool make_map_fp4(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int64_t inner,
+                  int box_rows) {
+  return make_map_u8(m, base, BH, rows, inner, box_rows, 64);
 }
 
 // bf16 tensor [B, H, N, d] (element strides sb, sh, sn), box = 64 x rows, 128B swizzle.
@@ -371,6 +382,9 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
   a.q_sf = fp4 ? at<uint8_t>(ws, L.q_scales) : nullptr;
   a.k_sf = fp4 ? at<uint8_t>(ws, L.k_scales) : nullptr;
   a.v_sf = fp4 ? at<uint8_t>(ws, L.v_scales) : nullptr;
+  a.q_s8 = p->low == TA_LOW_FP8_E4M3 ? at<float>(ws, L.q_scales) : nullptr;
+  a.k_s8 = p->low == TA_LOW_FP8_E4M3 ? at<float>(ws, L.k_scales) : nullptr;
+  a.v_s8 = p->low == TA_LOW_FP8_E4M3 ? at<float>(ws, L.v_scales) : nullptr;
   a.rq_sf = at<uint8_t>(ws, L.rq_scales);
   a.rk_sf = at<uint8_t>(ws, L.rk_scales);
   a.rv_sf = at<uint8_t>(ws, L.rv_scales);
@@ -396,6 +410,11 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
       maps[7] = maps[4];
       maps[8] = maps[5];
     }
+  } else if (native_fp8(p)) {
+    const int64_t BH = (int64_t)p->B * p->H;
+    ok = ok && make_map_u8(&maps[3], at<void>(ws, L.q_codes), BH, p->N, p->d, p->block_q, 128) &&
+         make_map_u8(&maps[4], at<void>(ws, L.k_codes), BH, p->N, p->d, p->block_k, 128) &&
+         make_map_u8(&maps[5], at<void>(ws, L.v_codes), BH, p->N, p->d, p->block_k, 128);
   } else if (L.dq != kAbsent) {
     const void* dq = at<void>(ws, L.dq);
     const void* dk = at<void>(ws, L.dk);

@@ -161,14 +161,22 @@ __device__ __forceinline__ __half2 e2m1x2_to_half2(uint32_t codes) {
 }
 
 // Shared-memory layout (offsets from a 1024-aligned base).
-template <int D, int BK, bool FP4, bool RES>
+// Low-tier execution mode of a kernel instance.
+enum LowMode { LM_IMAGE = 0, LM_NVFP4 = 1, LM_NVFP4_RES = 2, LM_FP8 = 3 };
+
+template <int D, int BK, int LM>
 struct Smem {
+  static constexpr bool FP4 = (LM == LM_NVFP4 || LM == LM_NVFP4_RES);
+  static constexpr bool RES = (LM == LM_NVFP4_RES);
+  static constexpr bool F8 = (LM == LM_FP8);
   static constexpr int NC = RES ? 2 : 1;      // NVFP4 copies per operand
   static constexpr int kQ = 128 * D * 2;      // one query tile, 128 rows
   static constexpr int kKV = BK * D * 2;      // one K or V tile
   static constexpr int kPfp4 = 128 * 64 + 1024;  // one NVFP4 tile: codes + scales
-  static constexpr int kQlow = FP4 ? NC * kPfp4 : kQ;  // low query copies
-  static constexpr int kP = FP4 ? 2 * NC * kPfp4 : 0;  // bf16 P lives in TMEM
+  static constexpr int kF8 = 128 * 128;                // one FP8 tile (128 rows x 128 B)
+  static constexpr int kQlow = FP4 ? NC * kPfp4 : (F8 ? kF8 : kQ);  // low query copies
+  // P: bf16 P lives in TMEM; NVFP4 / FP8 P in two shared-memory buffers
+  static constexpr int kP = FP4 ? 2 * NC * kPfp4 : (F8 ? 2 * kF8 + 1024 : 0);
   static constexpr int oQ = 0;
   static constexpr int oDQ = oQ + kQ;
   static constexpr int oK0 = oDQ + kQlow;
@@ -196,6 +204,9 @@ enum {
 // 2 chunks per operand), after S0, S1 and O.
 template <int D, int BK, bool RES>
 struct TmemSf {
+  // FP8 tiles: UE8M0 scale factors of P (constant 2^0) and of V (per stage)
+  static constexpr __device__ uint32_t sfaP8() { return 2 * BK + D; }
+  static constexpr __device__ uint32_t sfbV8(int s) { return 2 * BK + D + 4 + 4 * s; }
   static constexpr uint32_t NC = RES ? 2 : 1;   // copies (first + residual)
   static constexpr uint32_t kBase = 2 * BK + D;
   // query copy c; K copy c of stage s; V copy c of stage s; P copy c of buffer b
@@ -227,22 +238,23 @@ __device__ __forceinline__ void gather_row_sf(unsigned char* dst, const uint8_t*
   }
 }
 
-template <int D, int BK, bool FP4, bool RES>
+template <int D, int BK, int LM>
 __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
     attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmQ,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
                 const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmRQ,
                 const __grid_constant__ CUtensorMap tmRK, const __grid_constant__ CUtensorMap tmRV) {
-  static_assert(!RES || FP4, "residual tiles are NVFP4 tiles");
-  using L = Smem<D, BK, FP4, RES>;
+  using L = Smem<D, BK, LM>;
+  constexpr bool FP4 = L::FP4, RES = L::RES, F8 = L::F8;
   using TS = TmemSf<D, BK, RES>;
   using RL = Roles<D, BK>;
   constexpr int kSplit = RL::kSplit, kSoftmaxWarps = RL::kSoftmaxWarps;
   constexpr int kProducerKWarp = RL::kProducerKWarp, kProducerVWarp = RL::kProducerVWarp;
   constexpr int kMmaWarp = RL::kMmaWarp;
-  static_assert(!FP4 || (D == 128 && BK == 128), "native NVFP4 tiles need d = 128, 128-key tiles");
-  constexpr uint32_t kTmemCols = FP4 ? 512u : L::kTmemCols;
+  static_assert(!(FP4 || F8) || (D == 128 && BK == 128),
+                "native NVFP4 / FP8 tiles need d = 128, 128-key tiles");
+  constexpr uint32_t kTmemCols = (FP4 || F8) ? 512u : L::kTmemCols;
   static_assert(!FP4 || TS::kEnd <= 512u, "TMEM columns");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw;
@@ -292,6 +304,11 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
     mbar_init(&bars[BAR_PD1], 1);
     mbar_init(&bars[BAR_DRAIN], 1);
     fence_mbar_init();
+  }
+  if (F8 && threadIdx.x < 128) {
+    // UE8M0 scale factors of the FP8 P operand: all 2^0
+    *reinterpret_cast<uint32_t*>(sm + L::oP + 2 * L::kF8 + threadIdx.x * 4) = 0x7F7F7F7Fu;
+    fence_proxy_async_smem();
   }
   if (FP4 && threadIdx.x < 128) {
     // ue4m3 code -> (value, correctly rounded reciprocal) for P' quantisation
@@ -345,7 +362,8 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         const uint32_t qbytes = (uint32_t)a.bq * D * 2;
-        const uint32_t lbytes = FP4 ? (uint32_t)(nq * a.bq * 64) : (has_low ? qbytes : 0u);
+        const uint32_t lbytes = FP4 ? (uint32_t)(nq * a.bq * 64)
+                                : (has_low ? (F8 ? (uint32_t)a.bq * 128 : qbytes) : 0u);
         mbar_arrive_expect_tx(&bars[BAR_Q], qbytes + lbytes);
         for (int x = 0; x < D / 64; ++x)
           tma_load_4d(sm + L::oQ + x * (128 * 128), &tmQ, &bars[BAR_Q], x * 64, q0, h, b);
@@ -353,6 +371,8 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           if (FP4) {
             tma_load_3d(sm + L::oDQ, &tmDQ, &bars[BAR_Q], 0, q0, bh);
             if (nq > 1) tma_load_3d(sm + L::oDQ + L::kPfp4, &tmRQ, &bars[BAR_Q], 0, q0, bh);
+          } else if (F8) {
+            tma_load_3d(sm + L::oDQ, &tmDQ, &bars[BAR_Q], 0, q0, bh);
           } else {
             for (int x = 0; x < D / 64; ++x)
               tma_load_4d(sm + L::oDQ + x * (128 * 128), &tmDQ, &bars[BAR_Q], x * 64, q0, h, b);
@@ -417,6 +437,26 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
               else
                 tma_load_3d(st + c * L::kPfp4, c ? &tmRV : &tmDV, &full[s], j * 64, 0, bh);
             }
+            issued[s]++;
+          }
+        }
+      } else if (F8 && kind == KIND_LOW) {
+        const int j = rp.list[first];
+        if (!isK) {
+          // UE8M0 scale factor of this V tile: the exponent of its power-of-two scale
+          const uint32_t e = (__float_as_uint(a.v_s8[(int64_t)bh * a.nKb + j]) >> 23) & 0xFFu;
+          reinterpret_cast<uint32_t*>(st + L::kF8)[lane * 4 + 0] = e * 0x01010101u;
+          reinterpret_cast<uint32_t*>(st + L::kF8)[lane * 4 + 1] = e * 0x01010101u;
+          reinterpret_cast<uint32_t*>(st + L::kF8)[lane * 4 + 2] = e * 0x01010101u;
+          reinterpret_cast<uint32_t*>(st + L::kF8)[lane * 4 + 3] = e * 0x01010101u;
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          const bool drop = isK && (t == 0) && (a.debug_flags & TA_DEBUG_DROP_FIRST_K);
+          if (!drop) {
+            mbar_arrive_expect_tx(&full[s], BK * 128);
+            tma_load_3d(st, isK ? &tmDK : &tmDV, &full[s], 0, j * BK, bh);
             issued[s]++;
           }
         }
@@ -496,6 +536,12 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
                            tmem + TS::sfbK(s, 0) + kk * 4, 1u);
             }
           }
+        } else if (F8 && kind == KIND_LOW) {
+          // FP8 codes: 4 MMAs of K = 32 over the 128-byte rows (scales applied in softmax)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f8_ss(s ? tS1 : tS0, smem_desc_sw128(aq + kk * 32, 16, 1024),
+                      smem_desc_sw128(sk + kk * 32, 16, 1024), idesc_f8(128, BK), kk > 0 ? 1u : 0u);
         } else {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -511,6 +557,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
       bool ok = mbar_wait(&bars[BAR_Q], 0, ctx, 3);
       if (ok) {
         tc_fence_after();
+        if (F8) tc_cp_sf(tmem + TS::sfaP8(), smem_desc_rows16(sP + 2 * L::kF8));
         if (FP4) {
           for (int c = 0; c < nq; ++c) {
             tc_cp_sf(tmem + TS::sfaQ(c), smem_desc_rows16(sDQ + c * L::kPfp4 + kFp4Sf));
@@ -553,6 +600,16 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
                            tmem + TS::sfbV(s, 0) + kk * 4, 1u);
             }
           }
+        } else if (F8 && kind_t == KIND_LOW) {
+          // FP8 P codes (scale 2^0) x FP8 V codes (MN-major) with V's power-of-two
+          // tile scale as the UE8M0 block scale
+          const uint32_t pb = sP + s * L::kF8;
+          tc_cp_sf(tmem + TS::sfbV8(s), smem_desc_rows16(sv + L::kF8));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_mxf8_ss(tO, smem_desc_sw128(pb + kk * 32, 16, 1024),
+                        smem_desc_sw128(sv + kk * 32 * 128, 16, 1024), idesc_mxf8_bmn(128, D),
+                        tmem + TS::sfaP8(), tmem + TS::sfbV8(s), (t > 0 || kk > 0) ? 1u : 0u);
         } else {
           // A = bf16 P' in the TMEM columns of this tile's S buffer
           const uint32_t pa = s ? tS1 : tS0;
@@ -584,7 +641,9 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
     const float2* sc_tab = reinterpret_cast<const float2*>(sm + L::oScTab);
     const float c2 = a.scale_log2;           // S -> log2 units
     const float o_off = (float)a.p_offset;
-    float m = -INFINITY, l = 0.0f;           // running max (raw S units), part row sum
+    // FP8 tiles hold the dot products of the codes: their true S is S * s_q * s_k
+    const float s_q8 = F8 ? a.q_s8[(int64_t)bh * a.nQb + qb] : 1.0f;
+    float m = -INFINITY, l = 0.0f;           // running max (S units), part row sum
     for (int t = 0; t < rp.T; ++t) {
       const int s = t & 1;
       bool ok = mbar_wait(&bars[BAR_S0 + s], (t >> 1) & 1, ctx, 6);
@@ -598,6 +657,8 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         nvalid = min(BK, a.N - rp.list[first] * BK);
       }
       const int nv = min(max(nvalid - part * HB, 0), HB);  // valid columns of this part
+      const float sqk = (F8 && kind == KIND_LOW) ? s_q8 * a.k_s8[(int64_t)bh * a.nKb + rp.list[first]]
+                                                 : 1.0f;   // exact: powers of two
       float x[HB];
       float tmax = -INFINITY;
       if (ok) {
@@ -617,7 +678,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < HB; ++c) pm[c & 3] = fmaxf(pm[c & 3], x[c]);
-        tmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+        tmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) * sqk;
         xchg[(s * 4 + part) * 128 + r] = tmax;
       }
       // swap part maxima with the warps sharing these rows; leave together on abort
@@ -628,15 +689,16 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
       for (int q = 0; q < kSplit; ++q) m_new = fmaxf(m_new, xchg[(s * 4 + q) * 128 + r]);
       const float alpha = fast_exp2((m - m_new) * c2);  // 0 on the first tile
       const float mc = m_new * c2 - o_off;              // P' = 2^(s*c2 - mc)
+      const float c2t = c2 * sqk;                       // this tile's S -> log2 units
       if constexpr (kPolyEvery > 0) {
 #pragma unroll
         for (int c = 0; c < HB; ++c) {
-          const float e = fmaf(x[c], c2, -mc);
+          const float e = fmaf(x[c], c2t, -mc);
           x[c] = (c % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) ? exp2_poly(e) : fast_exp2(e);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < HB; ++c) x[c] = fast_exp2(fmaf(x[c], c2, -mc));
+        for (int c = 0; c < HB; ++c) x[c] = fast_exp2(fmaf(x[c], c2t, -mc));
       }
       if (kind == KIND_SKIP) {
 #pragma unroll
@@ -710,6 +772,11 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           }
           p[8 + HB / 8] = scw2;
         }
+      } else if (F8 && kind == KIND_LOW) {
+        // e4m3 codes of P' (scale 1), four per word
+#pragma unroll
+        for (int c = 0; c < HB; c += 4)
+          p[c / 4] = cvt_e4m3x2(x[c], x[c + 1]) | (cvt_e4m3x2(x[c + 2], x[c + 3]) << 16);
       } else if (kind == KIND_LOW && a.low == TA_LOW_FP8_E4M3) {
 #pragma unroll
         for (int c = 0; c < HB; c += 2) {
@@ -745,7 +812,8 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
       // The warps sharing these rows see the same maxima, so they agree on
       // `rescale` and on `reuse` and wait (and leave on abort) together.
       const bool rescale = (t > 0) && __any_sync(0xffffffffu, alpha != 1.0f);
-      const bool reuse = FP4 && (kind == KIND_LOW || kind == KIND_RES) && t >= 2;
+      const bool smem_p = (FP4 && (kind == KIND_LOW || kind == KIND_RES)) || (F8 && kind == KIND_LOW);
+      const bool reuse = smem_p && t >= 2;
       if (rescale || reuse) {
         bool ok2 = true;
         if (reuse) ok2 = mbar_wait(&bars[BAR_PD0 + s], ((t >> 1) - 1) & 1, ctx, 7);
@@ -779,6 +847,15 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           *reinterpret_cast<uint4*>(pbuf + L::kPfp4 + off) = make_uint4(p[8], p[9], p[10], p[11]);
           *reinterpret_cast<uint16_t*>(pbuf + L::kPfp4 + soff) = (uint16_t)p[8 + HB / 8];
         }
+      } else if (F8 && kind == KIND_LOW) {
+        // FP8 P part: 32 codes into the 128-byte-swizzled tile of buffer s
+        unsigned char* pbuf = sm + L::oP + s * L::kF8;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int ch = part * 2 + q;
+          *reinterpret_cast<uint4*>(pbuf + r * 128 + ((ch ^ (r & 7)) * 16)) =
+              make_uint4(p[q * 4 + 0], p[q * 4 + 1], p[q * 4 + 2], p[q * 4 + 3]);
+        }
       } else {
         // bf16 P' of this part into the S buffer's first BK/2 columns (every
         // part has loaded its S columns before the row barrier above)
@@ -787,7 +864,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           tmem_st16((s ? tS1 : tS0) + lane_off + part * (HB / 2) + q, p + q);
       }
       tmem_wait_st();
-      if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) fence_proxy_async_smem();
+      if (smem_p) fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[BAR_P]);
     }
@@ -836,10 +913,10 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int D, int BK, bool FP4, bool RES>
+template <int D, int BK, int LM>
 cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
-  using L = Smem<D, BK, FP4, RES>;
-  auto k = attn_kernel<D, BK, FP4, RES>;
+  using L = Smem<D, BK, LM>;
+  auto k = attn_kernel<D, BK, LM>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nQb, a.B * a.H);
@@ -851,12 +928,13 @@ cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s)
 }  // namespace
 
 cudaError_t launch_attn(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
-  if (a.d == 64 && a.bk == 64) return launch_d<64, 64, false, false>(a, maps, s);
-  if (a.d == 64 && a.bk == 128) return launch_d<64, 128, false, false>(a, maps, s);
-  if (a.d == 128 && a.bk == 64) return launch_d<128, 64, false, false>(a, maps, s);
-  if (a.low == TA_LOW_NVFP4) return launch_d<128, 128, true, false>(a, maps, s);
-  if (a.low == TA_LOW_NVFP4_RES) return launch_d<128, 128, true, true>(a, maps, s);
-  return launch_d<128, 128, false, false>(a, maps, s);
+  if (a.d == 64 && a.bk == 64) return launch_d<64, 64, LM_IMAGE>(a, maps, s);
+  if (a.d == 64 && a.bk == 128) return launch_d<64, 128, LM_IMAGE>(a, maps, s);
+  if (a.d == 128 && a.bk == 64) return launch_d<128, 64, LM_IMAGE>(a, maps, s);
+  if (a.low == TA_LOW_NVFP4) return launch_d<128, 128, LM_NVFP4>(a, maps, s);
+  if (a.low == TA_LOW_NVFP4_RES) return launch_d<128, 128, LM_NVFP4_RES>(a, maps, s);
+  if (a.low == TA_LOW_FP8_E4M3 && a.bq == 128) return launch_d<128, 128, LM_FP8>(a, maps, s);
+  return launch_d<128, 128, LM_IMAGE>(a, maps, s);
 }
 
 }  // namespace ta

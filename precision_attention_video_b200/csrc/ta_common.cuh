@@ -185,6 +185,30 @@ __device__ __forceinline__ void mma_nvfp4_ss(uint32_t d_tmem, uint64_t adesc, ui
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 (e4m3 operands, fp32 D).
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D[tmem] (+)= (A * SFA) * (B * SFB)^T, kind::mxf8f6f4: e4m3 operands, one
+// UE8M0 (power-of-two) scale per 32 elements along K, scale factors in TMEM.
+__device__ __forceinline__ void mma_mxf8_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
 // Shared memory [32 rows][16 bytes] -> TMEM lanes 0..31 of every 32-lane
 // subpartition (replicated 4x), 4 columns: the scale-factor layout of an
 // M = 128 block-scaled MMA operand (row 32*m1 + m0 at lane m0, column m1,
@@ -211,6 +235,17 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
 // [17,23), M >> 4 at [24,29), K-major operands, scale-factor ids 0, K = 64.
 __host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor of kind::f8f6f4: A, B e4m3 (format 0), fp32 D (bits
+// [4,6) = 1), K-major operands.
+__host__ __device__ constexpr uint32_t idesc_f8(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// Instruction descriptor of kind::mxf8f6f4 (block scaled): A, B e4m3, B
+// MN-major (bit 16), scale format UE8M0 (bit 23), scale-factor ids 0.
+__host__ __device__ constexpr uint32_t idesc_mxf8_bmn(int M, int N) {
+  return (1u << 16) | (1u << 23) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // Instruction descriptor of kind::f16 with bf16 A/B, fp32 D, dense.

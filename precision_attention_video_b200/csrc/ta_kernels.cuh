@@ -66,6 +66,10 @@ struct AttnArgs {
   const uint8_t* rq_sf;
   const uint8_t* rk_sf;
   const uint8_t* rv_sf;
+  // per-tile power-of-two scales of the FP8 copies: Q [BH, nQb], K / V [BH, nKb]
+  const float* q_s8;
+  const float* k_s8;
+  const float* v_s8;
   int Np;
 };
 
