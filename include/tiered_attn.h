@@ -88,7 +88,7 @@ typedef struct {
 #define TA_DEBUG_DROP_FIRST_K 1
 
 /* Device pointers into a planned workspace (see tiered_attn_plan_views).
- * BH = B*H, nQb = ceil(N/block_q), nKb = ceil(N/block_k), Np = 16*ceil(N/16).
+ * BH = B*H, nQb = ceil(N/block_q), nKb = ceil(N/block_k), Np = 32*ceil(N/32).
  * Pointers of data the configured low format does not produce are NULL. */
 typedef struct {
   int32_t* status;           /* int32[4]: [0] ta_status of the last kernel error */
@@ -108,7 +108,8 @@ typedef struct {
    * NVFP4 copies: Q, K codes packed two per byte along d, u8 [BH, N, d/2]
    * (element 2c in the low nibble), scales ue4m3 u8 [BH, N, d/16];
    * V codes transposed and packed along tokens, u8 [BH, d, Np/2], scales
-   * u8 [BH, Np/16, d] (groups of 16 tokens from token 0, zero past N). */
+   * u8 [BH, Np/16, d] (groups of 16 tokens from token 0; codes and scales of
+   * tokens past N are zero, and the pitch Np keeps rows 16-byte aligned). */
   uint8_t* q_codes; uint8_t* k_codes; uint8_t* v_codes;
   void*    q_scales; void* k_scales; void* v_scales;
   /* residual NVFP4 copies (TA_LOW_NVFP4_RES), same layouts as above */

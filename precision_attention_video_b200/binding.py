@@ -199,7 +199,7 @@ def plan_views(p: ta_params, ws: torch.Tensor) -> Dict[str, torch.Tensor]:
     N, d = p.N, p.d
     nqb = -(-N // p.block_q)
     nkb = -(-N // p.block_k)
-    Np = 16 * (-(-N // 16))
+    Np = 32 * (-(-N // 32))
     u8, i32, f64, f32, b16 = torch.uint8, torch.int32, torch.float64, torch.float32, torch.bfloat16
     shapes = {
         "status": (i32, (4,)), "qbar": (f64, (BH, nqb, d)), "kbar": (f64, (BH, nkb, d)),

@@ -26,7 +26,9 @@ Shape shape_of(const ta_params* p) {
   s.d = p->d;
   s.nQb = (p->N + p->block_q - 1) / p->block_q;
   s.nKb = (p->N + p->block_k - 1) / p->block_k;
-  s.Np = 16 * ((p->N + 15) / 16);
+  // token pitch of the transposed NVFP4 V copy: a multiple of 32 tokens, so that
+  // its rows (Np/2 bytes) meet TMA's 16-byte stride rule
+  s.Np = 32 * ((p->N + 31) / 32);
   return s;
 }
 

@@ -201,10 +201,11 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const PlanArgs a) {
       } else {
         // V: groups of 16 tokens per column; codes [BH, D, Np/2] (transposed),
         // scales [BH, Np/16, D].  Thread map: column slow, group fast.
-        const int ng = (nrows + 15) / 16;
+        // every group of 16 tokens below the padded pitch Np: groups past N come
+        // out as zero codes with a zero scale
         for (int idx = tid; idx < D * (R / 16); idx += kThreads) {
           const int c = idx / (R / 16), g = idx % (R / 16);
-          if (g >= ng) continue;
+          if (r0 + g * 16 >= a.Np) continue;
           float x[16], dqv[16];
           uint32_t pk[2], scc;
 #pragma unroll

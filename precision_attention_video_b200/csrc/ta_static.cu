@@ -92,7 +92,7 @@ extern "C" ta_status tiered_attn_route_noalloc(const ta_params* p, const void* Q
   a.R = p->block_q > p->block_k ? p->block_q : p->block_k;
   a.nQb = (int)nQb;
   a.nKb = (int)nKb;
-  a.Np = 16 * ((p->N + 15) / 16);
+  a.Np = 32 * ((p->N + 31) / 32);
   a.n_tau = p->n_thresholds;
   for (int i = 0; i < 3; ++i) a.tau[i] = i < p->n_thresholds ? p->tau[i] : 0.0;
   a.keep_diag = p->keep_diag_full;

@@ -93,6 +93,20 @@ def check_lists(tiers: np.ndarray, counts: np.ndarray, lists: np.ndarray, mass: 
         assert pos == tiers.shape[1]
 
 
+def check_vt(gpu_codes_packed: np.ndarray, gpu_sc: np.ndarray, o_codes: np.ndarray,
+             o_sc: np.ndarray):
+    """GPU transposed NVFP4 V copy ([d, Np/2] packed, scales [Np/16, d]) equals
+    the oracle's column copy ([Np16, d], scales [Np16/16, d]); the extra pitch
+    tokens are zero."""
+    vt = unpack_fp4(gpu_codes_packed).T
+    n = o_codes.shape[0]
+    np.testing.assert_array_equal(vt[:n], o_codes)
+    assert not vt[n:].any()
+    g = o_sc.shape[0]
+    np.testing.assert_array_equal(gpu_sc[:g], o_sc)
+    assert not gpu_sc[g:].any()
+
+
 def out_errors(O_gpu: np.ndarray, O_ref: np.ndarray):
     m = ~np.isnan(O_ref[:, 0])
     a, r = O_gpu[m], O_ref[m]

@@ -12,8 +12,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import (assert_out_close, check_lists, compare_tiers, inputs, oracle_head,
-                         run_gpu, to64, unpack_fp4)
+from gpu_helpers import (assert_out_close, check_lists, check_vt, compare_tiers, inputs,
+                         oracle_head, run_gpu, to64, unpack_fp4)
 from oracle import quant as Qz
 
 pytestmark = pytest.mark.gpu
@@ -53,9 +53,8 @@ def _plan_parity(cfg, Q, K, V, views, heads):
                     np.testing.assert_array_equal(unpack_fp4(views[f"{pre}{t}_codes"][bh].numpy()),
                                                   qt[f"{pre}{t}_codes"])
                     np.testing.assert_array_equal(views[f"{pre}{t}_scales"][bh].numpy(), qt[f"{pre}{t}_sc"])
-                vt = unpack_fp4(views[f"{pre}v_codes"][bh].numpy()).T
-                np.testing.assert_array_equal(vt, qt[f"{pre}v_codes"])
-                np.testing.assert_array_equal(views[f"{pre}v_scales"][bh].numpy(), qt[f"{pre}v_sc"])
+                check_vt(views[f"{pre}v_codes"][bh].numpy(), views[f"{pre}v_scales"][bh].numpy(),
+                         qt[f"{pre}v_codes"], qt[f"{pre}v_sc"])
             for t in "qkv":
                 if f"d{t}" in views:   # bf16 images exist only where a tile path reads them
                     np.testing.assert_array_equal(to64(views[f"d{t}"][bh]), qt[f"d{t}"][:cfg.N])
