@@ -15,37 +15,40 @@
 //               kbar_b / vbar_b into a "pseudo-key" tile, so a skip chunk costs
 //               one tile of MMA for up to BK skipped blocks and never touches
 //               their K / V;
-//   warp 4S+2   MMA issuer: tcgen05.mma kind::f16, S = Q K^T into a double-
-//               buffered TMEM accumulator, O += P V into a TMEM accumulator;
-//               completion is signalled with tcgen05.commit on mbarriers;
+//   warp 4S+2   MMA issuer: S = Q K^T into a double-buffered TMEM accumulator
+//               and O += P V into a TMEM accumulator, one thread issuing
+//               tcgen05.mma: kind::f16 for full and skip tiles and for FP8
+//               tiles of the small shapes (bf16 images of the codes);
+//               kind::mxf4nvf4.block16 for NVFP4 tiles (ue4m3 scales copied to
+//               TMEM with tcgen05.cp; three MMAs per product on residual
+//               tiles); kind::f8f6f4 for FP8 S and kind::mxf8f6f4 for FP8 PV
+//               (V's power-of-two tile scale as a UE8M0 block scale).
+//               Completion is signalled with tcgen05.commit on mbarriers;
 //   warps 0..4S-1 softmax (S = min(d, BK)/32 column parts): the S warps with
 //               equal w%4 share TMEM lanes 32(w%4).. (query rows) and split
 //               each row's columns into S parts of 32; they swap their part
 //               maxima through shared memory and a named barrier.  Each thread
 //               loads its part of an S row, keeps the running max m and its
-//               part of the sum l, forms
-//               P' = 2^o exp(s - m'), rounds it as the tile's tier demands
-//               (bf16; e4m3; NVFP4 per 16 keys), rescales O in TMEM when m
-//               grows, and hands P' to the PV MMA: bf16 P' is stored into the
-//               TMEM columns of its own S buffer (the A operand of a TMEM x
-//               shared-memory MMA), so the two S buffers double as two P
-//               buffers; NVFP4 P' (codes + scales) goes to one of two small
-//               shared-memory buffers.  A tile's softmax waits for the previous
-//               tile's PV only when it must rescale O.
+//               part of the sum l, and hands the rest of the tile to a tail
+//               specialised for the tile's P format: P' = 2^o exp(s - m'),
+//               rounded as the tier demands (bf16; e4m3; NVFP4 per 16 keys,
+//               plus its residual), O rescaled in TMEM when m grew, and P'
+//               handed to the PV MMA: bf16 P' is stored into the TMEM columns
+//               of its own S buffer (the A operand of a TMEM x shared-memory
+//               MMA), NVFP4 / FP8 P' into one of two shared-memory buffers.
 //               The epilogue writes O = acc / l in bf16.
 //
-// Low tiles run through the same bf16 tensor-core path on the exact bf16
-// values of their dequantised FP8 / NVFP4 operands and of the quantised P'
-// (every FP8 and NVFP4 value is exactly representable in bf16), so the
-// products equal those of the low-precision operands up to fp32 accumulation
-// order.  All waits are bounded: a wait that runs out sets the CTA's abort
-// flag and the workspace status word, every role leaves its loop, in-flight
-// copies and MMAs are drained (bounded), and TMEM is freed before return.
+// All waits are bounded: a wait that runs out sets the CTA's abort flag and
+// the workspace status word, every role leaves its loop, in-flight copies and
+// MMAs are drained (bounded), and TMEM is freed before return.
 #include "ta_common.cuh"
 #include "ta_kernels.cuh"
+#include "ta_attn_common.cuh"
 
 namespace ta {
 namespace {
+
+using namespace tile;
 
 // Softmax warps: warp w owns TMEM lanes 32*(w%4).. (query rows) and column
 // part w/4 of those rows; kSplit parts per row (32 columns of S and of O each).
@@ -58,81 +61,6 @@ struct Roles {
   static constexpr int kMmaWarp = kSoftmaxWarps + 2;
   static constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
 };
-
-enum TileKind { KIND_FULL = 0, KIND_LOW = 1, KIND_SKIP = 2, KIND_RES = 3 };
-
-struct RowPlan {
-  int n_full, n_res, n_low, n_skip;
-  int T;             // number of tiles (skip blocks chunked by BK)
-  const int* list;   // this row's list
-};
-
-// Tile t of a row: its kind and the position of its (first) key block in the
-// row's list.  Kept tiles come in list order (full, residual, low); skipped
-// blocks follow in chunks of BK.
-template <int BK>
-__device__ __forceinline__ void tile_of(const RowPlan& rp, int t, int& kind, int& first) {
-  const int kept = rp.n_full + rp.n_res + rp.n_low;
-  if (t < kept) {
-    kind = t < rp.n_full ? KIND_FULL : (t < rp.n_full + rp.n_res ? KIND_RES : KIND_LOW);
-    first = t;
-  } else {
-    kind = KIND_SKIP;
-    first = kept + (t - kept) * BK;
-  }
-}
-
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// 2^x on the FMA pipe, to share the exponentials with the MUFU unit:
-// x = n + f with n = round(x) (adding 1.5 * 2^23 leaves round(x) in the low
-// mantissa bits) and f in [-0.5, 0.5]; 2^f from a degree-5 polynomial fitted
-// here for relative error (max 1.8e-7 on [-0.5, 0.5], evaluated in fp32); 2^n
-// added to the exponent field.  Inputs below -125 return 0; x <= 127.
-// Every kPolyEvery-th exponential of a softmax thread uses exp2_poly (0: none).
-// Measured on this kernel: a polynomial costs more issue slots than it saves
-// on the MUFU pipe, so it is off.
-constexpr int kPolyEvery = 0;
-
-[[maybe_unused]] __device__ __forceinline__ float exp2_poly(float x) {
-  const float xc = fmaxf(x, -125.0f);
-  const float t = xc + 12582912.0f;
-  const float n = t - 12582912.0f;
-  const float f = xc - n;
-  float p = 0.0013281889259815216f;
-  p = fmaf(p, f, 0.00967559777200222f);
-  p = fmaf(p, f, 0.05550696700811386f);
-  p = fmaf(p, f, 0.24022118747234344f);
-  p = fmaf(p, f, 0.6931470036506653f);
-  p = fmaf(p, f, 1.0000001192092896f);
-  const int ni = __float_as_int(t) - 0x4B400000;
-  const float r = __int_as_float(__float_as_int(p) + (ni << 23));
-  return x < -125.0f ? 0.0f : r;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Eight floats to eight e2m1 codes (RNE, satfinite) in one word, element i in
-// nibble i.
-__device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(r)
-      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
-  return r;
-}
 
 // Named barrier over `count` threads that also ANDs a predicate across them:
 // the warps of a softmax pair leave their loop together or not at all.
@@ -149,21 +77,7 @@ __device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
   return out != 0;
 }
 
-// Two e2m1 codes (low nibble first) to f16x2 (exact).
-__device__ __forceinline__ __half2 e2m1x2_to_half2(uint32_t codes) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
-      : "=r"(r)
-      : "r"(codes));
-  return *reinterpret_cast<__half2*>(&r);
-}
-
 // Shared-memory layout (offsets from a 1024-aligned base).
-// Low-tier execution mode of a kernel instance.
-enum LowMode { LM_IMAGE = 0, LM_NVFP4 = 1, LM_NVFP4_RES = 2, LM_FP8 = 3 };
-
 template <int D, int BK, int LM>
 struct Smem {
   static constexpr bool FP4 = (LM == LM_NVFP4 || LM == LM_NVFP4_RES);
@@ -200,42 +114,142 @@ enum {
   BAR_VE0 = 13, BAR_VE1 = 14
 };
 
-// TMEM columns of the NVFP4 scale factors (4 columns per 64-element K chunk,
-// 2 chunks per operand), after S0, S1 and O.
-template <int D, int BK, bool RES>
-struct TmemSf {
-  // FP8 tiles: UE8M0 scale factors of P (constant 2^0) and of V (per stage)
-  static constexpr __device__ uint32_t sfaP8() { return 2 * BK + D; }
-  static constexpr __device__ uint32_t sfbV8(int s) { return 2 * BK + D + 4 + 4 * s; }
-  static constexpr uint32_t NC = RES ? 2 : 1;   // copies (first + residual)
-  static constexpr uint32_t kBase = 2 * BK + D;
-  // query copy c; K copy c of stage s; V copy c of stage s; P copy c of buffer b
-  static constexpr __device__ uint32_t sfaQ(int c) { return kBase + 8 * c; }
-  static constexpr __device__ uint32_t sfbK(int s, int c) { return kBase + 8 * NC + 8 * (s * NC + c); }
-  static constexpr __device__ uint32_t sfbV(int s, int c) { return kBase + 24 * NC + 8 * (s * NC + c); }
-  static constexpr __device__ uint32_t sfaP(int b, int c) { return kBase + 40 * NC + 8 * (b * NC + c); }
-  static constexpr uint32_t kEnd = kBase + 56 * NC;  // <= 512 (496 with residual copies)
+// Formats of P' in the softmax's tile tail.
+enum { PK_BF16 = 0, PK_SKIP = 1, PK_FP4 = 2, PK_RES = 3, PK_F8 = 4, PK_IMG_F8 = 5 };
+
+// What the tail of one tile's softmax needs (one thread: one query row, one
+// column part of HB keys).
+struct SoftmaxTail {
+  float* x;                 // the part's S values (masked to -inf past nv)
+  int nv;                   // valid columns of this part
+  float c2t, mc;            // P' = 2^(s * c2t - mc)
+  float alpha;              // exp(m - m') of this row
+  int t;                    // tile index in the row
+  const int* list;          // list entries of this part's columns
+  int N;
+  uint64_t* bars;
+  AbortCtx ctx;
+  int row_bar;
+  unsigned char* sm;
+  uint32_t tS, tO;          // this lane's S buffer and O accumulator
+  int part, quarter, lane, r;
+  const float2* sc_tab;     // ue4m3 code -> (value, 1 / value)
 };
 
-// NVFP4 tiles in shared memory: codes [rows][64 B] with 64-byte swizzle, then
-// the two [32][16 B] scale-factor blocks at +kFp4Sf.
-constexpr int kFp4Sf = 128 * 64;
-
-// Gather the ue4m3 scales of `nrows` rows (row-major, 8 bytes = 8 groups of 16
-// along d = 128) into the two [32][16 B] blocks at `dst`: row 32*m1 + m0 of K
-// chunk c (groups 4c..4c+3) at dst + c*512 + m0*16 + m1*4.  Rows past
-// `nrows` get zero scales.
-__device__ __forceinline__ void gather_row_sf(unsigned char* dst, const uint8_t* src, int nrows,
-                                              int lane) {
+// Tail of one tile's softmax for one P format, in straight-line code:
+// P' = 2^o exp(s - m') and its part row sum, P' rounded as the tier demands,
+// O rescaled when the maximum grew (after the previous PV), and P' handed to
+// the PV MMA (bf16 in the S buffer's TMEM columns; NVFP4 / FP8 in a shared
+// memory buffer).  False when the CTA aborts.
+template <int PK, int D, int BK, int LM>
+__device__ __forceinline__ bool softmax_tail(const SoftmaxTail q, float& psum) {
+  using L = Smem<D, BK, LM>;
+  constexpr int kSplit = Roles<D, BK>::kSplit;
+  constexpr int HB = BK / kSplit, HD = D / kSplit;
+  constexpr int kBarThreads = 32 * kSplit;
+  constexpr bool smem_p = (PK == PK_FP4 || PK == PK_RES || PK == PK_F8);
+  const int s = q.t & 1;
+  float* x = q.x;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int rr = lane * 4 + i;
-    uint2 v = make_uint2(0u, 0u);
-    if (rr < nrows) v = *reinterpret_cast<const uint2*>(src + (int64_t)rr * 8);
-    const int off = (rr & 31) * 16 + (rr >> 5) * 4;
-    *reinterpret_cast<uint32_t*>(dst + off) = v.x;
-    *reinterpret_cast<uint32_t*>(dst + 512 + off) = v.y;
+  for (int c = 0; c < HB; ++c) x[c] = fast_exp2(fmaf(x[c], q.c2t, -q.mc));
+  if constexpr (PK == PK_SKIP) {
+    // pooled keys weigh n_j
+#pragma unroll
+    for (int c = 0; c < HB; ++c) {
+      if (c < q.nv) {
+        const int j = q.list[c];
+        x[c] *= (float)min(BK, q.N - j * BK);
+      }
+    }
   }
+  float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int c = 0; c < HB; ++c) ps[c & 3] += x[c];
+  psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+
+  // round P' as the tier demands
+  uint32_t p[(PK == PK_RES) ? 13 : (HB / 2)];
+  if constexpr (PK == PK_FP4 || PK == PK_RES) {
+    // codes of this part (HB = 32 keys, half an MMA K chunk) in p[0..3], its
+    // two ue4m3 scales in p[4]; the residual copy in p[8..12]
+    static_assert(HB == 32, "NVFP4 parts are 32 keys");
+    p[4] = nvfp4_quant32(x, q.sc_tab, p);
+    if constexpr (PK == PK_RES) p[12] = nvfp4_residual32(x, p, p[4], q.sc_tab, p + 8);
+  } else if constexpr (PK == PK_F8) {
+    // e4m3 codes of P' (scale 1), four per word
+#pragma unroll
+    for (int c = 0; c < HB; c += 4)
+      p[c / 4] = cvt_e4m3x2(x[c], x[c + 1]) | (cvt_e4m3x2(x[c + 2], x[c + 3]) << 16);
+  } else if constexpr (PK == PK_IMG_F8) {
+    // e4m3 rounding of P', carried exactly in bf16
+#pragma unroll
+    for (int c = 0; c < HB; c += 2) {
+      const float2 f = e4m3x2_to_float2(cvt_e4m3x2(x[c], x[c + 1]));
+      p[c / 2] = pack_bf16(f.x, f.y);
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < HB; c += 2) p[c / 2] = pack_bf16(x[c], x[c + 1]);
+  }
+
+  // O may be rescaled only once the previous tile's PV is done; a shared
+  // memory P buffer may be rewritten once the PV two tiles back is done.  The
+  // warps sharing these rows see the same maxima, so they agree on `rescale`
+  // and on `reuse` and wait (and leave on abort) together.
+  const bool rescale = (q.t > 0) && __any_sync(0xffffffffu, q.alpha != 1.0f);
+  const bool reuse = smem_p && q.t >= 2;
+  if (rescale || reuse) {
+    bool ok2 = true;
+    if (reuse) ok2 = mbar_wait(&q.bars[BAR_PD0 + s], ((q.t >> 1) - 1) & 1, q.ctx, 7);
+    if (rescale && ok2) ok2 = mbar_wait(&q.bars[BAR_PD0 + (s ^ 1)], ((q.t - 1) >> 1) & 1, q.ctx, 9);
+    ok2 = __all_sync(0xffffffffu, ok2);
+    ok2 = bar_and(q.row_bar, kBarThreads, ok2);
+    if (!ok2) return false;
+  }
+  if (rescale) {
+    tc_fence_after();
+#pragma unroll
+    for (int c0 = 0; c0 < HD; c0 += 32) {
+      uint32_t raw[32];
+      tmem_ld32(q.tO + q.part * HD + c0, raw);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * q.alpha);
+      tmem_st32(q.tO + q.part * HD + c0, raw);
+    }
+  }
+  if constexpr (PK == PK_FP4 || PK == PK_RES) {
+    // NVFP4 P part: 16 bytes of codes into the 64-byte-swizzled tile, 2
+    // scale bytes into the scale-factor block of K chunk part/2 (and the same
+    // for the residual copy on residual tiles)
+    unsigned char* pbuf = q.sm + L::oP + s * L::NC * L::kPfp4;
+    const uint32_t off = q.r * 64 + ((q.part ^ ((q.r >> 1) & 3)) * 16);
+    const uint32_t soff = kFp4Sf + (q.part >> 1) * 512 + q.lane * 16 + q.quarter * 4 + (q.part & 1) * 2;
+    *reinterpret_cast<uint4*>(pbuf + off) = make_uint4(p[0], p[1], p[2], p[3]);
+    *reinterpret_cast<uint16_t*>(pbuf + soff) = (uint16_t)p[4];
+    if constexpr (PK == PK_RES) {
+      *reinterpret_cast<uint4*>(pbuf + L::kPfp4 + off) = make_uint4(p[8], p[9], p[10], p[11]);
+      *reinterpret_cast<uint16_t*>(pbuf + L::kPfp4 + soff) = (uint16_t)p[12];
+    }
+  } else if constexpr (PK == PK_F8) {
+    // FP8 P part: 32 codes into the 128-byte-swizzled tile of buffer s
+    unsigned char* pbuf = q.sm + L::oP + s * L::kF8;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int ch = q.part * 2 + h;
+      *reinterpret_cast<uint4*>(pbuf + q.r * 128 + ((ch ^ (q.r & 7)) * 16)) =
+          make_uint4(p[h * 4 + 0], p[h * 4 + 1], p[h * 4 + 2], p[h * 4 + 3]);
+    }
+  } else {
+    // bf16 P' of this part into the S buffer's first BK/2 columns (every
+    // part has loaded its S columns before the row barrier)
+#pragma unroll
+    for (int h = 0; h < HB / 2; h += 16) tmem_st16(q.tS + q.part * (HB / 2) + h, p + h);
+  }
+  if constexpr (smem_p) fence_proxy_async_smem();
+  tmem_wait_st();
+  tc_fence_before();
+  mbar_arrive(&q.bars[BAR_P]);
+  return true;
 }
 
 template <int D, int BK, int LM>
@@ -690,183 +704,47 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
       const float alpha = fast_exp2((m - m_new) * c2);  // 0 on the first tile
       const float mc = m_new * c2 - o_off;              // P' = 2^(s*c2 - mc)
       const float c2t = c2 * sqk;                       // this tile's S -> log2 units
-      if constexpr (kPolyEvery > 0) {
-#pragma unroll
-        for (int c = 0; c < HB; ++c) {
-          const float e = fmaf(x[c], c2t, -mc);
-          x[c] = (c % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) ? exp2_poly(e) : fast_exp2(e);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < HB; ++c) x[c] = fast_exp2(fmaf(x[c], c2t, -mc));
-      }
+      SoftmaxTail q;
+      q.x = x;
+      q.nv = nv;
+      q.c2t = c2t;
+      q.mc = mc;
+      q.alpha = alpha;
+      q.t = t;
+      q.list = rp.list + first + part * HB;
+      q.N = a.N;
+      q.bars = bars;
+      q.ctx = ctx;
+      q.row_bar = row_bar;
+      q.sm = sm;
+      q.tS = (s ? tS1 : tS0) + lane_off;
+      q.tO = tO + lane_off;
+      q.part = part;
+      q.quarter = quarter;
+      q.lane = lane;
+      q.r = r;
+      q.sc_tab = sc_tab;
+      float psum = 0.0f;
+      bool ok3;
       if (kind == KIND_SKIP) {
-#pragma unroll
-        for (int c = 0; c < HB; ++c) {
-          if (c < nv) {
-            const int j = rp.list[first + part * HB + c];
-            x[c] *= (float)min(BK, a.N - j * BK);
-          }
+        ok3 = softmax_tail<PK_SKIP, D, BK, LM>(q, psum);
+      } else if (kind == KIND_FULL) {
+        ok3 = softmax_tail<PK_BF16, D, BK, LM>(q, psum);
+      } else {
+        if constexpr (RES) {
+          ok3 = (kind == KIND_RES) ? softmax_tail<PK_RES, D, BK, LM>(q, psum)
+                                   : softmax_tail<PK_FP4, D, BK, LM>(q, psum);
+        } else if constexpr (FP4) {
+          ok3 = softmax_tail<PK_FP4, D, BK, LM>(q, psum);
+        } else if constexpr (F8) {
+          ok3 = softmax_tail<PK_F8, D, BK, LM>(q, psum);
+        } else {
+          ok3 = softmax_tail<PK_IMG_F8, D, BK, LM>(q, psum);
         }
       }
-      float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-      for (int c = 0; c < HB; ++c) ps[c & 3] += x[c];
-      l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+      if (!ok3) { aborted = true; break; }
+      l = l * alpha + psum;
       m = m_new;
-
-      // round P' as the tier demands, into bf16 pairs (or NVFP4 codes)
-      uint32_t p[HB / 2];
-      if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
-        // codes of this part (HB = 32 keys, half an MMA K chunk) in p[0..3],
-        // ue4m3 scales of its 2 groups in p[4]
-        uint32_t scw = 0u;
-#pragma unroll
-        for (int g = 0; g < HB / 16; ++g) {
-          float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-          for (int i = 0; i < 16; ++i) am[i & 3] = fmaxf(am[i & 3], x[g * 16 + i]);
-          const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
-          const uint32_t scc = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xFFu;
-          const float inv = sc_tab[scc].y;
-          scw |= scc << (8 * g);
-#pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            float y[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(x[g * 16 + w * 8 + i], inv);
-            p[g * 2 + w] = cvt_e2m1x8(y);
-          }
-        }
-        p[HB / 8] = scw;
-        if (RES && kind == KIND_RES) {
-          // second copy: NVFP4 of the residual fp32(P' - deq(P1)), in p[8..12]
-          uint32_t scw2 = 0u;
-#pragma unroll
-          for (int g = 0; g < HB / 16; ++g) {
-            const float sc1 = sc_tab[(scw >> (8 * g)) & 0xFFu].x;
-            float rr[16];
-#pragma unroll
-            for (int w = 0; w < 2; ++w) {
-#pragma unroll
-              for (int bb = 0; bb < 4; ++bb) {
-                const float2 f = __half22float2(e2m1x2_to_half2(p[g * 2 + w] >> (8 * bb)));
-                const int c = w * 8 + 2 * bb;
-                rr[c] = __fsub_rn(x[g * 16 + c], __fmul_rn(f.x, sc1));
-                rr[c + 1] = __fsub_rn(x[g * 16 + c + 1], __fmul_rn(f.y, sc1));
-              }
-            }
-            float am = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(rr[i]));
-            const uint32_t scc2 = cvt_e4m3x2(__fdiv_rn(am, 6.0f), 0.0f) & 0xFFu;
-            const float inv2 = sc_tab[scc2].y;
-            scw2 |= scc2 << (8 * g);
-#pragma unroll
-            for (int w = 0; w < 2; ++w) {
-              float y[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(rr[w * 8 + i], inv2);
-              p[8 + g * 2 + w] = cvt_e2m1x8(y);
-            }
-          }
-          p[8 + HB / 8] = scw2;
-        }
-      } else if (F8 && kind == KIND_LOW) {
-        // e4m3 codes of P' (scale 1), four per word
-#pragma unroll
-        for (int c = 0; c < HB; c += 4)
-          p[c / 4] = cvt_e4m3x2(x[c], x[c + 1]) | (cvt_e4m3x2(x[c + 2], x[c + 3]) << 16);
-      } else if (kind == KIND_LOW && a.low == TA_LOW_FP8_E4M3) {
-#pragma unroll
-        for (int c = 0; c < HB; c += 2) {
-          const float2 f = e4m3x2_to_float2(cvt_e4m3x2(x[c], x[c + 1]));
-          p[c / 2] = pack_bf16(f.x, f.y);
-        }
-      } else if (kind == KIND_LOW) {
-#pragma unroll
-        for (int g = 0; g < HB; g += 16) {
-          float amax = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) amax = fmaxf(amax, x[g + i]);
-          const uint32_t scc = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xFFu;
-          const float sc = e4m3_to_float(scc);
-          const float inv = (sc > 0.0f) ? __frcp_rn(sc) : 0.0f;
-          const __half2 sc2 = __float2half2_rn(sc);  // exact: a ue4m3 value
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            const uint32_t cc = cvt_e2m1x2(__fmul_rn(x[g + i], inv), __fmul_rn(x[g + i + 1], inv));
-            const float2 f = __half22float2(__hmul2(e2m1x2_to_half2(cc), sc2));  // exact
-            p[(g + i) / 2] = pack_bf16(f.x, f.y);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < HB; c += 2) p[c / 2] = pack_bf16(x[c], x[c + 1]);
-      }
-
-      // O may be rescaled only once the previous tile's PV is done; an NVFP4
-      // P buffer may be rewritten once the PV two tiles back is done.  (The
-      // maxima exchange is double-buffered: a slot is rewritten two tiles on,
-      // after every reader has passed the next tile's row barrier.)
-      // The warps sharing these rows see the same maxima, so they agree on
-      // `rescale` and on `reuse` and wait (and leave on abort) together.
-      const bool rescale = (t > 0) && __any_sync(0xffffffffu, alpha != 1.0f);
-      const bool smem_p = (FP4 && (kind == KIND_LOW || kind == KIND_RES)) || (F8 && kind == KIND_LOW);
-      const bool reuse = smem_p && t >= 2;
-      if (rescale || reuse) {
-        bool ok2 = true;
-        if (reuse) ok2 = mbar_wait(&bars[BAR_PD0 + s], ((t >> 1) - 1) & 1, ctx, 7);
-        if (rescale && ok2)
-          ok2 = mbar_wait(&bars[BAR_PD0 + (s ^ 1)], ((t - 1) >> 1) & 1, ctx, 9);
-        ok2 = __all_sync(0xffffffffu, ok2);
-        ok2 = bar_and(row_bar, kBarThreads, ok2);
-        if (!ok2) { aborted = true; break; }
-      }
-      if (rescale) {
-        tc_fence_after();
-#pragma unroll
-        for (int c0 = 0; c0 < HD; c0 += 32) {
-          uint32_t raw[32];
-          tmem_ld32(tO + lane_off + part * HD + c0, raw);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * alpha);
-          tmem_st32(tO + lane_off + part * HD + c0, raw);
-        }
-      }
-      if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
-        // NVFP4 P part: 16 bytes of codes into the 64-byte-swizzled tile, 2
-        // scale bytes into the scale-factor block of K chunk part/2 (and the
-        // same for the residual copy on residual tiles)
-        unsigned char* pbuf = sm + L::oP + s * L::NC * L::kPfp4;
-        const uint32_t off = r * 64 + ((part ^ ((r >> 1) & 3)) * 16);
-        const uint32_t soff = kFp4Sf + (part >> 1) * 512 + lane * 16 + quarter * 4 + (part & 1) * 2;
-        *reinterpret_cast<uint4*>(pbuf + off) = make_uint4(p[0], p[1], p[2], p[3]);
-        *reinterpret_cast<uint16_t*>(pbuf + soff) = (uint16_t)p[HB / 8];
-        if (RES && kind == KIND_RES) {
-          *reinterpret_cast<uint4*>(pbuf + L::kPfp4 + off) = make_uint4(p[8], p[9], p[10], p[11]);
-          *reinterpret_cast<uint16_t*>(pbuf + L::kPfp4 + soff) = (uint16_t)p[8 + HB / 8];
-        }
-      } else if (F8 && kind == KIND_LOW) {
-        // FP8 P part: 32 codes into the 128-byte-swizzled tile of buffer s
-        unsigned char* pbuf = sm + L::oP + s * L::kF8;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int ch = part * 2 + q;
-          *reinterpret_cast<uint4*>(pbuf + r * 128 + ((ch ^ (r & 7)) * 16)) =
-              make_uint4(p[q * 4 + 0], p[q * 4 + 1], p[q * 4 + 2], p[q * 4 + 3]);
-        }
-      } else {
-        // bf16 P' of this part into the S buffer's first BK/2 columns (every
-        // part has loaded its S columns before the row barrier above)
-#pragma unroll
-        for (int q = 0; q < HB / 2; q += 16)
-          tmem_st16((s ? tS1 : tS0) + lane_off + part * (HB / 2) + q, p + q);
-      }
-      tmem_wait_st();
-      if (smem_p) fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bars[BAR_P]);
     }
     if (!aborted) {
       bool ok = mbar_wait(&bars[BAR_PD0 + ((rp.T - 1) & 1)], ((rp.T - 1) >> 1) & 1, ctx, 8);

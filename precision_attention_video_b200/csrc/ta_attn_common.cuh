@@ -1,0 +1,179 @@
+// ta_attn_common.cuh -- pieces shared by the fused attention kernels: the
+// tile walk of a row's compacted list, exponentials and number-format packing
+// of P', and the TMEM / shared-memory layout of NVFP4 block scales.
+#pragma once
+
+#include "ta_common.cuh"
+#include "ta_kernels.cuh"
+
+namespace ta {
+namespace tile {
+
+enum TileKind { KIND_FULL = 0, KIND_LOW = 1, KIND_SKIP = 2, KIND_RES = 3 };
+
+struct RowPlan {
+  int n_full, n_res, n_low, n_skip;
+  int T;             // number of tiles (skip blocks chunked by BK)
+  const int* list;   // this row's list
+};
+
+// Tile t of a row: its kind and the position of its (first) key block in the
+// row's list.  Kept tiles come in list order (full, residual, low); skipped
+// blocks follow in chunks of BK.
+template <int BK>
+__device__ __forceinline__ void tile_of(const RowPlan& rp, int t, int& kind, int& first) {
+  const int kept = rp.n_full + rp.n_res + rp.n_low;
+  if (t < kept) {
+    kind = t < rp.n_full ? KIND_FULL : (t < rp.n_full + rp.n_res ? KIND_RES : KIND_LOW);
+    first = t;
+  } else {
+    kind = KIND_SKIP;
+    first = kept + (t - kept) * BK;
+  }
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Eight floats to eight e2m1 codes (RNE, satfinite) in one word, element i in
+// nibble i.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float* v) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return r;
+}
+
+// Two e2m1 codes (low nibble first) to f16x2 (exact).
+__device__ __forceinline__ __half2 e2m1x2_to_half2(uint32_t codes) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
+      : "=r"(r)
+      : "r"(codes));
+  return *reinterpret_cast<__half2*>(&r);
+}
+
+// Low-tier execution mode of a kernel instance.
+enum LowMode { LM_IMAGE = 0, LM_NVFP4 = 1, LM_NVFP4_RES = 2, LM_FP8 = 3 };
+
+// TMEM columns of the NVFP4 scale factors (4 columns per 64-element K chunk,
+// 2 chunks per operand), after S0, S1 and O.
+template <int D, int BK, bool RES>
+struct TmemSf {
+  // FP8 tiles: UE8M0 scale factors of P (constant 2^0) and of V (per stage)
+  static constexpr __device__ uint32_t sfaP8() { return 2 * BK + D; }
+  static constexpr __device__ uint32_t sfbV8(int s) { return 2 * BK + D + 4 + 4 * s; }
+  static constexpr uint32_t NC = RES ? 2 : 1;   // copies (first + residual)
+  static constexpr uint32_t kBase = 2 * BK + D;
+  // query copy c; K copy c of stage s; V copy c of stage s; P copy c of buffer b
+  static constexpr __device__ uint32_t sfaQ(int c) { return kBase + 8 * c; }
+  static constexpr __device__ uint32_t sfbK(int s, int c) { return kBase + 8 * NC + 8 * (s * NC + c); }
+  static constexpr __device__ uint32_t sfbV(int s, int c) { return kBase + 24 * NC + 8 * (s * NC + c); }
+  static constexpr __device__ uint32_t sfaP(int b, int c) { return kBase + 40 * NC + 8 * (b * NC + c); }
+  static constexpr uint32_t kEnd = kBase + 56 * NC;  // <= 512 (496 with residual copies)
+};
+
+// NVFP4 tiles in shared memory: codes [rows][64 B] with 64-byte swizzle, then
+// the two [32][16 B] scale-factor blocks at +kFp4Sf.
+constexpr int kFp4Sf = 128 * 64;
+
+// Gather the ue4m3 scales of `nrows` rows (row-major, 8 bytes = 8 groups of 16
+// along d = 128) into the two [32][16 B] blocks at `dst`: row 32*m1 + m0 of K
+// chunk c (groups 4c..4c+3) at dst + c*512 + m0*16 + m1*4.  Rows past
+// `nrows` get zero scales.
+__device__ __forceinline__ void gather_row_sf(unsigned char* dst, const uint8_t* src, int nrows,
+                                              int lane) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = lane * 4 + i;
+    uint2 v = make_uint2(0u, 0u);
+    if (rr < nrows) v = *reinterpret_cast<const uint2*>(src + (int64_t)rr * 8);
+    const int off = (rr & 31) * 16 + (rr >> 5) * 4;
+    *reinterpret_cast<uint32_t*>(dst + off) = v.x;
+    *reinterpret_cast<uint32_t*>(dst + 512 + off) = v.y;
+  }
+}
+
+// NVFP4 of 32 non-negative P' values, two groups of 16 keys: sc =
+// ue4m3_rn(fp32(amax / 6)), code = e2m1_rn_satfinite(fp32(x * fp32(1 / sc)))
+// (code 0 when sc = 0).  Codes go to p[0..3] (element i of a word in nibble
+// i); the two scale codes come back in the low 16 bits.  `sc_tab[c]` holds
+// (value, correctly rounded reciprocal) of ue4m3 code c.
+__device__ __forceinline__ uint32_t nvfp4_quant32(const float* x, const float2* sc_tab,
+                                                  uint32_t* p) {
+  uint32_t scw = 0u;
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) am[i & 3] = fmaxf(am[i & 3], x[g * 16 + i]);
+    const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
+    const uint32_t scc = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xFFu;
+    const float inv = sc_tab[scc].y;
+    scw |= scc << (8 * g);
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      float y[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(x[g * 16 + w * 8 + i], inv);
+      p[g * 2 + w] = cvt_e2m1x8(y);
+    }
+  }
+  return scw;
+}
+
+// The residual copy of the same 32 values: r = fp32(x - deq(first copy)),
+// quantised by the same rule on |r| (codes keep the sign).
+__device__ __forceinline__ uint32_t nvfp4_residual32(const float* x, const uint32_t* p,
+                                                     uint32_t scw, const float2* sc_tab,
+                                                     uint32_t* p2) {
+  uint32_t scw2 = 0u;
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const float sc1 = sc_tab[(scw >> (8 * g)) & 0xFFu].x;
+    float rr[16];
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        const float2 f = __half22float2(e2m1x2_to_half2(p[g * 2 + w] >> (8 * bb)));
+        const int c = w * 8 + 2 * bb;
+        rr[c] = __fsub_rn(x[g * 16 + c], __fmul_rn(f.x, sc1));
+        rr[c + 1] = __fsub_rn(x[g * 16 + c + 1], __fmul_rn(f.y, sc1));
+      }
+    }
+    float am = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(rr[i]));
+    const uint32_t scc2 = cvt_e4m3x2(__fdiv_rn(am, 6.0f), 0.0f) & 0xFFu;
+    const float inv2 = sc_tab[scc2].y;
+    scw2 |= scc2 << (8 * g);
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      float y[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(rr[w * 8 + i], inv2);
+      p2[g * 2 + w] = cvt_e2m1x8(y);
+    }
+  }
+  return scw2;
+}
+
+}  // namespace tile
+}  // namespace ta

@@ -68,7 +68,7 @@ struct AbortCtx {
   int* gstatus;          // workspace status word (global), may be null
 };
 
-static __device__ __noinline__ void report_timeout(const AbortCtx& ctx, int site) {
+static __device__ __noinline__ void report_timeout(AbortCtx ctx, int site) {
   *ctx.abort = 1;
   if (ctx.gstatus) {
     if (atomicCAS(ctx.gstatus + ST_CODE, 0, (int)TA_ERR_TIMEOUT) == 0) {
@@ -80,7 +80,7 @@ static __device__ __noinline__ void report_timeout(const AbortCtx& ctx, int site
 
 // Wait for phase `parity` of `bar`; false when the CTA is aborting or the
 // budget ran out (then the abort is raised here).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const AbortCtx& ctx,
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, AbortCtx ctx,
                                           int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
