@@ -488,16 +488,27 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           }
         }
       } else {
-        // gather pooled rows of the skipped blocks into a pseudo K (or V) tile
+        // gather pooled rows of the skipped blocks into a pseudo K (or V)
+        // tile: the chunk's list entries once (lane l holds columns l, l+32,
+        // ...), then every 16-byte piece as an asynchronous copy, all in
+        // flight together (zero fill past the chunk's last column)
         const int cnt = min(BK, rp.n_skip - (first - rp.n_full - rp.n_res - rp.n_low));
-#pragma unroll 8
-        for (int e = lane; e < BK * (D / 8); e += 32) {
-          const int c = e / (D / 8), ch = e % (D / 8);
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (c < cnt) v = *reinterpret_cast<const uint4*>(pooled + (int64_t)rp.list[first + c] * D + ch * 8);
-          const uint32_t off = (ch >> 3) * (BK * 128) + c * 128 + (((ch & 7) ^ (c & 7)) * 16);
-          *reinterpret_cast<uint4*>(st + off) = v;
+        constexpr int kCh = D / 8;             // 16-byte pieces per pooled row
+        constexpr int kCols = 32 / kCh;        // rows per warp-wide step
+        int jl[BK / 32];
+#pragma unroll
+        for (int i = 0; i < BK / 32; ++i) {
+          const int c = lane + 32 * i;
+          jl[i] = (c < cnt) ? rp.list[first + c] : 0;
         }
+#pragma unroll
+        for (int c0 = 0; c0 < BK; c0 += kCols) {
+          const int c = c0 + lane / kCh, ch = lane % kCh;
+          const int j = __shfl_sync(0xffffffffu, jl[c0 / 32], c % 32);
+          const uint32_t off = (ch >> 3) * (BK * 128) + c * 128 + (((ch & 7) ^ (c & 7)) * 16);
+          cp_async16(st + off, pooled + (int64_t)j * D + ch * 8, c < cnt ? 16u : 0u);
+        }
+        cp_async_wait_all();
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
