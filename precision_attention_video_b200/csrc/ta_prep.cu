@@ -16,8 +16,9 @@
 //     fp32(x - dequant(x)) the same way;
 //   * the dequantised values of each copy, in bf16 (exact: at most 6
 //     significant bits), row-major like the input.
-// One CTA per (chunk of R = max(bq, bk) tokens, head); the chunk is staged in
-// shared memory with 16-byte coalesced loads and written back coalesced.
+// One CTA per (chunk of R = max(bq, bk) tokens, head, operand Q / K / V); the
+// chunk is staged in shared memory with 16-byte coalesced loads and written
+// back coalesced.
 #include "ta_common.cuh"
 #include "ta_kernels.cuh"
 
@@ -38,32 +39,38 @@ __device__ __forceinline__ float fp8_pow2_scale(float amax) {
 }
 
 // NVFP4 of one group of 16 values: packed codes (element 2i in the low nibble
-// of byte i), the ue4m3 scale code, and the dequantised values.
+// of byte i) and the ue4m3 scale code; the scale value comes back in `sc`.
 __device__ __forceinline__ void nvfp4_group(const float (&x)[16], uint32_t (&packed)[2],
-                                            uint32_t& sc_code, float (&deq)[16]) {
+                                            uint32_t& sc_code, float& sc) {
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
   sc_code = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xFFu;
-  const float sc = e4m3_to_float(sc_code);
+  sc = e4m3_to_float(sc_code);
   packed[0] = packed[1] = 0u;
-  if (sc == 0.0f) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) deq[i] = 0.0f;
-    return;
-  }
+  if (sc == 0.0f) return;
   const float inv = __frcp_rn(sc);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t c = cvt_e2m1x2(__fmul_rn(x[2 * i], inv), __fmul_rn(x[2 * i + 1], inv));
     packed[i >> 2] |= c << (8 * (i & 3));
+  }
+}
+
+// The values a packed group stands for: code value times the scale (exact in
+// fp32: at most 3 + 4 significant bits).
+__device__ __forceinline__ void nvfp4_dequant(const uint32_t (&packed)[2], float sc,
+                                              float (&deq)[16]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t c = (packed[i >> 2] >> (8 * (i & 3))) & 0xFFu;
     deq[2 * i] = e2m1_value(c & 0xFu) * sc;
     deq[2 * i + 1] = e2m1_value(c >> 4) * sc;
   }
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) prep_kernel(const PlanArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) prep_kernel(const PlanArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   constexpr int LD = D + 8;  // padded row stride (elements)
   const int R = a.R;
@@ -79,8 +86,10 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const PlanArgs a) {
   const int nrows = min(R, a.N - r0);
   const int64_t in_off = (int64_t)b * a.sb + (int64_t)h * a.sh;
   const int64_t bhN = (int64_t)bh * a.N;
+  double* psum = reinterpret_cast<double*>(tile_scale + 8);   // [kThreads] partial block sums
 
-  for (int which = 0; which < 3; ++which) {
+  {
+    const int which = blockIdx.z;
     const __nv_bfloat16* src = (which == 0 ? a.Q : which == 1 ? a.K : a.V) + in_off;
     // ---- stage the chunk (rows past N read as zero) ----
     for (int idx = tid; idx < R * (D / 8); idx += kThreads) {
@@ -91,20 +100,45 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const PlanArgs a) {
     }
     __syncthreads();
 
-    // ---- block sums (fp64, exact for bf16 inputs) and per-column amax ----
+    // ---- block sums (fp64: exact for bf16 inputs, so the order of the
+    // additions does not matter) and per-column amax; kSeg threads share a
+    // (block, column) and each sums a run of its rows ----
     const int blk = (which == 0) ? a.bq : a.bk;
     const int nb = R / blk;
-    for (int w = tid; w < nb * D; w += kThreads) {
+    const int kSeg = kThreads / (nb * D) > 0 ? kThreads / (nb * D) : 1;
+    for (int w0 = tid; w0 < nb * D * kSeg; w0 += kThreads) {
+      const int w = w0 % (nb * D), seg = w0 / (nb * D);
       const int jb = w / D, c = w % D;
       const int rs = jb * blk, re = min(rs + blk, nrows);
-      double s = 0.0;
+      const int len = (blk + kSeg - 1) / kSeg;
+      const int s0 = rs + seg * len, s1 = min(s0 + len, re);
+      double sum = 0.0;
       float amax = 0.0f;
-      for (int r = rs; r < re; ++r) {
+      for (int r = s0; r < s1; ++r) {
         const float x = bf2f(tile[r * LD + c]);
-        s += (double)x;
+        sum += (double)x;
         amax = fmaxf(amax, fabsf(x));
       }
-      red[w] = amax;
+      psum[w0] = sum;
+      red[w0] = amax;
+    }
+    __syncthreads();
+    // nb * D <= 256 = kThreads: one (block, column) per thread
+    const bool mine = tid < nb * D;
+    double s = 0.0;
+    float amax_c = 0.0f;
+    if (mine) {
+      for (int seg = 0; seg < kSeg; ++seg) {
+        s += psum[seg * nb * D + tid];
+        amax_c = fmaxf(amax_c, red[seg * nb * D + tid]);
+      }
+    }
+    __syncthreads();
+    if (mine) {
+      const int w = tid;
+      const int jb = w / D, c = w % D;
+      const int rs = jb * blk, re = min(rs + blk, nrows);
+      red[w] = amax_c;
       if (re > rs) {
         const int gb = r0 / blk + jb;
         const double mean = s / (double)(re - rs);
@@ -120,7 +154,7 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const PlanArgs a) {
       }
     }
     __syncthreads();
-    if (a.low == TA_LOW_NONE) continue;
+    if (a.low == TA_LOW_NONE) return;
 
     uint8_t* codes = which == 0 ? a.q_codes : which == 1 ? a.k_codes : a.v_codes;
     __nv_bfloat16* deq_out = which == 0 ? a.dq : which == 1 ? a.dk : a.dv;
@@ -170,32 +204,39 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const PlanArgs a) {
                                                    : which == 1 ? a.k_scales
                                                                 : a.v_scales);
       uint8_t* rscales = which == 0 ? a.rq_scales : which == 1 ? a.rk_scales : a.rv_scales;
+      __nv_bfloat16* rdeq_out = which == 0 ? a.drq : which == 1 ? a.drk : a.drv;
       if (which < 2) {
         // groups of 16 along d; codes [BH, N, D/2], scales [BH, N, D/16]
         for (int idx = tid; idx < R * (D / 16); idx += kThreads) {
           const int r = idx / (D / 16), g = idx % (D / 16);
           if (r >= nrows) continue;
           __nv_bfloat16* px = tile + r * LD + g * 16;
-          float x[16], dqv[16];
+          float x[16], dqv[16], sc;
           uint32_t pk[2], scc;
 #pragma unroll
           for (int i = 0; i < 16; ++i) x[i] = bf2f(px[i]);
-          nvfp4_group(x, pk, scc, dqv);
+          nvfp4_group(x, pk, scc, sc);
           const int64_t row = bhN + r0 + r;
           *reinterpret_cast<uint2*>(codes + row * (D / 2) + g * 8) = make_uint2(pk[0], pk[1]);
           scales[row * (D / 16) + g] = (uint8_t)scc;
+          if (deq_out != nullptr || res) nvfp4_dequant(pk, sc, dqv);
+          if (deq_out != nullptr) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) px[i] = __float2bfloat16_rn(dqv[i]);
+            for (int i = 0; i < 16; ++i) px[i] = __float2bfloat16_rn(dqv[i]);
+          }
           if (res) {
-            float rr[16], rdq[16];
+            float rr[16], rdq[16], rsc;
 #pragma unroll
             for (int i = 0; i < 16; ++i) rr[i] = __fsub_rn(x[i], dqv[i]);
-            nvfp4_group(rr, pk, scc, rdq);
+            nvfp4_group(rr, pk, scc, rsc);
+            if (rdeq_out != nullptr) nvfp4_dequant(pk, rsc, rdq);
             *reinterpret_cast<uint2*>(rcodes + row * (D / 2) + g * 8) = make_uint2(pk[0], pk[1]);
             rscales[row * (D / 16) + g] = (uint8_t)scc;
-            __nv_bfloat16* pr = rtile + r * LD + g * 16;
+            if (rdeq_out != nullptr) {
+              __nv_bfloat16* pr = rtile + r * LD + g * 16;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) pr[i] = __float2bfloat16_rn(rdq[i]);
+              for (int i = 0; i < 16; ++i) pr[i] = __float2bfloat16_rn(rdq[i]);
+            }
           }
         }
       } else {
@@ -206,41 +247,46 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(const PlanArgs a) {
         for (int idx = tid; idx < D * (R / 16); idx += kThreads) {
           const int c = idx / (R / 16), g = idx % (R / 16);
           if (r0 + g * 16 >= a.Np) continue;
-          float x[16], dqv[16];
+          float x[16], dqv[16], sc;
           uint32_t pk[2], scc;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int r = g * 16 + i;
             x[i] = (r < nrows) ? bf2f(tile[r * LD + c]) : 0.0f;
           }
-          nvfp4_group(x, pk, scc, dqv);
+          nvfp4_group(x, pk, scc, sc);
+          if (deq_out != nullptr || res) nvfp4_dequant(pk, sc, dqv);
           const int64_t tok = r0 + g * 16;
           *reinterpret_cast<uint2*>(codes + ((int64_t)bh * D + c) * (a.Np / 2) + tok / 2) =
               make_uint2(pk[0], pk[1]);
           scales[((int64_t)bh * (a.Np / 16) + tok / 16) * D + c] = (uint8_t)scc;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int r = g * 16 + i;
-            if (r < nrows) tile[r * LD + c] = __float2bfloat16_rn(dqv[i]);
-          }
-          if (res) {
-            float rr[16], rdq[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) rr[i] = __fsub_rn(x[i], dqv[i]);
-            nvfp4_group(rr, pk, scc, rdq);
-            *reinterpret_cast<uint2*>(rcodes + ((int64_t)bh * D + c) * (a.Np / 2) + tok / 2) =
-                make_uint2(pk[0], pk[1]);
-            rscales[((int64_t)bh * (a.Np / 16) + tok / 16) * D + c] = (uint8_t)scc;
+          if (deq_out != nullptr) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int r = g * 16 + i;
-              if (r < nrows) rtile[r * LD + c] = __float2bfloat16_rn(rdq[i]);
+              if (r < nrows) tile[r * LD + c] = __float2bfloat16_rn(dqv[i]);
+            }
+          }
+          if (res) {
+            float rr[16], rdq[16], rsc;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) rr[i] = __fsub_rn(x[i], dqv[i]);
+            nvfp4_group(rr, pk, scc, rsc);
+            if (rdeq_out != nullptr) nvfp4_dequant(pk, rsc, rdq);
+            *reinterpret_cast<uint2*>(rcodes + ((int64_t)bh * D + c) * (a.Np / 2) + tok / 2) =
+                make_uint2(pk[0], pk[1]);
+            rscales[((int64_t)bh * (a.Np / 16) + tok / 16) * D + c] = (uint8_t)scc;
+            if (rdeq_out != nullptr) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int r = g * 16 + i;
+                if (r < nrows) rtile[r * LD + c] = __float2bfloat16_rn(rdq[i]);
+              }
             }
           }
         }
       }
       __syncthreads();
-      __nv_bfloat16* rdeq_out = which == 0 ? a.drq : which == 1 ? a.drk : a.drv;
       if (res && rdeq_out != nullptr) {
         for (int idx = tid; idx < R * (D / 8); idx += kThreads) {
           const int r = idx / (D / 8), c8 = idx % (D / 8);
@@ -267,11 +313,11 @@ template <int D>
 cudaError_t launch_prep_d(const PlanArgs& a, cudaStream_t s) {
   const int chunks = (a.N + a.R - 1) / a.R;
   const size_t smem = (size_t)2 * a.R * (D + 8) * sizeof(__nv_bfloat16) +
-                      (size_t)(kThreads + 8) * sizeof(float);
+                      (size_t)(kThreads + 8) * sizeof(float) + (size_t)kThreads * sizeof(double);
   auto k = prep_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(chunks, a.B * a.H);
+  dim3 grid(chunks, a.B * a.H, 3);
   k<<<grid, kThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
