@@ -42,10 +42,12 @@ METRIC = "dense-equiv attention TFLOPS & ms/layer @32760 tok; % tensor-pipe peak
 UNIT = "TFLOPS"
 L2_BYTES = 126 * 2 ** 20
 
-# DRAM traffic of one tiered_attn_forward launch on this workload, from the ncu
-# capture summarised in profiles/ (dram__bytes_read.sum + dram__bytes_write.sum);
-# valid only for the kernel source it was measured on.
-ATTN_TRAFFIC = {"source_sha1": None, "bytes_per_launch": None}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one forward
+# launch of the 480p-video-like layer, from the ncu capture summarised in
+# profiles/attn_kernel_480p_h8.md (8 heads, scaled to 40 by heads: traffic
+# grows with the (head, query block) rows); valid only for the kernel source it
+# was measured on and for that workload.
+ATTN_TRAFFIC = {"source_sha1": "00cdfb33a971abfc7050fa5922c9ddeb9b358280", "bytes_per_launch": 1595880960}
 
 
 def _env_int(name, default):
@@ -65,9 +67,13 @@ def load_peaks():
 
 
 def attn_source_sha1():
-    p = os.path.join(ROOT, "precision_attention_video_b200", "csrc", "ta_attn.cu")
-    with open(p, "rb") as f:
-        return hashlib.sha1(f.read()).hexdigest()
+    """Hash of the attention kernel's sources (the kernel and the headers it
+    inlines): a traffic figure holds only for the code it was measured on."""
+    h = hashlib.sha1()
+    for name in ("ta_attn.cu", "ta_attn_common.cuh", "ta_common.cuh"):
+        with open(os.path.join(ROOT, "precision_attention_video_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 class ClockSampler:
@@ -128,26 +134,30 @@ class ClockSampler:
 
 
 def algorithmic_attn_flops(cfg, counts: np.ndarray, lists: np.ndarray):
-    """FLOPs the tiered forward is defined to execute, by tier: 4*|q_i|*|k_j|*d
-    per full / residual / low tile and 4*|q_i|*d per skipped block, with real
-    (ragged) block sizes.  Returns (full, low, skip)."""
+    """FLOPs the tiered forward is defined to execute, by tier, with real
+    (ragged) block sizes: 4*|q_i|*|k_j|*d per full and low tile, three times
+    that per residual tile (A1 B1 + A1 B2 + A2 B1 for S and for P V), and
+    4*|q_i|*d per skipped block.  Returns (full, res, low, skip)."""
     N, d, bq, bk = cfg.N, cfg.d, cfg.block_q, cfg.block_k
     nqb, nkb = cfg.n_qb, cfg.n_kb
     qrows = np.array([min(bq, N - i * bq) for i in range(nqb)], dtype=np.float64)
     kcols = np.array([min(bk, N - j * bk) for j in range(nkb)], dtype=np.float64)
     BH = counts.shape[0]
     full_cols = np.zeros((BH, nqb))
+    res_cols = np.zeros((BH, nqb))
     low_cols = np.zeros((BH, nqb))
     n_skip = counts[..., 3].astype(np.float64)
     for bh in range(BH):
         for i in range(nqb):
             nf, nr, nl = (int(x) for x in counts[bh, i, :3])
-            full_cols[bh, i] = kcols[lists[bh, i, :nf + nr]].sum()
+            full_cols[bh, i] = kcols[lists[bh, i, :nf]].sum()
+            res_cols[bh, i] = kcols[lists[bh, i, nf:nf + nr]].sum()
             low_cols[bh, i] = kcols[lists[bh, i, nf + nr:nf + nr + nl]].sum()
     full = 4.0 * d * (full_cols * qrows[None, :]).sum()
+    res = 3.0 * 4.0 * d * (res_cols * qrows[None, :]).sum()
     low = 4.0 * d * (low_cols * qrows[None, :]).sum()
     skip = 4.0 * d * (n_skip * qrows[None, :]).sum()
-    return full, low, skip
+    return full, res, low, skip
 
 
 def workload(args, name=None):
@@ -233,7 +243,7 @@ def run_gpu_arm(args, rank, world, local_rank):
     counts = views["row_counts"].cpu().numpy()
     lists = views["row_lists"].cpu().numpy()
     tiers = views["tier_map"].cpu().numpy()
-    full_flops, low_flops, skip_flops = algorithmic_attn_flops(cfg, counts, lists)
+    full_flops, res_flops, low_flops, skip_flops = algorithmic_attn_flops(cfg, counts, lists)
 
     # timed region: K whole steps, events around each forward for the roofline
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -279,7 +289,8 @@ def run_gpu_arm(args, rank, world, local_rank):
 
     res = {
         "total_ms": total_ms, "plan_ms": plan_ms, "fwd_ms": fwd_ms, "e2e_ms": e2e_ms,
-        "clocks": clk.summary(), "full_flops": full_flops, "low_flops": low_flops,
+        "clocks": clk.summary(), "full_flops": full_flops, "res_flops": res_flops,
+        "low_flops": low_flops,
         "skip_flops": skip_flops,
         "tier_frac": {n: float((tiers == t).mean()) for n, t in
                       (("full", 3), ("res", 2), ("low", 1), ("skip", 0))},
@@ -397,16 +408,20 @@ def main():
         e2e_ms = r["e2e_ms"]
     peaks, peak_src = load_peaks()
     p_bf16 = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    # full tiles and skip chunks run on the bf16 pipe; NVFP4 low tiles on the
-    # FP4 pipe, whose peak is taken as 4x the measured bf16 one (nominal ratio).
-    # FP8 low tiles (other workloads) run on bf16 images, at the bf16 peak.
-    p_low = 4.0 * p_bf16 if cfg.low == 2 else p_bf16
-    executed = r["full_flops"] + r["low_flops"] + r["skip_flops"]
-    t_min = (r["full_flops"] + r["skip_flops"]) / (p_bf16 * 1e12) + r["low_flops"] / (p_low * 1e12)
+    # Full tiles and skip chunks run on the bf16 pipe; NVFP4 tiles (low and
+    # residual) on the FP4 pipe and native FP8 tiles (d = 128, 128 x 128) on
+    # the FP8 pipe, whose peaks are taken as 4x and 2x the measured bf16 one
+    # (the nominal ratios); FP8 tiles of other shapes run on bf16 images.
+    native_f8 = cfg.d == 128 and cfg.block_q == 128 and cfg.block_k == 128
+    p_fp4 = 4.0 * p_bf16
+    p_low = {1: (2.0 if native_f8 else 1.0) * p_bf16, 2: p_fp4, 3: p_fp4}.get(cfg.low, p_bf16)
+    executed = r["full_flops"] + r["res_flops"] + r["low_flops"] + r["skip_flops"]
+    t_min = ((r["full_flops"] + r["skip_flops"]) / (p_bf16 * 1e12) + r["res_flops"] / (p_fp4 * 1e12)
+             + r["low_flops"] / (p_low * 1e12))
     peak = executed / t_min / 1e12          # blended tensor peak of this launch's FLOP mix
     achieved = executed / (fwd_ms * 1e-3) / 1e12
     traffic = None
-    if ATTN_TRAFFIC["source_sha1"] == attn_source_sha1():
+    if ATTN_TRAFFIC["source_sha1"] == attn_source_sha1() and cfg.name == WORKLOAD and cfg.H == 40:
         traffic = ATTN_TRAFFIC["bytes_per_launch"]
 
     if rank == 0:
@@ -421,11 +436,11 @@ def main():
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": (f"blend of {peak_src} bf16_tflops_sustained "
-                                         f"{p_bf16:.1f} and nvfp4 = 4x that, weighted by "
-                                         "the launch's FLOPs per tier"),
+                                         f"{p_bf16:.1f}, nvfp4 = 4x and native fp8 = 2x "
+                                         "that, weighted by the launch's FLOPs per tier"),
                          "flops_per_launch": executed,
-                         "flops_by_tier": {"full": r["full_flops"], "low": r["low_flops"],
-                                           "skip": r["skip_flops"]}},
+                         "flops_by_tier": {"full": r["full_flops"], "res": r["res_flops"],
+                                           "low": r["low_flops"], "skip": r["skip_flops"]}},
             "e2e": {"value": world * dense / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                     "ms_per_step": e2e_ms},

@@ -1,0 +1,37 @@
+"""Host-side logic of the benchmark: the algorithmic FLOP count per tier that
+the roofline line divides by, checked against a hand count on a small plan."""
+
+import importlib.util
+import os
+
+import numpy as np
+
+from latent_gen import get_config
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_algorithmic_flops_by_tier():
+    bench = _bench()
+    # N = 300 tokens in 128 x 128 tiles: blocks of 128, 128 and 44 rows / keys
+    cfg = get_config("480p").with_(H=1, grid=(1, 3, 100), low=3, tau=(0.5, 0.7, 0.9))
+    assert cfg.N == 300 and cfg.n_qb == 3 and cfg.n_kb == 3
+    # one head; per query block: counts (full, res, low, skip) and list order
+    counts = np.array([[[1, 1, 1, 0], [2, 0, 0, 1], [1, 0, 1, 1]]], dtype=np.int32)
+    lists = np.array([[[0, 2, 1], [1, 2, 0], [2, 0, 1]]], dtype=np.int32)
+    full, res, low, skip = bench.algorithmic_attn_flops(cfg, counts, lists)
+    d = 128
+    q = [128, 128, 44]
+    k = [128, 128, 44]
+    want_full = 4 * d * (q[0] * k[0] + q[1] * (k[1] + k[2]) + q[2] * k[2])
+    want_res = 3 * 4 * d * (q[0] * k[2])
+    want_low = 4 * d * (q[0] * k[1] + q[2] * k[0])
+    want_skip = 4 * d * (q[1] * 1 + q[2] * 1)
+    assert (full, res, low, skip) == (want_full, want_res, want_low, want_skip)
