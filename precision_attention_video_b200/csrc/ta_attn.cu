@@ -15,15 +15,18 @@
 //               kbar_b / vbar_b into a "pseudo-key" tile, so a skip chunk costs
 //               one tile of MMA for up to BK skipped blocks and never touches
 //               their K / V;
-//   warp 4S+2   MMA issuer: S = Q K^T into a double-buffered TMEM accumulator
-//               and O += P V into a TMEM accumulator, one thread issuing
-//               tcgen05.mma: kind::f16 for full and skip tiles and for FP8
-//               tiles of the small shapes (bf16 images of the codes);
-//               kind::mxf4nvf4.block16 for NVFP4 tiles (ue4m3 scales copied to
-//               TMEM with tcgen05.cp; three MMAs per product on residual
+//   warp 4S+2   S issuer: S = Q K^T into a double-buffered TMEM accumulator,
+//               as soon as the softmax has read the buffer's previous S;
+//   warp 4S+3   PV issuer: O += P V into a TMEM accumulator.  One thread each
+//               issues tcgen05.mma: kind::f16 for full and skip tiles and for
+//               FP8 tiles of the small shapes (bf16 images of the codes);
+//               kind::mxf4nvf4.block16 for NVFP4 tiles (ue4m3 scales copied
+//               to TMEM with tcgen05.cp; three MMAs per product on residual
 //               tiles); kind::f8f6f4 for FP8 S and kind::mxf8f6f4 for FP8 PV
-//               (V's power-of-two tile scale as a UE8M0 block scale).
-//               Completion is signalled with tcgen05.commit on mbarriers;
+//               (V's power-of-two tile scale as a UE8M0 block scale).  Two
+//               threads, because one thread issues an N <= 128 MMA only every
+//               ~100 cycles.  Completion is signalled with tcgen05.commit on
+//               mbarriers;
 //   warps 0..4S-1 softmax (S = min(d, BK)/32 column parts): the S warps with
 //               equal w%4 share TMEM lanes 32(w%4).. (query rows) and split
 //               each row's columns into S parts of 32; they swap their part
@@ -33,9 +36,9 @@
 //               specialised for the tile's P format: P' = 2^o exp(s - m'),
 //               rounded as the tier demands (bf16; e4m3; NVFP4 per 16 keys,
 //               plus its residual), O rescaled in TMEM when m grew, and P'
-//               handed to the PV MMA: bf16 P' is stored into the TMEM columns
-//               of its own S buffer (the A operand of a TMEM x shared-memory
-//               MMA), NVFP4 / FP8 P' into one of two shared-memory buffers.
+//               handed to the PV MMA: bf16 P' is stored into TMEM columns of
+//               its own (the A operand of a TMEM x shared-memory MMA), NVFP4 /
+//               FP8 P' into one of two shared-memory buffers.
 //               The epilogue writes O = acc / l in bf16.
 //
 // All waits are bounded: a wait that runs out sets the CTA's abort flag and
@@ -58,8 +61,9 @@ struct Roles {
   static constexpr int kSoftmaxWarps = 4 * kSplit;
   static constexpr int kProducerKWarp = kSoftmaxWarps;      // Q and K tiles
   static constexpr int kProducerVWarp = kSoftmaxWarps + 1;  // V tiles
-  static constexpr int kMmaWarp = kSoftmaxWarps + 2;
-  static constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
+  static constexpr int kMmaWarp = kSoftmaxWarps + 2;        // S = Q K^T issuer
+  static constexpr int kPvWarp = kSoftmaxWarps + 3;         // O += P V issuer
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 4);
 };
 
 // Named barrier over `count` threads that also ANDs a predicate across them:
@@ -99,19 +103,21 @@ struct Smem {
   static constexpr int oV1 = oK1 + kKV;
   static constexpr int oP = oV1 + kKV;
   static constexpr int oBar = oP + kP;
-  static constexpr int kBars = 16;
+  static constexpr int kBars = 24;
   static constexpr int oMisc = oBar + kBars * 8;
   static constexpr int oXchg = oMisc + 64;           // float [2 slots][4 parts][128 rows]
   static constexpr int oScTab = oXchg + 2 * 4 * 128 * 4;  // float2 [128]: ue4m3 value, 1/value
   static constexpr int kTotal = oScTab + 128 * 8;
   static constexpr int kAlloc = kTotal;  // the base is checked for 1024-byte alignment
-  static constexpr uint32_t kTmemCols = (2 * BK + D) <= 256 ? 256u : 512u;
 };
 
+// mbarriers; pairs are indexed by the parity of the tile
+//   S   S of the tile is in TMEM (S issuer)      SC  the softmax has read that S
+//   P   the tile's P is written (softmax)        PD  the tile's PV is done (PV issuer)
 enum {
   BAR_Q = 0, BAR_K0 = 1, BAR_K1 = 2, BAR_V0 = 3, BAR_V1 = 4, BAR_KE0 = 5, BAR_KE1 = 6,
-  BAR_S0 = 7, BAR_S1 = 8, BAR_P = 9, BAR_PD0 = 10, BAR_PD1 = 11, BAR_DRAIN = 12,
-  BAR_VE0 = 13, BAR_VE1 = 14
+  BAR_S0 = 7, BAR_S1 = 8, BAR_P0 = 9, BAR_P1 = 10, BAR_PD0 = 11, BAR_PD1 = 12,
+  BAR_DRAIN_S = 13, BAR_DRAIN_PV = 14, BAR_VE0 = 15, BAR_VE1 = 16, BAR_SC0 = 17, BAR_SC1 = 18
 };
 
 // Formats of P' in the softmax's tile tail.
@@ -131,7 +137,7 @@ struct SoftmaxTail {
   AbortCtx ctx;
   int row_bar;
   unsigned char* sm;
-  uint32_t tS, tO;          // this lane's S buffer and O accumulator
+  uint32_t tP, tO;          // this lane's bf16 P columns and O accumulator
   int part, quarter, lane, r;
   const float2* sc_tab;     // ue4m3 code -> (value, 1 / value)
 };
@@ -139,14 +145,15 @@ struct SoftmaxTail {
 // Tail of one tile's softmax for one P format, in straight-line code:
 // P' = 2^o exp(s - m') and its part row sum, P' rounded as the tier demands,
 // O rescaled when the maximum grew (after the previous PV), and P' handed to
-// the PV MMA (bf16 in the S buffer's TMEM columns; NVFP4 / FP8 in a shared
-// memory buffer).  False when the CTA aborts.
+// the PV MMA (bf16 in the TMEM P columns, once the previous PV has read
+// them; NVFP4 / FP8 in a shared-memory buffer, once the PV two tiles back has
+// read it).  False when the CTA aborts; the warp then leaves at the row
+// group's next named barrier.
 template <int PK, int D, int BK, int LM>
 __device__ __forceinline__ bool softmax_tail(const SoftmaxTail q, float& psum) {
   using L = Smem<D, BK, LM>;
   constexpr int kSplit = Roles<D, BK>::kSplit;
   constexpr int HB = BK / kSplit, HD = D / kSplit;
-  constexpr int kBarThreads = 32 * kSplit;
   constexpr bool smem_p = (PK == PK_FP4 || PK == PK_RES || PK == PK_F8);
   const int s = q.t & 1;
   float* x = q.x;
@@ -192,19 +199,18 @@ __device__ __forceinline__ bool softmax_tail(const SoftmaxTail q, float& psum) {
     for (int c = 0; c < HB; c += 2) p[c / 2] = pack_bf16(x[c], x[c + 1]);
   }
 
-  // O may be rescaled only once the previous tile's PV is done; a shared
-  // memory P buffer may be rewritten once the PV two tiles back is done.  The
-  // warps sharing these rows see the same maxima, so they agree on `rescale`
-  // and on `reuse` and wait (and leave on abort) together.
+  // O may be rescaled, and the TMEM P columns rewritten, only once the
+  // previous tile's PV is done; a shared-memory P buffer may be rewritten
+  // once the PV two tiles back is done.  Each warp decides and waits for
+  // itself (it rescales and writes only its own columns).
   const bool rescale = (q.t > 0) && __any_sync(0xffffffffu, q.alpha != 1.0f);
+  const bool prev = (q.t > 0) && (rescale || !smem_p);
   const bool reuse = smem_p && q.t >= 2;
-  if (rescale || reuse) {
+  if (prev || reuse) {
     bool ok2 = true;
     if (reuse) ok2 = mbar_wait(&q.bars[BAR_PD0 + s], ((q.t >> 1) - 1) & 1, q.ctx, 7);
-    if (rescale && ok2) ok2 = mbar_wait(&q.bars[BAR_PD0 + (s ^ 1)], ((q.t - 1) >> 1) & 1, q.ctx, 9);
-    ok2 = __all_sync(0xffffffffu, ok2);
-    ok2 = bar_and(q.row_bar, kBarThreads, ok2);
-    if (!ok2) return false;
+    if (prev && ok2) ok2 = mbar_wait(&q.bars[BAR_PD0 + (s ^ 1)], ((q.t - 1) >> 1) & 1, q.ctx, 9);
+    if (!__all_sync(0xffffffffu, ok2)) return false;
   }
   if (rescale) {
     tc_fence_after();
@@ -240,15 +246,14 @@ __device__ __forceinline__ bool softmax_tail(const SoftmaxTail q, float& psum) {
           make_uint4(p[h * 4 + 0], p[h * 4 + 1], p[h * 4 + 2], p[h * 4 + 3]);
     }
   } else {
-    // bf16 P' of this part into the S buffer's first BK/2 columns (every
-    // part has loaded its S columns before the row barrier)
+    // bf16 P' of this part into the TMEM P columns
 #pragma unroll
-    for (int h = 0; h < HB / 2; h += 16) tmem_st16(q.tS + q.part * (HB / 2) + h, p + h);
+    for (int h = 0; h < HB / 2; h += 16) tmem_st16(q.tP + q.part * (HB / 2) + h, p + h);
   }
   if constexpr (smem_p) fence_proxy_async_smem();
   tmem_wait_st();
   tc_fence_before();
-  mbar_arrive(&q.bars[BAR_P]);
+  mbar_arrive(&q.bars[BAR_P0 + s]);
   return true;
 }
 
@@ -261,15 +266,14 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
                 const __grid_constant__ CUtensorMap tmRK, const __grid_constant__ CUtensorMap tmRV) {
   using L = Smem<D, BK, LM>;
   constexpr bool FP4 = L::FP4, RES = L::RES, F8 = L::F8;
-  using TS = TmemSf<D, BK, RES>;
+  using TS = TmemMap<D, BK, LM>;
   using RL = Roles<D, BK>;
   constexpr int kSplit = RL::kSplit, kSoftmaxWarps = RL::kSoftmaxWarps;
   constexpr int kProducerKWarp = RL::kProducerKWarp, kProducerVWarp = RL::kProducerVWarp;
-  constexpr int kMmaWarp = RL::kMmaWarp;
+  constexpr int kMmaWarp = RL::kMmaWarp, kPvWarp = RL::kPvWarp;
   static_assert(!(FP4 || F8) || (D == 128 && BK == 128),
                 "native NVFP4 / FP8 tiles need d = 128, 128-key tiles");
-  constexpr uint32_t kTmemCols = (FP4 || F8) ? 512u : L::kTmemCols;
-  static_assert(!FP4 || TS::kEnd <= 512u, "TMEM columns");
+  constexpr uint32_t kTmemCols = TS::kCols;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw;
   if (smem_u32(sm) & 1023u) {
@@ -313,10 +317,14 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
     mbar_init(&bars[BAR_VE1], 1);
     mbar_init(&bars[BAR_S0], 1);
     mbar_init(&bars[BAR_S1], 1);
-    mbar_init(&bars[BAR_P], kSplit * a.bq);  // every column part of every live row
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[BAR_P0 + i], kSplit * a.bq);   // every column part of every live row
+      mbar_init(&bars[BAR_SC0 + i], kSplit * a.bq);
+    }
     mbar_init(&bars[BAR_PD0], 1);
     mbar_init(&bars[BAR_PD1], 1);
-    mbar_init(&bars[BAR_DRAIN], 1);
+    mbar_init(&bars[BAR_DRAIN_S], 1);
+    mbar_init(&bars[BAR_DRAIN_PV], 1);
     fence_mbar_init();
   }
   if (F8 && threadIdx.x < 128) {
@@ -340,7 +348,8 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         *reinterpret_cast<uint4*>(sm + L::oQ + off) = make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(sm + L::oDQ + off) = make_uint4(0, 0, 0, 0);
       }
-      // (rows >= bq of S, and so of the P aliased onto it, are exact zeros)
+      // (rows >= bq of S are exact zeros; rows >= bq of P and O are never
+      // read back: a product's row depends on its own row of P only)
       fence_proxy_async_smem();
     }
   }
@@ -352,7 +361,8 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS0 = tmem, tS1 = tmem + BK, tO = tmem + 2 * BK;
+  const uint32_t tS0 = tmem + TS::kS0, tS1 = tmem + TS::kS1, tO = tmem + TS::kO;
+  const uint32_t tP = tmem + TS::kP;
 
   bool aborted = false;
 
@@ -524,77 +534,86 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
       if (isK) mbar_wait_drain(&bars[BAR_Q], 0);
     }
   } else if (warp == kMmaWarp) {
-    // ===================== MMA issuer =====================
+    // ===================== S issuer: S = Q K^T =====================
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, BK, false);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, D, true);
       const uint32_t sQ = smem_u32(sm + L::oQ), sDQ = smem_u32(sm + L::oDQ);
-      const uint32_t sP = smem_u32(sm + L::oP);  // NVFP4 P buffers
-      auto issue_s = [&](int t) -> bool {
-        const int s = t & 1;
-        if (!mbar_wait(&bars[BAR_K0 + s], (t >> 1) & 1, ctx, 2)) return false;
-        tc_fence_after();
-        int kind, first;
-        tile_of<BK>(rp, t, kind, first);
-        const uint32_t aq = (kind == KIND_LOW || kind == KIND_RES) ? sDQ : sQ;
-        const uint32_t sk = smem_u32(sm + (s ? L::oK1 : L::oK0));
-        if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
-          // NVFP4: Q1 K1 (+ Q1 K2 + Q2 K1 on residual tiles), block scales in TMEM
-          const int ncopy = (RES && kind == KIND_RES) ? 2 : 1;
-          for (int c = 0; c < ncopy; ++c) {
-            const uint32_t sfb = tmem + TS::sfbK(s, c);
-            tc_cp_sf(sfb, smem_desc_rows16(sk + c * L::kPfp4 + kFp4Sf));
-            tc_cp_sf(sfb + 4, smem_desc_rows16(sk + c * L::kPfp4 + kFp4Sf + 512));
-          }
-          const uint32_t d = s ? tS1 : tS0;
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            mma_nvfp4_ss(d, smem_desc_sw64(aq + kk * 32), smem_desc_sw64(sk + kk * 32),
-                         idesc_nvfp4(128, BK), tmem + TS::sfaQ(0) + kk * 4,
-                         tmem + TS::sfbK(s, 0) + kk * 4, kk > 0 ? 1u : 0u);
-            if (RES && kind == KIND_RES) {
-              mma_nvfp4_ss(d, smem_desc_sw64(aq + kk * 32), smem_desc_sw64(sk + L::kPfp4 + kk * 32),
-                           idesc_nvfp4(128, BK), tmem + TS::sfaQ(0) + kk * 4,
-                           tmem + TS::sfbK(s, 1) + kk * 4, 1u);
-              mma_nvfp4_ss(d, smem_desc_sw64(aq + L::kPfp4 + kk * 32), smem_desc_sw64(sk + kk * 32),
-                           idesc_nvfp4(128, BK), tmem + TS::sfaQ(1) + kk * 4,
-                           tmem + TS::sfbK(s, 0) + kk * 4, 1u);
-            }
-          }
-        } else if (F8 && kind == KIND_LOW) {
-          // FP8 codes: 4 MMAs of K = 32 over the 128-byte rows (scales applied in softmax)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f8_ss(s ? tS1 : tS0, smem_desc_sw128(aq + kk * 32, 16, 1024),
-                      smem_desc_sw128(sk + kk * 32, 16, 1024), idesc_f8(128, BK), kk > 0 ? 1u : 0u);
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(aq + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(sk + (kk >> 2) * (BK * 128) + (kk & 3) * 32, 16, 1024);
-            mma_f16_ss(s ? tS1 : tS0, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-        }
-        tc_commit(&bars[BAR_S0 + s]);
-        tc_commit(&bars[BAR_KE0 + s]);   // the K stage is free once S is done
-        return true;
-      };
       bool ok = mbar_wait(&bars[BAR_Q], 0, ctx, 3);
       if (ok) {
         tc_fence_after();
-        if (F8) tc_cp_sf(tmem + TS::sfaP8(), smem_desc_rows16(sP + 2 * L::kF8));
         if (FP4) {
           for (int c = 0; c < nq; ++c) {
             tc_cp_sf(tmem + TS::sfaQ(c), smem_desc_rows16(sDQ + c * L::kPfp4 + kFp4Sf));
             tc_cp_sf(tmem + TS::sfaQ(c) + 4, smem_desc_rows16(sDQ + c * L::kPfp4 + kFp4Sf + 512));
           }
         }
-        ok = issue_s(0);
       }
       for (int t = 0; ok && t < rp.T; ++t) {
         const int s = t & 1;
-        if (t + 1 < rp.T && !issue_s(t + 1)) { ok = false; break; }
-        if (!mbar_wait(&bars[BAR_P], t & 1, ctx, 4)) { ok = false; break; }
+        // the S buffer is free once the softmax has read S of tile t-2
+        if (t >= 2 && !mbar_wait(&bars[BAR_SC0 + s], ((t - 2) >> 1) & 1, ctx, 10)) { ok = false; break; }
+        if (!mbar_wait(&bars[BAR_K0 + s], (t >> 1) & 1, ctx, 2)) { ok = false; break; }
+        tc_fence_after();
+        int kind, first;
+        tile_of<BK>(rp, t, kind, first);
+        const uint32_t aq = (kind == KIND_LOW || kind == KIND_RES) ? sDQ : sQ;
+        const uint32_t sk = smem_u32(sm + (s ? L::oK1 : L::oK0));
+        const uint32_t d = s ? tS1 : tS0;
+        if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
+          // NVFP4: Q1 K1 (+ Q1 K2 + Q2 K1 on residual tiles), block scales in TMEM
+          const int ncopy = (RES && kind == KIND_RES) ? 2 : 1;
+          for (int c = 0; c < ncopy; ++c) {
+            const uint32_t sfb = tmem + TS::sfbK(c);
+            tc_cp_sf(sfb, smem_desc_rows16(sk + c * L::kPfp4 + kFp4Sf));
+            tc_cp_sf(sfb + 4, smem_desc_rows16(sk + c * L::kPfp4 + kFp4Sf + 512));
+          }
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            mma_nvfp4_ss(d, smem_desc_sw64(aq + kk * 32), smem_desc_sw64(sk + kk * 32),
+                         idesc_nvfp4(128, BK), tmem + TS::sfaQ(0) + kk * 4,
+                         tmem + TS::sfbK(0) + kk * 4, kk > 0 ? 1u : 0u);
+            if (RES && kind == KIND_RES) {
+              mma_nvfp4_ss(d, smem_desc_sw64(aq + kk * 32), smem_desc_sw64(sk + L::kPfp4 + kk * 32),
+                           idesc_nvfp4(128, BK), tmem + TS::sfaQ(0) + kk * 4,
+                           tmem + TS::sfbK(1) + kk * 4, 1u);
+              mma_nvfp4_ss(d, smem_desc_sw64(aq + L::kPfp4 + kk * 32), smem_desc_sw64(sk + kk * 32),
+                           idesc_nvfp4(128, BK), tmem + TS::sfaQ(1) + kk * 4,
+                           tmem + TS::sfbK(0) + kk * 4, 1u);
+            }
+          }
+        } else if (F8 && kind == KIND_LOW) {
+          // FP8 codes: 4 MMAs of K = 32 over the 128-byte rows (scales applied in softmax)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f8_ss(d, smem_desc_sw128(aq + kk * 32, 16, 1024),
+                      smem_desc_sw128(sk + kk * 32, 16, 1024), idesc_f8(128, BK), kk > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(aq + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sk + (kk >> 2) * (BK * 128) + (kk & 3) * 32, 16, 1024);
+            mma_f16_ss(d, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+        }
+        tc_commit(&bars[BAR_S0 + s]);
+        tc_commit(&bars[BAR_KE0 + s]);   // the K stage is free once S is done
+      }
+      if (!ok) {
+        aborted = true;
+        tc_commit(&bars[BAR_DRAIN_S]);
+        mbar_wait_drain(&bars[BAR_DRAIN_S], 0);
+      }
+    }
+  } else if (warp == kPvWarp) {
+    // ===================== PV issuer: O += P V =====================
+    if (lane == 0) {
+      constexpr uint32_t idesc_pv = idesc_bf16(128, D, true);
+      const uint32_t sP = smem_u32(sm + L::oP);  // NVFP4 / FP8 P buffers
+      if (F8) tc_cp_sf(tmem + TS::sfaP8(), smem_desc_rows16(sP + 2 * L::kF8));
+      bool ok = true;
+      for (int t = 0; t < rp.T; ++t) {
+        const int s = t & 1;
+        if (!mbar_wait(&bars[BAR_P0 + s], (t >> 1) & 1, ctx, 4)) { ok = false; break; }
         if (!mbar_wait(&bars[BAR_V0 + s], (t >> 1) & 1, ctx, 5)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sv = smem_u32(sm + (s ? L::oV1 : L::oV0));
@@ -605,7 +624,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           const int ncopy = (RES && kind_t == KIND_RES) ? 2 : 1;
           const uint32_t pb = sP + s * L::NC * L::kPfp4;
           for (int c = 0; c < ncopy; ++c) {
-            const uint32_t sfa = tmem + TS::sfaP(s, c), sfb = tmem + TS::sfbV(s, c);
+            const uint32_t sfa = tmem + TS::sfaP(c), sfb = tmem + TS::sfbV(c);
             tc_cp_sf(sfa, smem_desc_rows16(pb + c * L::kPfp4 + kFp4Sf));
             tc_cp_sf(sfa + 4, smem_desc_rows16(pb + c * L::kPfp4 + kFp4Sf + 512));
             tc_cp_sf(sfb, smem_desc_rows16(sv + c * L::kPfp4 + kFp4Sf));
@@ -614,34 +633,33 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
             mma_nvfp4_ss(tO, smem_desc_sw64(pb + kk * 32), smem_desc_sw64(sv + kk * 32),
-                         idesc_nvfp4(128, D), tmem + TS::sfaP(s, 0) + kk * 4,
-                         tmem + TS::sfbV(s, 0) + kk * 4, (t > 0 || kk > 0) ? 1u : 0u);
+                         idesc_nvfp4(128, D), tmem + TS::sfaP(0) + kk * 4,
+                         tmem + TS::sfbV(0) + kk * 4, (t > 0 || kk > 0) ? 1u : 0u);
             if (RES && kind_t == KIND_RES) {
               mma_nvfp4_ss(tO, smem_desc_sw64(pb + kk * 32), smem_desc_sw64(sv + L::kPfp4 + kk * 32),
-                           idesc_nvfp4(128, D), tmem + TS::sfaP(s, 0) + kk * 4,
-                           tmem + TS::sfbV(s, 1) + kk * 4, 1u);
+                           idesc_nvfp4(128, D), tmem + TS::sfaP(0) + kk * 4,
+                           tmem + TS::sfbV(1) + kk * 4, 1u);
               mma_nvfp4_ss(tO, smem_desc_sw64(pb + L::kPfp4 + kk * 32), smem_desc_sw64(sv + kk * 32),
-                           idesc_nvfp4(128, D), tmem + TS::sfaP(s, 1) + kk * 4,
-                           tmem + TS::sfbV(s, 0) + kk * 4, 1u);
+                           idesc_nvfp4(128, D), tmem + TS::sfaP(1) + kk * 4,
+                           tmem + TS::sfbV(0) + kk * 4, 1u);
             }
           }
         } else if (F8 && kind_t == KIND_LOW) {
           // FP8 P codes (scale 2^0) x FP8 V codes (MN-major) with V's power-of-two
           // tile scale as the UE8M0 block scale
           const uint32_t pb = sP + s * L::kF8;
-          tc_cp_sf(tmem + TS::sfbV8(s), smem_desc_rows16(sv + L::kF8));
+          tc_cp_sf(tmem + TS::sfbV8(), smem_desc_rows16(sv + L::kF8));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_mxf8_ss(tO, smem_desc_sw128(pb + kk * 32, 16, 1024),
                         smem_desc_sw128(sv + kk * 32 * 128, 16, 1024), idesc_mxf8_bmn(128, D),
-                        tmem + TS::sfaP8(), tmem + TS::sfbV8(s), (t > 0 || kk > 0) ? 1u : 0u);
+                        tmem + TS::sfaP8(), tmem + TS::sfbV8(), (t > 0 || kk > 0) ? 1u : 0u);
         } else {
-          // A = bf16 P' in the TMEM columns of this tile's S buffer
-          const uint32_t pa = s ? tS1 : tS0;
+          // A = bf16 P' in the TMEM P columns
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t bd = smem_desc_sw128(sv + kk * 16 * 128, BK * 128, 1024);
-            mma_f16_ts(tO, pa + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+            mma_f16_ts(tO, tP + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
           }
         }
         tc_commit(&bars[BAR_PD0 + s]);
@@ -649,8 +667,8 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
       }
       if (!ok) {
         aborted = true;
-        tc_commit(&bars[BAR_DRAIN]);
-        mbar_wait_drain(&bars[BAR_DRAIN], 0);
+        tc_commit(&bars[BAR_DRAIN_PV]);
+        mbar_wait_drain(&bars[BAR_DRAIN_PV], 0);
       }
     }
   } else if (warp < kSoftmaxWarps && (warp & 3) * 32 < a.bq) {
@@ -669,9 +687,10 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
     // FP8 tiles hold the dot products of the codes: their true S is S * s_q * s_k
     const float s_q8 = F8 ? a.q_s8[(int64_t)bh * a.nQb + qb] : 1.0f;
     float m = -INFINITY, l = 0.0f;           // running max (S units), part row sum
+    bool tail_ok = true;   // false once a wait in a tile's tail failed (abort)
     for (int t = 0; t < rp.T; ++t) {
       const int s = t & 1;
-      bool ok = mbar_wait(&bars[BAR_S0 + s], (t >> 1) & 1, ctx, 6);
+      bool ok = tail_ok && mbar_wait(&bars[BAR_S0 + s], (t >> 1) & 1, ctx, 6);
       ok = __all_sync(0xffffffffu, ok);
       int kind, first;
       tile_of<BK>(rp, t, kind, first);
@@ -695,6 +714,9 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) x[c0 + c] = __uint_as_float(raw[c]);
         }
+        // this part of S is in registers: the S buffer may take tile t+2
+        tc_fence_before();
+        mbar_arrive(&bars[BAR_SC0 + s]);
         if (nv < HB) {
 #pragma unroll
           for (int c = 0; c < HB; ++c)
@@ -728,7 +750,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
       q.ctx = ctx;
       q.row_bar = row_bar;
       q.sm = sm;
-      q.tS = (s ? tS1 : tS0) + lane_off;
+      q.tP = tP + lane_off;
       q.tO = tO + lane_off;
       q.part = part;
       q.quarter = quarter;
@@ -753,12 +775,14 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           ok3 = softmax_tail<PK_IMG_F8, D, BK, LM>(q, psum);
         }
       }
-      if (!ok3) { aborted = true; break; }
+      // a failed wait leaves the loop at the next row barrier, with the other
+      // warps of these rows
+      if (!ok3) tail_ok = false;
       l = l * alpha + psum;
       m = m_new;
     }
     if (!aborted) {
-      bool ok = mbar_wait(&bars[BAR_PD0 + ((rp.T - 1) & 1)], ((rp.T - 1) >> 1) & 1, ctx, 8);
+      bool ok = tail_ok && mbar_wait(&bars[BAR_PD0 + ((rp.T - 1) & 1)], ((rp.T - 1) >> 1) & 1, ctx, 8);
       ok = __all_sync(0xffffffffu, ok);
       // row sums through the exchange slot the last tile did not use (its
       // last readers passed the last tile's row barrier)

@@ -72,21 +72,31 @@ __device__ __forceinline__ __half2 e2m1x2_to_half2(uint32_t codes) {
 // Low-tier execution mode of a kernel instance.
 enum LowMode { LM_IMAGE = 0, LM_NVFP4 = 1, LM_NVFP4_RES = 2, LM_FP8 = 3 };
 
-// TMEM columns of the NVFP4 scale factors (4 columns per 64-element K chunk,
-// 2 chunks per operand), after S0, S1 and O.
-template <int D, int BK, bool RES>
-struct TmemSf {
-  // FP8 tiles: UE8M0 scale factors of P (constant 2^0) and of V (per stage)
-  static constexpr __device__ uint32_t sfaP8() { return 2 * BK + D; }
-  static constexpr __device__ uint32_t sfbV8(int s) { return 2 * BK + D + 4 + 4 * s; }
-  static constexpr uint32_t NC = RES ? 2 : 1;   // copies (first + residual)
-  static constexpr uint32_t kBase = 2 * BK + D;
-  // query copy c; K copy c of stage s; V copy c of stage s; P copy c of buffer b
-  static constexpr __device__ uint32_t sfaQ(int c) { return kBase + 8 * c; }
-  static constexpr __device__ uint32_t sfbK(int s, int c) { return kBase + 8 * NC + 8 * (s * NC + c); }
-  static constexpr __device__ uint32_t sfbV(int s, int c) { return kBase + 24 * NC + 8 * (s * NC + c); }
-  static constexpr __device__ uint32_t sfaP(int b, int c) { return kBase + 40 * NC + 8 * (b * NC + c); }
-  static constexpr uint32_t kEnd = kBase + 56 * NC;  // <= 512 (496 with residual copies)
+// TMEM columns of one CTA: S of even and of odd tiles, the O accumulator, the
+// block scales of the narrow MMAs, and bf16 P (the A operand of the TMEM x
+// shared-memory PV product).  Block scales (4 columns per 64-element K chunk,
+// 2 chunks per operand) have one slot per operand: the thread that issues the
+// MMAs reading a slot also refills it, and its tcgen05 operations run in issue
+// order.
+template <int D, int BK, int LM>
+struct TmemMap {
+  static constexpr bool FP4 = (LM == LM_NVFP4 || LM == LM_NVFP4_RES);
+  static constexpr bool F8 = (LM == LM_FP8);
+  static constexpr uint32_t NC = (LM == LM_NVFP4_RES) ? 2 : 1;   // NVFP4 copies
+  static constexpr uint32_t kS0 = 0, kS1 = BK, kO = 2 * BK, kSf = 2 * BK + D;
+  // NVFP4: query copy c, key copy c, V copy c, P copy c
+  static constexpr __device__ uint32_t sfaQ(int c) { return kSf + 8 * c; }
+  static constexpr __device__ uint32_t sfbK(int c) { return kSf + 8 * NC + 8 * c; }
+  static constexpr __device__ uint32_t sfbV(int c) { return kSf + 16 * NC + 8 * c; }
+  static constexpr __device__ uint32_t sfaP(int c) { return kSf + 24 * NC + 8 * c; }
+  // FP8: UE8M0 scale factors of P (constant 2^0) and of V
+  static constexpr __device__ uint32_t sfaP8() { return kSf; }
+  static constexpr __device__ uint32_t sfbV8() { return kSf + 4; }
+  static constexpr uint32_t kSfEnd = FP4 ? kSf + 32 * NC : (F8 ? kSf + 8 : kSf);
+  static constexpr uint32_t kP = kSfEnd;            // bf16 P: BK/2 columns
+  static constexpr uint32_t kEnd = kP + BK / 2;
+  static constexpr uint32_t kCols = kEnd <= 256 ? 256u : 512u;
+  static_assert(kEnd <= 512, "TMEM columns");
 };
 
 // NVFP4 tiles in shared memory: codes [rows][64 B] with 64-byte swizzle, then
