@@ -60,6 +60,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of phase `parity` of `bar` (no suspension).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Shared abort state of one CTA: the first wait that runs out sets `abort`
 // and records the error in the global status word; every other wait of the
 // CTA sees `abort` and returns false, so all roles leave their loops.
@@ -82,6 +95,7 @@ static __device__ __noinline__ void report_timeout(AbortCtx ctx, int site) {
 // budget ran out (then the abort is raised here).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, AbortCtx ctx,
                                           int site) {
+  if (mbar_test(bar, parity)) return true;   // already complete: no suspension
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
