@@ -173,3 +173,49 @@ def test_skip_only_rows(cuda_ok):
     for h in range(cfg.H):
         rt, _, Oref = oracle_head(cfg, Q, K, V, 0, h, tau=(0.0, 0.0))
         assert_out_close(to64(O[0, h]), Oref, f"skip-only head {h}")
+
+
+def _forward_parity(cfg, Q, K, V, what, need_tiers=()):
+    _, views, O, st = run_gpu(cfg, Q, K, V)
+    assert st == 0
+    _plan_parity(cfg, Q, K, V, views, [(0, h) for h in range(cfg.H)])
+    t = views["tier_map"].numpy()
+    for code in need_tiers:
+        assert (t == code).any(), f"{what}: no tile of tier {code}"
+    for h in range(cfg.H):
+        rt, qt, Oref = oracle_head(cfg, Q, K, V, 0, h)
+        _, rows = compare_tiers(views["tier_map"][h].numpy(), rt)
+        for i in rows:
+            Oref[i * cfg.block_q:(i + 1) * cfg.block_q] = np.nan
+        assert_out_close(to64(O[0, h]), Oref, f"{what} head {h}")
+
+
+def test_forward_parity_d128_query_blocks_of_64(cuda_ok):
+    # d = 128 with 64-row query blocks and 128-key tiles: the FP8 tiles run on
+    # bf16 images, and the TMEM lanes of rows 64..127 carry no query rows
+    cfg, Q, K, V = inputs("sweep70", grid=(3, 10, 21), H=2, block_q=64)
+    _forward_parity(cfg, Q, K, V, "d128 bq64", need_tiers=(1, 3))
+
+
+def test_forward_parity_d128_key_blocks_of_64(cuda_ok):
+    # d = 128 with 128-row query blocks and 64-key tiles (two column parts of S)
+    cfg, Q, K, V = inputs("sweep70", grid=(3, 10, 21), H=2, block_k=64)
+    _forward_parity(cfg, Q, K, V, "d128 bk64", need_tiers=(1, 3))
+
+
+def test_forward_parity_no_low_tier(cuda_ok):
+    # one threshold: full and skipped tiles only (d = 128, 128 x 128 tiles)
+    cfg, Q, K, V = inputs("sweep70", grid=(3, 10, 21), H=2, low=0, tau=(0.7,))
+    _forward_parity(cfg, Q, K, V, "no low tier", need_tiers=(0, 3))
+
+
+def test_all_full_d128_matches_sdpa(cuda_ok):
+    # every tile full at d = 128: the bf16 path against torch's own attention
+    cfg, Q, K, V = inputs("480p", grid=(3, 10, 21), H=3)
+    _, views, O, st = run_gpu(cfg, Q, K, V, tau=(2.0, 2.0))
+    assert st == 0
+    assert (views["tier_map"].numpy() == 3).all()
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q.cuda().float(), K.cuda().float(), V.cuda().float()).cpu()
+    rel = (O.float() - ref).norm() / ref.norm()
+    assert rel < 1e-2
