@@ -150,9 +150,24 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q_dev, const void*
 
 /* Whole layer from host memory: copies Q, K, V (host, [B,H,N,d] with the
  * strides of `p`) into the caller's device buffers, plans, runs the forward and
- * copies O back to O_host, all enqueued on `stream` (one cudaMemcpyAsync per
- * tensor).  Does not synchronise: the caller synchronises `stream` before
- * reading O_host. */
+ * copies O back to O_host.  Host buffers should be pinned for the copies to
+ * overlap anything.
+ *  - Packed layout (stride_n = d, stride_h = N*d, stride_b = H*N*d) with more
+ *    than one (b, h) slice: the layer runs in up to 8 chunks of consecutive
+ *    slices (each head is independent, so O is bit for bit that of one plan +
+ *    forward).  The copies in of chunk c+1 and out of chunk c-1 overlap the
+ *    kernels of chunk c: copies in are enqueued on one library-owned stream,
+ *    copies out on another, the kernels on `stream`, ordered by events.  The
+ *    copy streams and events are created on first use, once per device, and
+ *    kept for the life of the process (no device memory is allocated).  Work
+ *    enqueued on `stream` before the call is complete before the first copy
+ *    in; `stream` waits for the last copy out.  Calls from several host
+ *    threads are serialised while they enqueue.
+ *  - Otherwise everything is enqueued on `stream`, one cudaMemcpyAsync per
+ *    tensor.
+ * Does not synchronise: the caller synchronises `stream` before reading
+ * O_host.  Errors as tiered_attn_plan / tiered_attn_forward; TA_ERR_CUDA when a
+ * copy, stream or event call fails. */
 ta_status tiered_attn_layer_from_host(const ta_params* p, const void* Q_host, const void* K_host,
                                       const void* V_host, void* O_host, void* Q_dev, void* K_dev,
                                       void* V_dev, void* O_dev, void* ws_dev, size_t ws_bytes,

@@ -1,6 +1,8 @@
 // ta_api.cu -- the C ABI of libtiered_attn.so: argument validation, the
 // workspace layout, TMA descriptors and the kernel launches.  The library
-// allocates no memory; every buffer, the workspace included, is the caller's.
+// allocates no device memory; every buffer, the workspace included, is the
+// caller's (tiered_attn_layer_from_host keeps two copy streams and a few
+// events per device).
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -14,6 +16,18 @@ constexpr size_t kAlign = 256;
 constexpr size_t kAbsent = ~static_cast<size_t>(0);  // array not in this layout
 
 inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+// Streams and events of tiered_attn_layer_from_host, created once per device
+// on first use and kept for the life of the process.
+constexpr int kMaxDevices = 64;
+constexpr int kChunks = 8;   // chunks of (b, h) slices a layer is split into
+struct CopyStreams {
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t ev[2 + 2 * kChunks] = {};
+};
+CopyStreams g_copy[kMaxDevices];
+std::mutex g_copy_mu;
 
 struct Shape {
   int64_t BH, N, d, nQb, nKb, Np;
@@ -314,8 +328,12 @@ ta_status tiered_attn_plan_views(const ta_params* p, void* ws, ta_plan_views* ou
   return TA_OK;
 }
 
-ta_status tiered_attn_prep(const ta_params* p, const void* Q, const void* K, const void* V,
-                           void* ws, size_t ws_bytes, void* stream) {
+namespace {
+
+// Pool and quantise; the status word is cleared first unless a caller that
+// runs several plans on one workspace keeps the first error.
+ta_status prep_impl(const ta_params* p, const void* Q, const void* K, const void* V, void* ws,
+                    size_t ws_bytes, void* stream, bool clear_status) {
   ta_status st = validate(p);
   if (st != TA_OK) return st;
   if ((st = check_tensor(Q)) || (st = check_tensor(K)) || (st = check_tensor(V))) return st;
@@ -323,8 +341,16 @@ ta_status tiered_attn_prep(const ta_params* p, const void* Q, const void* K, con
   ta::PlanArgs a;
   fill_plan_args(p, Q, K, V, ws, a);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(a.status, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return TA_ERR_CUDA;
+  if (clear_status && cudaMemsetAsync(a.status, 0, 4 * sizeof(int32_t), s) != cudaSuccess)
+    return TA_ERR_CUDA;
   return ta::launch_prep(a, s) == cudaSuccess ? TA_OK : TA_ERR_CUDA;
+}
+
+}  // namespace
+
+ta_status tiered_attn_prep(const ta_params* p, const void* Q, const void* K, const void* V,
+                           void* ws, size_t ws_bytes, void* stream) {
+  return prep_impl(p, Q, K, V, ws, ws_bytes, stream, true);
 }
 
 ta_status tiered_attn_route(const ta_params* p, void* ws, size_t ws_bytes, void* stream) {
@@ -449,18 +475,92 @@ ta_status tiered_attn_layer_from_host(const ta_params* p, const void* Qh, const 
       (st = check_tensor(Od)))
     return st;
   if ((st = check_ws(p, ws, ws_bytes)) != TA_OK) return st;
-  // extent of one tensor in elements, from its strides
-  const int64_t span = (int64_t)(p->B - 1) * p->stride_b + (int64_t)(p->H - 1) * p->stride_h +
-                       (int64_t)(p->N - 1) * p->stride_n + p->d;
-  const size_t bytes = (size_t)span * 2;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(Qd, Qh, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(Kd, Kh, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(Vd, Vh, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+  const int64_t head = (int64_t)p->N * p->d;   // elements of one (b, h) slice
+  const bool packed = p->stride_n == p->d && p->stride_h == head && p->stride_b == (int64_t)p->H * head;
+  const int64_t BH = (int64_t)p->B * p->H;
+  if (!packed || BH < 2) {
+    // one chunk, all on the caller's stream
+    const int64_t span = (int64_t)(p->B - 1) * p->stride_b + (int64_t)(p->H - 1) * p->stride_h +
+                         (int64_t)(p->N - 1) * p->stride_n + p->d;
+    const size_t bytes = (size_t)span * 2;
+    if (cudaMemcpyAsync(Qd, Qh, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(Kd, Kh, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(Vd, Vh, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return TA_ERR_CUDA;
+    if ((st = tiered_attn_plan(p, Qd, Kd, Vd, ws, ws_bytes, stream)) != TA_OK) return st;
+    if ((st = tiered_attn_forward(p, Qd, Kd, Vd, ws, ws_bytes, Od, stream)) != TA_OK) return st;
+    if (cudaMemcpyAsync(Oh, Od, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return TA_ERR_CUDA;
+    return TA_OK;
+  }
+
+  // Packed heads: the layer runs in chunks of consecutive (b, h) slices (every
+  // head is independent), so that the copy of chunk c+1 in, the attention of
+  // chunk c and the copy of chunk c-1 out overlap.  Copies in go on one
+  // library stream, copies out on another, the kernels on the caller's
+  // stream; events order them, and the caller's stream waits for the last
+  // copy out.
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TA_ERR_CUDA;
+  std::lock_guard<std::mutex> guard(g_copy_mu);
+  CopyStreams& cs = g_copy[dev];
+  if (!cs.ready) {
+    if (cudaStreamCreateWithFlags(&cs.in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&cs.out, cudaStreamNonBlocking) != cudaSuccess)
+      return TA_ERR_CUDA;
+    for (auto& e : cs.ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return TA_ERR_CUDA;
+    cs.ready = true;
+  }
+  const int nch = (int)(BH < kChunks ? BH : kChunks);
+  cudaEvent_t ev_entry = cs.ev[0], ev_done = cs.ev[1];
+  cudaEvent_t* ev_in = cs.ev + 2;
+  cudaEvent_t* ev_out = cs.ev + 2 + kChunks;
+  // every earlier use of the device buffers on the caller's stream comes first
+  if (cudaEventRecord(ev_entry, s) != cudaSuccess || cudaStreamWaitEvent(cs.in, ev_entry, 0) != cudaSuccess)
     return TA_ERR_CUDA;
-  if ((st = tiered_attn_plan(p, Qd, Kd, Vd, ws, ws_bytes, stream)) != TA_OK) return st;
-  if ((st = tiered_attn_forward(p, Qd, Kd, Vd, ws, ws_bytes, Od, stream)) != TA_OK) return st;
-  if (cudaMemcpyAsync(Oh, Od, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return TA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return TA_ERR_CUDA;  // status
+  auto chunk = [&](int c, int64_t& bh0, int64_t& n) {
+    bh0 = BH * c / nch;
+    n = BH * (c + 1) / nch - bh0;
+  };
+  const char* qh = static_cast<const char*>(Qh);
+  const char* kh = static_cast<const char*>(Kh);
+  const char* vh = static_cast<const char*>(Vh);
+  char* oh = static_cast<char*>(Oh);
+  char* qd = static_cast<char*>(Qd);
+  char* kd = static_cast<char*>(Kd);
+  char* vd = static_cast<char*>(Vd);
+  char* od = static_cast<char*>(Od);
+  for (int c = 0; c < nch; ++c) {
+    int64_t bh0, n;
+    chunk(c, bh0, n);
+    const size_t off = (size_t)bh0 * head * 2, bytes = (size_t)n * head * 2;
+    if (cudaMemcpyAsync(qd + off, qh + off, bytes, cudaMemcpyHostToDevice, cs.in) != cudaSuccess ||
+        cudaMemcpyAsync(kd + off, kh + off, bytes, cudaMemcpyHostToDevice, cs.in) != cudaSuccess ||
+        cudaMemcpyAsync(vd + off, vh + off, bytes, cudaMemcpyHostToDevice, cs.in) != cudaSuccess ||
+        cudaEventRecord(ev_in[c], cs.in) != cudaSuccess)
+      return TA_ERR_CUDA;
+  }
+  for (int c = 0; c < nch; ++c) {
+    int64_t bh0, n;
+    chunk(c, bh0, n);
+    const size_t off = (size_t)bh0 * head * 2, bytes = (size_t)n * head * 2;
+    ta_params pc = *p;   // the chunk as a layer of one batch of n heads
+    pc.B = 1;
+    pc.H = (int32_t)n;
+    pc.stride_b = (int64_t)n * head;
+    if (cudaStreamWaitEvent(s, ev_in[c], 0) != cudaSuccess) return TA_ERR_CUDA;
+    if ((st = prep_impl(&pc, qd + off, kd + off, vd + off, ws, ws_bytes, stream, false)) != TA_OK ||
+        (st = tiered_attn_route(&pc, ws, ws_bytes, stream)) != TA_OK ||
+        (st = tiered_attn_forward(&pc, qd + off, kd + off, vd + off, ws, ws_bytes, od + off, stream)) != TA_OK)
+      return st;
+    if (cudaEventRecord(ev_out[c], s) != cudaSuccess || cudaStreamWaitEvent(cs.out, ev_out[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(oh + off, od + off, bytes, cudaMemcpyDeviceToHost, cs.out) != cudaSuccess)
+      return TA_ERR_CUDA;
+  }
+  if (cudaEventRecord(ev_done, cs.out) != cudaSuccess || cudaStreamWaitEvent(s, ev_done, 0) != cudaSuccess)
+    return TA_ERR_CUDA;
   return TA_OK;
 }
 
