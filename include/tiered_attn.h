@@ -153,7 +153,7 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q_dev, const void*
  * copies O back to O_host.  Host buffers should be pinned for the copies to
  * overlap anything.
  *  - Packed layout (stride_n = d, stride_h = N*d, stride_b = H*N*d) with more
- *    than one (b, h) slice: the layer runs in up to 8 chunks of consecutive
+ *    than one (b, h) slice: the layer runs in up to 16 chunks of consecutive
  *    slices (each head is independent, so O is bit for bit that of one plan +
  *    forward).  The copies in of chunk c+1 and out of chunk c-1 overlap the
  *    kernels of chunk c: copies in are enqueued on one library-owned stream,

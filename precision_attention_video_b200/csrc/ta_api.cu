@@ -20,7 +20,7 @@ inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 // Streams and events of tiered_attn_layer_from_host, created once per device
 // on first use and kept for the life of the process.
 constexpr int kMaxDevices = 64;
-constexpr int kChunks = 8;   // chunks of (b, h) slices a layer is split into
+constexpr int kChunks = 16;  // chunks of (b, h) slices a layer is split into
 struct CopyStreams {
   bool ready = false;
   cudaStream_t in = nullptr, out = nullptr;
