@@ -120,6 +120,17 @@ __device__ __forceinline__ void gather_row_sf(unsigned char* dst, const uint8_t*
   }
 }
 
+// a / 6 for the ue4m3 block scale: a product with RN(1/6) corrected once by
+// its residual, which one FMA gives exactly (Markstein's correction step).
+// The result is the correctly rounded fp32 quotient for every a >= 2^-125
+// (checked over all floats); below that, the quotient lies far under the
+// smallest e4m3 subnormal, so the scale code it rounds to is 0 either way.
+__device__ __forceinline__ float div6(float a) {
+  const float r = 1.0f / 6.0f;
+  const float q0 = __fmul_rn(a, r);
+  return __fmaf_rn(__fmaf_rn(-6.0f, q0, a), r, q0);
+}
+
 // NVFP4 of 32 non-negative P' values, two groups of 16 keys: sc =
 // ue4m3_rn(fp32(amax / 6)), code = e2m1_rn_satfinite(fp32(x * fp32(1 / sc)))
 // (code 0 when sc = 0).  Codes go to p[0..3] (element i of a word in nibble
@@ -134,7 +145,7 @@ __device__ __forceinline__ uint32_t nvfp4_quant32(const float* x, const float2* 
 #pragma unroll
     for (int i = 0; i < 16; ++i) am[i & 3] = fmaxf(am[i & 3], x[g * 16 + i]);
     const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
-    const uint32_t scc = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xFFu;
+    const uint32_t scc = cvt_e4m3x2(div6(amax), 0.0f) & 0xFFu;
     const float inv = sc_tab[scc].y;
     scw |= scc << (8 * g);
 #pragma unroll
@@ -171,7 +182,7 @@ __device__ __forceinline__ uint32_t nvfp4_residual32(const float* x, const uint3
     float am = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(rr[i]));
-    const uint32_t scc2 = cvt_e4m3x2(__fdiv_rn(am, 6.0f), 0.0f) & 0xFFu;
+    const uint32_t scc2 = cvt_e4m3x2(div6(am), 0.0f) & 0xFFu;
     const float inv2 = sc_tab[scc2].y;
     scw2 |= scc2 << (8 * g);
 #pragma unroll
