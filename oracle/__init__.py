@@ -10,8 +10,8 @@ low-precision formats rounded in software:
 
 * ``formats``   bf16 / fp32 / FP8 e4m3 / FP4 e2m1 / ue4m3 rounding and codes;
 * ``quant``     per-tile FP8 and per-16 NVFP4 (+ residual) copies of Q, K, V;
-* ``route``     block pooling, pooled block softmax, cumulative-mass tiers,
-                threshold flags and per-row tile lists;
+* ``route``     block pooling, pooled block softmax, cumulative-mass tiers or
+                the price rule, their flags and per-row tile lists;
 * ``attention`` the one-pass online-softmax attention over the tiers;
 * ``dense``     naive fp64 softmax attention (a pin, not the method).
 
@@ -34,6 +34,7 @@ from .quant import (  # noqa: F401
 )
 from .route import (  # noqa: F401
     pool_means, pooled_mass, diag_blocks, assign_tiers, row_lists, route_head,
+    block_spread, price_tiers, assign_tiers_price, ROUTER_MASS, ROUTER_PRICE,
     TIER_SKIP, TIER_LOW, TIER_RES, TIER_FULL,
 )
 from .attention import tiered_attention_head, tiered_attention  # noqa: F401

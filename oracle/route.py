@@ -28,6 +28,28 @@ these at tile level:
 6. Lists.  Per row: full blocks, then residual, then low, then skip; within a
    tier in the sort order of step 4, so a row meets its heaviest blocks (and,
    nearly always, its largest logits) first.
+
+The price router (router = ROUTER_PRICE) replaces step 4 with Triage's rule as
+the abstract states it: predict each tile's error under each tier from block
+statistics and move a tile to a more accurate tier only when the predicted
+error reduction is worth the extra compute at a single price.  Reading:
+
+4'. Predicted error of tile (i, j) under tier t: e_t = M_ij * eps_t, with eps
+    the unit roundoff of the tier's arithmetic (bf16 2^-8; FP8 e4m3 2^-4;
+    NVFP4 e2m1 2^-2; NVFP4 plus its residual 2^-4, the square of e2m1's) and,
+    for skip, eps_skip = delta_ij = scale * sqrt(sum_c qbar_ic^2 var_jc), where
+    var_jc is the variance of coordinate c over block j's keys (the mean of
+    (k_c - kbar_jc)^2): the spread of the pooled query's logits across the
+    block were the block's key coordinates uncorrelated, which is what
+    replacing the block by its means ignores (0 when the block's keys are
+    equal, and then skipping is exact).  Cost of tier t: its tensor-pipe time
+    relative to an NVFP4 tile at the nominal rates (skip 0, NVFP4 1, FP8 2,
+    NVFP4 + residual 3, bf16 4).  The tile takes the tier of least
+    e_t + price * cost_t among the tiers the low format provides; on a tie the
+    cheaper tier.  The forced diagonal (step 4's last sentence) still applies,
+    and step 6 orders the lists as before.
+5'. A tile is flagged when another tier's objective is within 1e-6 (relative)
+    of the chosen one's.
 """
 
 from __future__ import annotations
@@ -37,9 +59,12 @@ import math
 import numpy as np
 
 from .formats import bf16_rne
+from .quant import LOW_FP8, LOW_NONE, LOW_NVFP4, LOW_NVFP4_RES
 
 TIER_SKIP, TIER_LOW, TIER_RES, TIER_FULL = 0, 1, 2, 3
 FLAG_REL = 1e-5
+ROUTER_MASS, ROUTER_PRICE = 0, 1
+FLAG_REL_PRICE = 1e-6
 
 
 def block_ranges(N: int, block: int):
@@ -107,6 +132,54 @@ def assign_tiers(M_row: np.ndarray, tau, diag=()):
     return tiers, flags
 
 
+def block_spread(X: np.ndarray, block: int) -> np.ndarray:
+    """var [nb, d]: per block, the variance of each coordinate over its rows,
+    the mean of (x_c - xbar_c)^2 (fp64, two passes)."""
+    out = []
+    for a, b in block_ranges(X.shape[0], block):
+        dev = X[a:b] - X[a:b].mean(axis=0)
+        out.append((dev * dev).mean(axis=0))
+    return np.stack(out)
+
+
+def price_tiers(low: int):
+    """(tier, eps, cost) of the tiers the low format provides, cheapest first;
+    eps None marks skip, whose error factor is the tile's delta (step 4')."""
+    skip, full = (TIER_SKIP, None, 0.0), (TIER_FULL, 2.0 ** -8, 4.0)
+    if low == LOW_NONE:
+        return [skip, full]
+    if low == LOW_FP8:
+        return [skip, (TIER_LOW, 2.0 ** -4, 2.0), full]
+    if low == LOW_NVFP4:
+        return [skip, (TIER_LOW, 2.0 ** -2, 1.0), full]
+    if low == LOW_NVFP4_RES:
+        return [skip, (TIER_LOW, 2.0 ** -2, 1.0), (TIER_RES, 2.0 ** -4, 3.0), full]
+    raise ValueError("unknown low format")
+
+
+def assign_tiers_price(M_row: np.ndarray, delta_row: np.ndarray, price: float, low: int,
+                       diag=()):
+    """Tiers (uint8 [nKb]) and flags (bool [nKb]) of one row by the price rule."""
+    n = M_row.shape[0]
+    table = price_tiers(low)
+    tiers = np.empty(n, dtype=np.uint8)
+    flags = np.zeros(n, dtype=bool)
+    for j in range(n):
+        objs = [M_row[j] * (delta_row[j] if eps is None else eps) + price * cost
+                for _, eps, cost in table]
+        best = 0
+        for t in range(1, len(objs)):
+            if objs[t] < objs[best]:
+                best = t
+        tiers[j] = table[best][0]
+        for t in range(len(objs)):
+            if t != best and abs(objs[t] - objs[best]) <= FLAG_REL_PRICE * max(abs(objs[t]), abs(objs[best])):
+                flags[j] = True
+    for jj in diag:
+        tiers[jj] = TIER_FULL
+    return tiers, flags
+
+
 def row_lists(tiers_row: np.ndarray, M_row: np.ndarray):
     """counts [full, res, low, skip] and the key-block list in that tier order;
     within a tier, blocks follow the router's (-M, j) order (largest pooled
@@ -118,8 +191,11 @@ def row_lists(tiers_row: np.ndarray, M_row: np.ndarray):
 
 
 def route_head(Qh, Kh, Vh, tau, block_q: int, block_k: int, scale: float = 0.0,
-               keep_diag_full: bool = True) -> dict:
-    """Router output for one head (fp64 values of bf16 Q, K, V [N, d])."""
+               keep_diag_full: bool = True, router: int = ROUTER_MASS, price: float = 0.0,
+               low: int = LOW_NVFP4) -> dict:
+    """Router output for one head (fp64 values of bf16 Q, K, V [N, d]).
+    ``router`` ROUTER_MASS uses ``tau`` (steps 4-5); ROUTER_PRICE uses
+    ``price`` and the tiers of ``low`` (steps 4'-5')."""
     N, d = Qh.shape
     if scale == 0.0:
         scale = 1.0 / math.sqrt(d)
@@ -127,6 +203,8 @@ def route_head(Qh, Kh, Vh, tau, block_q: int, block_k: int, scale: float = 0.0,
     kbar, n_k = pool_means(Kh, block_k)
     vbar, _ = pool_means(Vh, block_k)
     M = pooled_mass(qbar, kbar, n_k, scale)
+    kvar = block_spread(Kh, block_k)
+    delta = scale * np.sqrt((qbar * qbar) @ kvar.T)
     nqb, nkb = M.shape
     tiers = np.empty((nqb, nkb), dtype=np.uint8)
     flags = np.empty((nqb, nkb), dtype=bool)
@@ -134,8 +212,12 @@ def route_head(Qh, Kh, Vh, tau, block_q: int, block_k: int, scale: float = 0.0,
     lists = np.empty((nqb, nkb), dtype=np.int32)
     for i in range(nqb):
         diag = diag_blocks(i, block_q, block_k, N) if keep_diag_full else ()
-        tiers[i], flags[i] = assign_tiers(M[i], tau, diag)
+        if router == ROUTER_PRICE:
+            tiers[i], flags[i] = assign_tiers_price(M[i], delta[i], price, low, diag)
+        else:
+            tiers[i], flags[i] = assign_tiers(M[i], tau, diag)
         counts[i], lists[i] = row_lists(tiers[i], M[i])
     return {"qbar": qbar, "kbar": kbar, "vbar": vbar, "n_k": n_k, "M": M,
+            "kvar": kvar, "delta": delta,
             "kbar_b": bf16_rne(kbar), "vbar_b": bf16_rne(vbar), "scale": scale,
             "tiers": tiers, "flags": flags, "counts": counts, "lists": lists}
