@@ -65,6 +65,13 @@ typedef enum {
   TA_LOW_NVFP4_RES = 3       /* NVFP4 low tier plus an NVFP4+residual tier    */
 } ta_low_format;
 
+/* How tiers are chosen (see tiered_attn_plan). */
+typedef enum {
+  TA_ROUTER_MASS = 0,        /* cumulative pooled-mass thresholds tau         */
+  TA_ROUTER_PRICE = 1        /* per tile, the tier of least predicted error +
+                                price * compute cost ("Triage" abstract)       */
+} ta_router;
+
 /* Tier codes stored in the tier map. */
 enum { TA_TIER_SKIP = 0, TA_TIER_LOW = 1, TA_TIER_RES = 2, TA_TIER_FULL = 3 };
 
@@ -81,6 +88,10 @@ typedef struct {
   float   softmax_scale;     /* 0 selects 1/sqrt(d)                           */
   int32_t debug_flags;       /* test hooks, 0 in normal use (see TA_DEBUG_*)  */
   int64_t stride_b, stride_h, stride_n;  /* element strides of Q, K, V, O     */
+  int32_t router;            /* ta_router                                     */
+  double  price;             /* TA_ROUTER_PRICE: error per unit of compute the
+                                router pays for a more accurate tier (finite,
+                                >= 0); unused by TA_ROUTER_MASS                */
 } ta_params;
 
 /* Test hook: the attention producer never loads the first K tile, so the
@@ -121,6 +132,12 @@ typedef struct {
   uint16_t* dq; uint16_t* dk; uint16_t* dv;
   /* bf16 [BH, N, d] dequantised residual copies (TA_LOW_NVFP4_RES) */
   uint16_t* drq; uint16_t* drk; uint16_t* drv;
+  /* TA_ROUTER_PRICE only (NULL otherwise): f64 [BH, nKb, d] the variance of
+   * each coordinate over a key block's keys (mean of (k_c - kbar_c)^2), and
+   * f64 [BH, nQb, nKb] the skip tier's predicted relative error
+   * delta = scale * sqrt(sum_c qbar_c^2 kvar_c) */
+  double* kvar;
+  double* spread;
 } ta_plan_views;
 
 /* Bytes of workspace that tiered_attn_plan / tiered_attn_forward need for
@@ -130,12 +147,24 @@ size_t tiered_attn_workspace_bytes(const ta_params* p);
 /* Router + quantiser ("Triage" abstract: the router predicts from block
  * statistics; NVFP4 skim / refine copies).  Reads Q, K, V once: block means of
  * Q, K, V (fp64), the low-precision copies of Q, K, V (and, for FP8 and the
- * residual format, their dequantised bf16 values); then the pooled logits, the n_j-weighted pooled block softmax M,
- * the tiers by exclusive cumulative mass in (-M, j) order (most precise tier t
- * with prefix < tau[t], else skip; diagonal blocks forced full when
- * keep_diag_full), and the per-row tile lists.  Three kernel launches on
- * `stream`.  ws_dev must hold tiered_attn_workspace_bytes(p) bytes, 256-byte
- * aligned; its previous contents are overwritten (the status word is reset).
+ * residual format, their dequantised bf16 values); then the pooled logits, the
+ * n_j-weighted pooled block softmax M, the tiers, and the per-row tile lists.
+ * Tiers:
+ *  - TA_ROUTER_MASS: by exclusive cumulative mass in (-M, j) order (most
+ *    precise tier t with prefix < tau[t], else skip);
+ *  - TA_ROUTER_PRICE: each tile's error under tier t is predicted as
+ *    M * eps_t, eps the tier's unit roundoff (bf16 2^-8, FP8 2^-4, NVFP4 2^-2,
+ *    NVFP4 + residual 2^-4) and, for skip, delta = scale * sqrt(sum_c
+ *    qbar_c^2 kvar_c) with kvar_c the variance of coordinate c over the key
+ *    block; its cost is the tier's tensor-pipe time relative to an NVFP4 tile
+ *    (skip 0, NVFP4 1, FP8 2, NVFP4 + residual 3, bf16 4); the tile takes the
+ *    tier of least error + price * cost among those `low` provides (the
+ *    cheaper tier on a tie).  tau is then unused but must still be valid.
+ * Either way the diagonal blocks are forced full when keep_diag_full, and each
+ * row's list holds full, residual, low, then skip blocks, each in (-M, j)
+ * order.  Three kernel launches on `stream`.  ws_dev must hold
+ * tiered_attn_workspace_bytes(p) bytes, 256-byte aligned; its previous
+ * contents are overwritten (the status word is reset).
  * Returns TA_OK when the launches were enqueued. */
 ta_status tiered_attn_plan(const ta_params* p, const void* Q_dev, const void* K_dev,
                            const void* V_dev, void* ws_dev, size_t ws_bytes, void* stream);

@@ -45,6 +45,8 @@ class Workload:
     noise: float = 0.3                  # std of the i.i.d. noise added to Q and K
     n_features: int = 32                # cos/sin Fourier features per token
     keep_diag_full: int = 1
+    router: int = 0                     # 0: pooled-mass thresholds tau; 1: single price
+    price: float = 0.0                  # the price of router 1
     extra: Dict[str, float] = field(default_factory=dict)
 
     @property
@@ -77,6 +79,15 @@ def _sweep_tau() -> Dict[str, Tuple[float, float]]:
     return {k: tuple(v["tau"]) for k, v in raw["points"].items()}
 
 
+def _price() -> float:
+    """The price-router workload's price (written by oracle/calibrate_price.py)."""
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "price.json")
+    if not os.path.exists(path):
+        return 0.0
+    with open(path) as f:
+        return float(json.load(f)["price"])
+
+
 def _build() -> Dict[str, Workload]:
     c: Dict[str, Workload] = {}
     c["tiny"] = Workload("tiny", 1, 2, 64, (4, 16, 16), 64, 64, 3.0, LOW_FP8,
@@ -89,6 +100,11 @@ def _build() -> Dict[str, Workload]:
     # 0.675, NVFP4 up to 0.85, skip beyond.
     c["720p"] = Workload("720p", 1, 24, 128, (33, 45, 80), 128, 128, 4.0, LOW_NVFP4_RES,
                          (0.5, 0.675, 0.85), p_offset_log2=11)
+    # The 480p shape with all four tiers chosen by the single-price router;
+    # the price is calibrated on the oracle for half of the tiles skipped.
+    c["480p-price"] = Workload("480p-price", 1, 40, 128, (21, 30, 52), 128, 128, 4.0,
+                               LOW_NVFP4_RES, (0.5, 0.675, 0.85), p_offset_log2=11,
+                               router=1, price=_price())
     # Sparsity sweep on the 480p shape with an FP8 low tier; the 0% point runs
     # every tile in bf16 (thresholds above every cumulative mass).
     sweep = _sweep_tau()

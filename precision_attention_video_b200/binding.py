@@ -39,6 +39,7 @@ class ta_params(ctypes.Structure):
         ("keep_diag_full", ctypes.c_int32), ("p_offset_log2", ctypes.c_int32),
         ("softmax_scale", ctypes.c_float), ("debug_flags", ctypes.c_int32),
         ("stride_b", ctypes.c_int64), ("stride_h", ctypes.c_int64), ("stride_n", ctypes.c_int64),
+        ("router", ctypes.c_int32), ("price", ctypes.c_double),
     ]
 
 
@@ -46,7 +47,7 @@ _VIEW_FIELDS = [
     "status", "qbar", "kbar", "kbar_b", "vbar_b", "n_k", "logits", "mass", "tier_map",
     "row_counts", "row_lists", "q_codes", "k_codes", "v_codes", "q_scales", "k_scales",
     "v_scales", "rq_codes", "rk_codes", "rv_codes", "rq_scales", "rk_scales", "rv_scales",
-    "dq", "dk", "dv", "drq", "drk", "drv",
+    "dq", "dk", "dv", "drq", "drk", "drv", "kvar", "spread",
 ]
 
 
@@ -106,7 +107,8 @@ def _check(call: str, code: int) -> None:
 def make_params(B: int, H: int, N: int, d: int, block_q: int, block_k: int, low: int,
                 tau: Sequence[float], p_offset_log2: int, keep_diag_full: int = 1,
                 softmax_scale: float = 0.0, debug_flags: int = 0,
-                strides: Optional[Sequence[int]] = None) -> ta_params:
+                strides: Optional[Sequence[int]] = None, router: int = 0,
+                price: float = 0.0) -> ta_params:
     """ta_params for a [B, H, N, d] layout (contiguous unless ``strides`` = (sb, sh, sn))."""
     p = ta_params()
     p.B, p.H, p.N, p.d = B, H, N, d
@@ -118,6 +120,7 @@ def make_params(B: int, H: int, N: int, d: int, block_q: int, block_k: int, low:
     p.softmax_scale, p.debug_flags = softmax_scale, debug_flags
     sb, sh, sn = strides if strides is not None else (H * N * d, N * d, d)
     p.stride_b, p.stride_h, p.stride_n = sb, sh, sn
+    p.router, p.price = router, float(price)
     return p
 
 
@@ -125,7 +128,8 @@ def params_for(cfg, **overrides) -> ta_params:
     """ta_params of a ``latent_gen.Workload``."""
     kw = dict(B=cfg.B, H=cfg.H, N=cfg.N, d=cfg.d, block_q=cfg.block_q, block_k=cfg.block_k,
               low=cfg.low, tau=cfg.tau, p_offset_log2=cfg.p_offset_log2,
-              keep_diag_full=cfg.keep_diag_full)
+              keep_diag_full=cfg.keep_diag_full, router=getattr(cfg, "router", 0),
+              price=getattr(cfg, "price", 0.0))
     kw.update(overrides)
     return make_params(**kw)
 
@@ -209,6 +213,7 @@ def plan_views(p: ta_params, ws: torch.Tensor) -> Dict[str, torch.Tensor]:
         "row_lists": (i32, (BH, nqb, nkb)),
         "dq": (b16, (BH, N, d)), "dk": (b16, (BH, N, d)), "dv": (b16, (BH, N, d)),
         "drq": (b16, (BH, N, d)), "drk": (b16, (BH, N, d)), "drv": (b16, (BH, N, d)),
+        "kvar": (f64, (BH, nkb, d)), "spread": (f64, (BH, nqb, nkb)),
     }
     if p.low == TA_LOW_FP8_E4M3:
         shapes.update({"q_codes": (u8, (BH, N, d)), "k_codes": (u8, (BH, N, d)),

@@ -62,6 +62,9 @@ ta_status validate(const ta_params* p) {
   if (p->p_offset_log2 < 0 || p->p_offset_log2 > 15) return TA_ERR_INVALID_ARG;
   if (!std::isfinite(p->softmax_scale) || p->softmax_scale < 0.0f) return TA_ERR_INVALID_ARG;
   if (p->keep_diag_full != 0 && p->keep_diag_full != 1) return TA_ERR_INVALID_ARG;
+  if (p->router != TA_ROUTER_MASS && p->router != TA_ROUTER_PRICE) return TA_ERR_INVALID_ARG;
+  if (p->router == TA_ROUTER_PRICE && !(std::isfinite(p->price) && p->price >= 0.0))
+    return TA_ERR_INVALID_ARG;
   const Shape s = shape_of(p);
   if (s.nKb > ta::kMaxKeyBlocks) return TA_ERR_UNSUPPORTED;
   if ((int64_t)p->B * p->H > 65535 || s.nQb > 2147483647) return TA_ERR_UNSUPPORTED;
@@ -80,6 +83,7 @@ bool native_fp8(const ta_params* p) {
 // Workspace layout: byte offsets of every array (kAbsent when not produced).
 struct Layout {
   size_t status, n_k, qbar, kbar, kbar_b, vbar_b, logits, mass, tier_map, row_counts, row_lists;
+  size_t kvar, spread;
   size_t q_codes, k_codes, v_codes, q_scales, k_scales, v_scales;
   size_t rq_codes, rk_codes, rv_codes, rq_scales, rk_scales, rv_scales;
   size_t dq, dk, dv, drq, drk, drv;
@@ -107,6 +111,10 @@ Layout layout_of(const ta_params* p) {
   L.tier_map = take((size_t)s.BH * s.nQb * s.nKb);
   L.row_counts = take((size_t)s.BH * s.nQb * 4 * 4);
   L.row_lists = take((size_t)s.BH * s.nQb * s.nKb * 4);
+  if (p->router == TA_ROUTER_PRICE) {
+    L.kvar = take((size_t)s.BH * s.nKb * s.d * 8);
+    L.spread = take((size_t)s.BH * s.nQb * s.nKb * 8);
+  }
   const size_t tok = (size_t)s.BH * s.N * s.d;  // elements of one [BH, N, d] tensor
   if (p->low == TA_LOW_FP8_E4M3) {
     L.q_codes = take(tok);
@@ -181,6 +189,8 @@ void fill_plan_args(const ta_params* p, const void* Q, const void* K, const void
   a.n_tau = p->n_thresholds;
   for (int i = 0; i < 3; ++i) a.tau[i] = i < p->n_thresholds ? p->tau[i] : 0.0;
   a.keep_diag = p->keep_diag_full;
+  a.router = p->router;
+  a.price = p->price;
   a.scale = p->softmax_scale > 0.0f ? (double)p->softmax_scale : 1.0 / std::sqrt((double)p->d);
   a.status = at<int>(ws, L.status);
   a.qbar = at<double>(ws, L.qbar);
@@ -190,6 +200,8 @@ void fill_plan_args(const ta_params* p, const void* Q, const void* K, const void
   a.n_k = at<int>(ws, L.n_k);
   a.logits = at<double>(ws, L.logits);
   a.mass = at<double>(ws, L.mass);
+  a.kvar = at<double>(ws, L.kvar);
+  a.spread = at<double>(ws, L.spread);
   a.tier_map = at<uint8_t>(ws, L.tier_map);
   a.row_counts = at<int>(ws, L.row_counts);
   a.row_lists = at<int>(ws, L.row_lists);
@@ -325,6 +337,8 @@ ta_status tiered_attn_plan_views(const ta_params* p, void* ws, ta_plan_views* ou
   out->drq = at<uint16_t>(ws, L.drq);
   out->drk = at<uint16_t>(ws, L.drk);
   out->drv = at<uint16_t>(ws, L.drv);
+  out->kvar = at<double>(ws, L.kvar);
+  out->spread = at<double>(ws, L.spread);
   return TA_OK;
 }
 

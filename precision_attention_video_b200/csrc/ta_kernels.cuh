@@ -24,6 +24,8 @@ struct PlanArgs {
   int n_tau;
   double tau[3];
   int keep_diag;
+  int router;                   // ta_router
+  double price;                 // TA_ROUTER_PRICE's price
   double scale;                 // softmax scale (fp64 in the router)
   int* status;
   double* qbar;
@@ -33,6 +35,8 @@ struct PlanArgs {
   int* n_k;
   double* logits;
   double* mass;
+  double* kvar;                 // [BH, nKb, d] key-block coordinate variances (price router)
+  double* spread;               // [BH, nQb, nKb] skip error factor delta (price router)
   uint8_t* tier_map;
   int* row_counts;
   int* row_lists;

@@ -8,6 +8,7 @@
 // exactly once and produces all of them:
 //   * fp64 block sums -> qbar (per query block), kbar (per key block), and the
 //     bf16 (round-to-nearest-even) kbar_b / vbar_b used by the skip tier;
+//     for the price router also each key block's coordinate variances;
 //   * FP8 e4m3: one power-of-two scale per tile (the smallest 2^k with
 //     amax <= 448 * 2^k), codes = e4m3_rn_satfinite(x * 2^-k);
 //   * NVFP4: per 16 elements along d (Q, K rows) or along tokens (V columns,
@@ -148,6 +149,16 @@ __global__ void __launch_bounds__(kThreads, 3) prep_kernel(const PlanArgs a) {
           a.kbar[((int64_t)bh * a.nKb + gb) * D + c] = mean;
           a.kbar_b[((int64_t)bh * a.nKb + gb) * D + c] = bf16_from_double(mean);
           if (bh == 0 && c == 0) a.n_k[gb] = re - rs;
+          if (a.kvar) {
+            // variance of coordinate c over the block's keys (second pass
+            // over the staged rows, deviations from the fp64 mean)
+            double ss = 0.0;
+            for (int r = rs; r < re; ++r) {
+              const double dv = (double)bf2f(tile[r * LD + c]) - mean;
+              ss += dv * dv;
+            }
+            a.kvar[((int64_t)bh * a.nKb + gb) * D + c] = ss / (double)(re - rs);
+          }
         } else {
           a.vbar_b[((int64_t)bh * a.nKb + gb) * D + c] = bf16_from_double(mean);
         }

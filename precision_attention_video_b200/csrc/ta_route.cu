@@ -1,5 +1,5 @@
 // ta_route.cu -- the router: pooled block logits, pooled block softmax,
-// cumulative-mass tiers and compacted per-row tile lists.
+// cumulative-mass (or single-price) tiers and compacted per-row tile lists.
 //
 // "Triage" (zhuanzhiai paper page, abstract) predicts each tile's treatment
 // from block statistics; "HierPAS" (conference listing, abstract) estimates the
@@ -13,6 +13,10 @@
 //   key blocks meeting query block i's token range become full;
 //   list = full blocks, then residual, low, skip; within a tier in (-M, j)
 //   order, so a query block meets its heaviest key blocks first.
+// The price router ("Triage" abstract: move a tile to a more accurate tier
+// only when its predicted error reduction is worth the extra compute at a
+// single price) gives each tile the tier of least M * eps_t + price * cost_t,
+// with the skip tier's eps the block's logit spread delta (see price_tier).
 // The router runs in fp64 end to end (means, logits, exp, prefix), so its
 // cumulative masses agree with an fp64 evaluation to ~1e-15 relative and the
 // tier map only depends on the ordering rule, not on rounding.
@@ -24,22 +28,28 @@ namespace {
 
 // ---------------------------------------------------------------------------
 // Pooled logits: logits[bh, i, j] = scale * sum_c qbar[bh, i, c] kbar[bh, j, c]
+// and, for the price router, the skip tier's error factor
+// spread[bh, i, j] = scale * sqrt(sum_c qbar[bh, i, c]^2 kvar[bh, j, c]).
 // 32 x 32 output tile per CTA, 2 x 2 per thread, d staged 32 at a time.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) logits_kernel(const PlanArgs a) {
   __shared__ double qs[32][33];
   __shared__ double ks[32][33];
+  __shared__ double vs[32][33];
   const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
   const int bh = blockIdx.z, i0 = blockIdx.x * 32, j0 = blockIdx.y * 32;
   const int D = a.d;
   const double* qb = a.qbar + (int64_t)bh * a.nQb * D;
   const double* kb = a.kbar + (int64_t)bh * a.nKb * D;
+  const double* kvb = a.kvar ? a.kvar + (int64_t)bh * a.nKb * D : nullptr;
   double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+  double spr[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
   for (int c0 = 0; c0 < D; c0 += 32) {
     for (int e = tid; e < 32 * 32; e += 256) {
       const int r = e / 32, c = e % 32;
       qs[r][c] = (i0 + r < a.nQb) ? qb[(int64_t)(i0 + r) * D + c0 + c] : 0.0;
       ks[r][c] = (j0 + r < a.nKb) ? kb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
+      if (kvb) vs[r][c] = (j0 + r < a.nKb) ? kvb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
     }
     __syncthreads();
 #pragma unroll 8
@@ -51,13 +61,49 @@ __global__ void __launch_bounds__(256) logits_kernel(const PlanArgs a) {
       acc[1][0] += q1 * k0;
       acc[1][1] += q1 * k1;
     }
+    if (kvb) {
+#pragma unroll 8
+      for (int c = 0; c < 32; ++c) {
+        const double q0 = qs[ty * 2][c], q1 = qs[ty * 2 + 1][c];
+        const double v0 = vs[tx * 2][c], v1 = vs[tx * 2 + 1][c];
+        spr[0][0] += q0 * q0 * v0;
+        spr[0][1] += q0 * q0 * v1;
+        spr[1][0] += q1 * q1 * v0;
+        spr[1][1] += q1 * q1 * v1;
+      }
+    }
     __syncthreads();
   }
   for (int u = 0; u < 2; ++u)
     for (int v = 0; v < 2; ++v) {
       const int i = i0 + ty * 2 + u, j = j0 + tx * 2 + v;
-      if (i < a.nQb && j < a.nKb) a.logits[((int64_t)bh * a.nQb + i) * a.nKb + j] = acc[u][v] * a.scale;
+      if (i < a.nQb && j < a.nKb) {
+        a.logits[((int64_t)bh * a.nQb + i) * a.nKb + j] = acc[u][v] * a.scale;
+        if (kvb) a.spread[((int64_t)bh * a.nQb + i) * a.nKb + j] = a.scale * sqrt(spr[u][v]);
+      }
     }
+}
+
+// The price router's tier of one tile: the least predicted error + price *
+// cost among the tiers the low format provides, cheapest first, keeping the
+// cheaper tier on a tie.  Error = M * eps (eps: the tier's unit roundoff; for
+// skip, the tile's spread delta); cost = tensor-pipe time relative to an
+// NVFP4 tile.
+__device__ __forceinline__ int price_tier(double M, double delta, double price, int low) {
+  int best = TA_TIER_SKIP;
+  double obj = M * delta;
+  auto consider = [&](int tier, double eps, double cost) {
+    const double o = M * eps + price * cost;
+    if (o < obj) {
+      obj = o;
+      best = tier;
+    }
+  };
+  if (low == TA_LOW_FP8_E4M3) consider(TA_TIER_LOW, 0.0625, 2.0);
+  if (low == TA_LOW_NVFP4 || low == TA_LOW_NVFP4_RES) consider(TA_TIER_LOW, 0.25, 1.0);
+  if (low == TA_LOW_NVFP4_RES) consider(TA_TIER_RES, 0.0625, 3.0);
+  consider(TA_TIER_FULL, 0.00390625, 4.0);
+  return best;
 }
 
 // ---------------------------------------------------------------------------
@@ -116,6 +162,8 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs 
       key[j] = m;
       idx[j] = j;
       a.mass[g * nKb + j] = m;
+      if (a.router == TA_ROUTER_PRICE)
+        tier[j] = (uint8_t)price_tier(m, a.spread[g * nKb + j], a.price, a.low);
     } else {
       key[j] = -1.0;
       idx[j] = 0x7fffffff - (sortn - j);
@@ -167,15 +215,17 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs 
     codes[1] = TA_TIER_RES;
     codes[2] = TA_TIER_LOW;
   }
-  for (int r = lane * per; r < (lane + 1) * per; ++r) {
-    const int j = idx[r];
-    if (j < nKb) {
-      int t = TA_TIER_SKIP;
-      for (int q = a.n_tau - 1; q >= 0; --q)
-        if (C < a.tau[q]) t = codes[q];
-      tier[j] = (uint8_t)t;
+  if (a.router != TA_ROUTER_PRICE) {
+    for (int r = lane * per; r < (lane + 1) * per; ++r) {
+      const int j = idx[r];
+      if (j < nKb) {
+        int t = TA_TIER_SKIP;
+        for (int q = a.n_tau - 1; q >= 0; --q)
+          if (C < a.tau[q]) t = codes[q];
+        tier[j] = (uint8_t)t;
+      }
+      C += fmax(key[r], 0.0);
     }
-    C += fmax(key[r], 0.0);
   }
   __syncwarp();
   if (a.keep_diag && lane == 0) {

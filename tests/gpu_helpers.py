@@ -56,12 +56,19 @@ def unpack_fp4(packed: np.ndarray) -> np.ndarray:
     return np.stack([lo, hi], axis=-1).reshape(*packed.shape[:-1], packed.shape[-1] * 2)
 
 
+def router_kwargs(cfg, low=None):
+    """route_head keywords of the workload's router (mass thresholds or price)."""
+    return {"router": getattr(cfg, "router", 0), "price": getattr(cfg, "price", 0.0),
+            "low": cfg.low if low is None else low}
+
+
 def oracle_head(cfg, Q, K, V, b, h, qblocks=None, exact=False, tau=None, low=None,
                 keep_diag=True):
     Qh, Kh, Vh = to64(Q[b, h]), to64(K[b, h]), to64(V[b, h])
     tau = cfg.tau if tau is None else tau
     low = cfg.low if low is None else low
-    rt = Rt.route_head(Qh, Kh, Vh, tau, cfg.block_q, cfg.block_k, keep_diag_full=keep_diag)
+    rt = Rt.route_head(Qh, Kh, Vh, tau, cfg.block_q, cfg.block_k, keep_diag_full=keep_diag,
+                       **router_kwargs(cfg, low))
     qt = Qz.quantize_head(Qh, Kh, Vh, low, cfg.block_q, cfg.block_k)
     O = None
     if qblocks != []:

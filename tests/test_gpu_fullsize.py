@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from gpu_helpers import (assert_out_close, check_lists, check_vt, compare_tiers, oracle_head,
-                         to64, unpack_fp4)
+                         router_kwargs, to64, unpack_fp4)
 from latent_gen import get_config, make_qkv
 from oracle import quant as Qz
 from oracle import route as Rt
@@ -37,7 +37,10 @@ def _run_full(name):
 
 def _check_head(cfg, Q, K, V, views, O, h, qblocks):
     Qh, Kh, Vh = to64(Q[0, h]), to64(K[0, h]), to64(V[0, h])
-    rt = Rt.route_head(Qh, Kh, Vh, cfg.tau, cfg.block_q, cfg.block_k)
+    rt = Rt.route_head(Qh, Kh, Vh, cfg.tau, cfg.block_q, cfg.block_k, **router_kwargs(cfg))
+    if getattr(cfg, "router", 0) == Rt.ROUTER_PRICE:
+        np.testing.assert_allclose(views["kvar"][h].cpu().numpy(), rt["kvar"], rtol=1e-12, atol=0)
+        np.testing.assert_allclose(views["spread"][h].cpu().numpy(), rt["delta"], rtol=1e-12, atol=0)
     tiers = views["tier_map"][h].cpu().numpy()
     _, rows = compare_tiers(tiers, rt)
     check_lists(tiers, views["row_counts"][h].cpu().numpy(), views["row_lists"][h].cpu().numpy(),
@@ -63,7 +66,7 @@ def _check_head(cfg, Q, K, V, views, O, h, qblocks):
     return assert_out_close(to64(O[0, h].cpu()), Oref, f"{cfg.name} head {h}")
 
 
-@pytest.mark.parametrize("name", ["480p", "sweep70", "720p"])
+@pytest.mark.parametrize("name", ["480p", "sweep70", "720p", "480p-price"])
 def test_fullsize_sampled_parity(cuda_ok, name):
     cfg, Q, K, V, views, O = _run_full(name)
     nqb = cfg.n_qb

@@ -33,6 +33,11 @@ def _plan_parity(cfg, Q, K, V, views, heads):
         np.testing.assert_allclose(views["logits"][bh].numpy(), (rt["qbar"] @ rt["kbar"].T) * rt["scale"],
                                    rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(views["mass"][bh].numpy(), rt["M"], rtol=1e-10, atol=1e-15)
+        if getattr(cfg, "router", 0) == 1:
+            # the price router's block statistics: key-block coordinate
+            # variances and the skip tier's predicted error factor
+            np.testing.assert_allclose(views["kvar"][bh].numpy(), rt["kvar"], rtol=1e-12, atol=0)
+            np.testing.assert_allclose(views["spread"][bh].numpy(), rt["delta"], rtol=1e-12, atol=0)
         tiers = views["tier_map"][bh].numpy()
         compare_tiers(tiers, rt)
         check_lists(tiers, views["row_counts"][bh].numpy(), views["row_lists"][bh].numpy(),
@@ -219,3 +224,27 @@ def test_all_full_d128_matches_sdpa(cuda_ok):
         Q.cuda().float(), K.cuda().float(), V.cuda().float()).cpu()
     rel = (O.float() - ref).norm() / ref.norm()
     assert rel < 1e-2
+
+
+@pytest.mark.parametrize("name,grid,price", [
+    ("480p-price", (3, 10, 21), 0.02),   # four tiers: bf16, NVFP4 + residual, NVFP4, skip
+    ("480p", (3, 10, 21), 0.02),         # NVFP4 low tier
+    ("sweep70", (3, 10, 21), 0.03),      # native FP8 low tier
+    ("small", None, 0.002),              # FP8 low tier on bf16 images (d = 64, 64-key tiles)
+])
+def test_price_router_parity(cuda_ok, name, grid, price):
+    over = {"H": 3, "router": 1, "price": price}
+    if grid is not None:
+        over["grid"] = grid
+    cfg, Q, K, V = inputs(name, **over)
+    _, views, O, st = run_gpu(cfg, Q, K, V)
+    assert st == 0
+    t = views["tier_map"].numpy()
+    assert len(np.unique(t)) >= 3
+    _plan_parity(cfg, Q, K, V, views, [(0, h) for h in range(cfg.H)])
+    for h in range(cfg.H):
+        rt, qt, Oref = oracle_head(cfg, Q, K, V, 0, h)
+        _, rows = compare_tiers(views["tier_map"][h].numpy(), rt)
+        for i in rows:
+            Oref[i * cfg.block_q:(i + 1) * cfg.block_q] = np.nan
+        assert_out_close(to64(O[0, h]), Oref, f"price router {name} head {h}")
