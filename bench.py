@@ -215,6 +215,75 @@ def sweep(args):
         del ws
 
 
+def plan_reuse(args):
+    """Plan reuse across timesteps: on a slowly changing sequence of K inputs
+    (latent_gen.make_qkv_steps, correlation rho between steps), one plan
+    serves K layers (tiered_attn_prep + tiered_attn_forward on the others),
+    against a fresh plan on every step.  One JSON line: time per layer both
+    ways and how far the last step's output moves from the fresh plan's."""
+    import precision_attention_video_b200 as pav
+    from latent_gen.generator import make_qkv_steps
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = workload(args)
+    k = args.reuse
+    seq = [tuple(x.to(dev) for x in step) for step in make_qkv_steps(cfg, k, args.rho)]
+    p = pav.params_for(cfg)
+    ws = pav.alloc_workspace(p, dev)
+    ws_fresh = pav.alloc_workspace(p, dev)
+    O = torch.empty_like(seq[0][0])
+    O_fresh = torch.empty_like(O)
+
+    def reuse_group():
+        for t, (Q, K, V) in enumerate(seq):
+            (pav.plan if t == 0 else pav.prep)(p, Q, K, V, ws)
+            pav.forward(p, Q, K, V, ws, O)
+
+    def fresh_group():
+        for Q, K, V in seq:
+            pav.plan(p, Q, K, V, ws_fresh)
+            pav.forward(p, Q, K, V, ws_fresh, O_fresh)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for _ in range(args.steps):
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) / k)
+        return statistics.median(ts)
+
+    ms_reuse = timed(reuse_group)
+    ms_fresh = timed(fresh_group)
+    st = max(pav.get_status(ws), pav.get_status(ws_fresh), key=abs)
+    # both workspaces and outputs now hold the last step: compare them, and
+    # each with dense attention of that step (torch SDPA, measurement only)
+    rel = float((O.float() - O_fresh.float()).norm() / O_fresh.float().norm())
+    Ql, Kl, Vl = seq[-1]
+    dense_o = torch.nn.functional.scaled_dot_product_attention(Ql, Kl, Vl).float()
+    err_reuse = float((O.float() - dense_o).norm() / dense_o.norm())
+    err_fresh = float((O_fresh.float() - dense_o).norm() / dense_o.norm())
+    same = float((pav.plan_views(p, ws)["tier_map"] == pav.plan_views(p, ws_fresh)["tier_map"])
+                 .float().mean())
+    dense = 4.0 * cfg.B * cfg.H * float(cfg.N) ** 2 * cfg.d
+    print(json.dumps({
+        "metric": METRIC, "mode": "plan reuse across timesteps", "workload": cfg.name,
+        "every": k, "rho": args.rho, "status": st,
+        "ms_per_layer_reused_plan": ms_reuse, "ms_per_layer_fresh_plan": ms_fresh,
+        "dense_equiv_tflops_reused": dense / (ms_reuse * 1e-3) / 1e12,
+        "dense_equiv_tflops_fresh": dense / (ms_fresh * 1e-3) / 1e12,
+        "speedup": ms_fresh / ms_reuse,
+        "last_step": {"rel_l2_vs_fresh_plan": rel, "tier_map_agreement": same,
+                      "rel_l2_vs_dense_reused_plan": err_reuse,
+                      "rel_l2_vs_dense_fresh_plan": err_fresh}}), flush=True)
+
+
 def run_gpu_arm(args, rank, world, local_rank):
     import precision_attention_video_b200 as pav
 
@@ -351,11 +420,18 @@ def main():
                     help="workload name (latent_gen.configs); the contract line uses 480p")
     ap.add_argument("--sweep", action="store_true",
                     help="time the sparsity sweep instead (one JSON line per point)")
+    ap.add_argument("--reuse", type=int, default=0,
+                    help="time plan reuse instead: one plan per K timesteps of a correlated sequence")
+    ap.add_argument("--rho", type=float, default=0.99,
+                    help="correlation between consecutive timesteps for --reuse")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     if args.sweep:
         sweep(args)
+        return
+    if args.reuse > 0:
+        plan_reuse(args)
         return
     world = _env_int("WORLD_SIZE", 1)
     rank = _env_int("RANK", 0)

@@ -210,9 +210,19 @@ ta_status tiered_attn_plan_views(const ta_params* p, void* ws_dev, ta_plan_views
  * (TA_OK, or the first device-side error such as TA_ERR_TIMEOUT). */
 ta_status tiered_attn_get_status(const void* ws_dev, void* stream);
 
-/* Test entry points: each launches one stage of tiered_attn_plan alone. */
+/* The first stage of tiered_attn_plan alone: block means of Q, K, V (and the
+ * skip tier's bf16 copies) and the low-precision copies, one kernel launch.
+ * The router's output already in ws_dev (tier map, counts, lists) is left as
+ * it is, so tiered_attn_prep + tiered_attn_forward runs a layer on a plan made
+ * by an earlier tiered_attn_plan: plan reuse across diffusion timesteps ("APT"
+ * Lattice paper summary, TAFA: attention probabilities change slowly across
+ * timesteps), which skips the pooled logits and the routing.  Same
+ * requirements and errors as tiered_attn_plan; `p` must be the plan's. */
 ta_status tiered_attn_prep(const ta_params* p, const void* Q_dev, const void* K_dev,
                            const void* V_dev, void* ws_dev, size_t ws_bytes, void* stream);
+
+/* Test entry point: the second stage of tiered_attn_plan alone (pooled
+ * logits and routing over the block means already in ws_dev). */
 ta_status tiered_attn_route(const ta_params* p, void* ws_dev, size_t ws_bytes, void* stream);
 
 /* Router that allocates nothing (the pages have no counterpart: this is a

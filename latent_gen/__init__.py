@@ -6,4 +6,4 @@ attention method itself: it only draws Q, K, V and names the workloads.
 """
 
 from .configs import CONFIGS, Workload, get_config  # noqa: F401
-from .generator import grid_positions, make_qkv, make_head  # noqa: F401
+from .generator import grid_positions, make_qkv, make_head, make_qkv_steps  # noqa: F401

@@ -132,3 +132,18 @@ def make_qkv(cfg: Workload, threads: int = 0):
         with ThreadPoolExecutor(max_workers=threads) as ex:
             list(ex.map(one, range(n)))
     return Q, K, V
+
+
+def make_qkv_steps(cfg: Workload, steps: int, rho: float):
+    """A sequence of ``steps`` (Q, K, V) bf16 tensors for successive diffusion
+    timesteps that change slowly: step 0 is ``make_qkv(cfg)``; step t mixes the
+    previous step with a fresh draw of the same generator (seed shifted by t),
+    X_t = bf16(rho X_{t-1} + sqrt(1 - rho^2) Y_t) for each of Q, K, V, which
+    keeps every step's distribution and correlates consecutive steps by rho."""
+    seq = [make_qkv(cfg)]
+    a, b = float(rho), float(np.sqrt(max(0.0, 1.0 - rho * rho)))
+    for t in range(1, steps):
+        fresh = make_qkv(cfg.with_(seed=cfg.seed + 1000 + t))
+        seq.append(tuple((a * x.float() + b * y.float()).to(torch.bfloat16)
+                         for x, y in zip(seq[-1], fresh)))
+    return seq

@@ -50,6 +50,13 @@ error reduction is worth the extra compute at a single price.  Reading:
     and step 6 orders the lists as before.
 5'. A tile is flagged when another tier's objective is within 1e-6 (relative)
     of the chosen one's.
+
+Plan reuse ("APT" TAFA, Lattice paper summary: attention probabilities are
+predicted across diffusion timesteps from their similarity): a plan made on
+the inputs of one timestep serves the next ones.  Reading: a reused step keeps
+the plan's tier map, flags and lists (steps 4-6) and takes everything else
+from its own inputs: the block means (so the skip tier uses the current
+kbar_j, vbar_j) and the low-precision copies.
 """
 
 from __future__ import annotations
@@ -221,3 +228,19 @@ def route_head(Qh, Kh, Vh, tau, block_q: int, block_k: int, scale: float = 0.0,
             "kvar": kvar, "delta": delta,
             "kbar_b": bf16_rne(kbar), "vbar_b": bf16_rne(vbar), "scale": scale,
             "tiers": tiers, "flags": flags, "counts": counts, "lists": lists}
+
+
+def reuse_plan(rt_plan: dict, Qh, Kh, Vh, block_q: int, block_k: int, scale: float = 0.0) -> dict:
+    """Router output for the current inputs under a plan made on earlier ones:
+    ``rt_plan``'s tiers, flags, counts and lists; the current block means."""
+    N, d = Qh.shape
+    if scale == 0.0:
+        scale = 1.0 / math.sqrt(d)
+    qbar, _ = pool_means(Qh, block_q)
+    kbar, n_k = pool_means(Kh, block_k)
+    vbar, _ = pool_means(Vh, block_k)
+    out = dict(rt_plan)
+    out.update({"qbar": qbar, "kbar": kbar, "vbar": vbar, "n_k": n_k,
+                "M": pooled_mass(qbar, kbar, n_k, scale),
+                "kbar_b": bf16_rne(kbar), "vbar_b": bf16_rne(vbar), "scale": scale})
+    return out

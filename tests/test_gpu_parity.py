@@ -248,3 +248,44 @@ def test_price_router_parity(cuda_ok, name, grid, price):
         for i in rows:
             Oref[i * cfg.block_q:(i + 1) * cfg.block_q] = np.nan
         assert_out_close(to64(O[0, h]), Oref, f"price router {name} head {h}")
+
+
+def test_plan_reuse_parity(cuda_ok):
+    # a plan made on timestep 0 serves timestep 2 of a slowly changing
+    # sequence: tiers and lists from step 0, block means and low copies from step 2
+    import precision_attention_video_b200 as pav
+    from latent_gen import get_config
+    from latent_gen.generator import make_qkv_steps
+    from oracle import route as Rt
+    from oracle.attention import tiered_attention_head
+    cfg = get_config("480p").with_(H=2, grid=(3, 10, 21))
+    seq = make_qkv_steps(cfg, 3, rho=0.95)
+    dev = torch.device("cuda:0")
+    p = pav.params_for(cfg)
+    ws = pav.alloc_workspace(p, dev)
+    Q0, K0, V0 = (x.to(dev) for x in seq[0])
+    pav.plan(p, Q0, K0, V0, ws)
+    Q2, K2, V2 = (x.to(dev) for x in seq[2])
+    pav.prep(p, Q2, K2, V2, ws)
+    O = torch.empty_like(Q2)
+    pav.forward(p, Q2, K2, V2, ws, O)
+    torch.cuda.synchronize()
+    assert pav.get_status(ws) == 0
+    views = {k: v.cpu() for k, v in pav.plan_views(p, ws).items()}
+    for h in range(cfg.H):
+        s0 = [to64(x[0, h]) for x in seq[0]]
+        s2 = [to64(x[0, h]) for x in seq[2]]
+        rt0 = Rt.route_head(*s0, cfg.tau, cfg.block_q, cfg.block_k)
+        _, rows = compare_tiers(views["tier_map"][h].numpy(), rt0)
+        ru = Rt.reuse_plan(rt0, *s2, cfg.block_q, cfg.block_k)
+        np.testing.assert_array_equal(to64(views["kbar_b"][h]), ru["kbar_b"])
+        np.testing.assert_array_equal(to64(views["vbar_b"][h]), ru["vbar_b"])
+        qt = Qz.quantize_head(*s2, cfg.low, cfg.block_q, cfg.block_k)
+        for t in "qk":
+            np.testing.assert_array_equal(unpack_fp4(views[f"{t}_codes"][h].numpy()), qt[f"{t}_codes"])
+        check_vt(views["v_codes"][h].numpy(), views["v_scales"][h].numpy(), qt["v_codes"], qt["v_sc"])
+        Oref = tiered_attention_head(*s2, ru, qt, cfg.low, cfg.block_q, cfg.block_k,
+                                     cfg.p_offset_log2, ru["scale"], False)
+        for i in rows:
+            Oref[i * cfg.block_q:(i + 1) * cfg.block_q] = np.nan
+        assert_out_close(to64(O[0, h]), Oref, f"plan reuse head {h}")
