@@ -34,7 +34,8 @@ from .quant import (  # noqa: F401
 )
 from .route import (  # noqa: F401
     pool_means, pooled_mass, diag_blocks, assign_tiers, row_lists, route_head,
-    block_spread, price_tiers, assign_tiers_price, reuse_plan, ROUTER_MASS, ROUTER_PRICE,
+    block_spread, price_tiers, assign_tiers_price, reuse_plan, assign_tiers_entropy,
+    ROUTER_MASS, ROUTER_PRICE, ROUTER_ENTROPY,
     TIER_SKIP, TIER_LOW, TIER_RES, TIER_FULL,
 )
 from .attention import tiered_attention_head, tiered_attention  # noqa: F401

@@ -143,7 +143,7 @@ def tiered_attention_head(Qh, Kh, Vh, rt, qt, low, block_q, block_k, p_offset_lo
 
 def tiered_attention(Q, K, V, tau, low, block_q, block_k, p_offset_log2, scale=0.0,
                      keep_diag_full=True, exact=False, heads=None, qblocks=None, threads=1,
-                     router=0, price=0.0):
+                     router=0, price=0.0, kappa=1.0):
     """Route, quantise and attend over every (b, h) in ``heads`` (default all).
 
     Q, K, V: fp64 arrays [B, H, N, d] holding bf16 values.  Returns a dict
@@ -154,7 +154,7 @@ def tiered_attention(Q, K, V, tau, low, block_q, block_k, p_offset_log2, scale=0
     out = {}
     for b, h in heads:
         rt = route_head(Q[b, h], K[b, h], V[b, h], tau, block_q, block_k, scale, keep_diag_full,
-                        router=router, price=price, low=low)
+                        router=router, price=price, low=low, kappa=kappa)
         qt = quantize_head(Q[b, h], K[b, h], V[b, h], low, block_q, block_k)
         O = tiered_attention_head(Q[b, h], K[b, h], V[b, h], rt, qt, low, block_q, block_k,
                                   p_offset_log2, rt["scale"], exact, qblocks, threads)

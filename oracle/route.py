@@ -51,6 +51,22 @@ error reduction is worth the extra compute at a single price.  Reading:
 5'. A tile is flagged when another tier's objective is within 1e-6 (relative)
     of the chosen one's.
 
+The entropy router (router = ROUTER_ENTROPY) follows "HierPAS" (conference
+listing, abstract): retention ratios adapted across heads and blocks from an
+entropy analysis of a cheap estimate of the attention pattern, and precision
+reduced progressively on the less critical part.  Reading, per query block i
+(its pooled distribution M_i. is the pattern estimate of step 3):
+
+4''. H_i = -sum_j M_ij ln M_ij; the row keeps k_i = min(nKb, max(1,
+     ceil(kappa exp(H_i)))) key blocks, exp(H_i) being the effective number of
+     blocks it attends and kappa the retention scale.  In the (-M, j) order of
+     step 4, ranks r < k_i are kept, with the precision of step 4's prefix
+     rule (the most precise t with C_r < tau_t), or the least precise kept tier
+     when no threshold is met; ranks r >= k_i are skipped.  The forced
+     diagonal still applies.
+5''. A row's tiles are flagged when kappa exp(H_i) is within 1e-9 (relative)
+     of an integer, besides step 5's flags.
+
 Plan reuse ("APT" TAFA, Lattice paper summary: attention probabilities are
 predicted across diffusion timesteps from their similarity): a plan made on
 the inputs of one timestep serves the next ones.  Reading: a reused step keeps
@@ -70,7 +86,8 @@ from .quant import LOW_FP8, LOW_NONE, LOW_NVFP4, LOW_NVFP4_RES
 
 TIER_SKIP, TIER_LOW, TIER_RES, TIER_FULL = 0, 1, 2, 3
 FLAG_REL = 1e-5
-ROUTER_MASS, ROUTER_PRICE = 0, 1
+ROUTER_MASS, ROUTER_PRICE, ROUTER_ENTROPY = 0, 1, 2
+FLAG_REL_ENTROPY = 1e-9
 FLAG_REL_PRICE = 1e-6
 
 
@@ -139,6 +156,30 @@ def assign_tiers(M_row: np.ndarray, tau, diag=()):
     return tiers, flags
 
 
+def assign_tiers_entropy(M_row: np.ndarray, tau, kappa: float, diag=()):
+    """Tiers (uint8 [nKb]), flags (bool [nKb]) and k_i of one row by the
+    entropy retention rule (step 4'')."""
+    n = M_row.shape[0]
+    pos = M_row[M_row > 0]
+    H = float(-(pos * np.log(pos)).sum())
+    want = kappa * math.exp(H)
+    k = min(n, max(1, math.ceil(want)))
+    tiers, flags = assign_tiers(M_row, tau)          # precision by the prefix rule
+    order = np.lexsort((np.arange(n), -M_row))
+    kept_low = tier_codes_for(tau)[-1]
+    for r, j in enumerate(order):
+        if r >= k:
+            tiers[j] = TIER_SKIP
+        elif tiers[j] == TIER_SKIP:
+            tiers[j] = kept_low
+    near = abs(want - round(want)) <= FLAG_REL_ENTROPY * max(1.0, want)
+    if near:
+        flags[:] = True
+    for jj in diag:
+        tiers[jj] = TIER_FULL
+    return tiers, flags, k
+
+
 def block_spread(X: np.ndarray, block: int) -> np.ndarray:
     """var [nb, d]: per block, the variance of each coordinate over its rows,
     the mean of (x_c - xbar_c)^2 (fp64, two passes)."""
@@ -199,10 +240,11 @@ def row_lists(tiers_row: np.ndarray, M_row: np.ndarray):
 
 def route_head(Qh, Kh, Vh, tau, block_q: int, block_k: int, scale: float = 0.0,
                keep_diag_full: bool = True, router: int = ROUTER_MASS, price: float = 0.0,
-               low: int = LOW_NVFP4) -> dict:
+               low: int = LOW_NVFP4, kappa: float = 1.0) -> dict:
     """Router output for one head (fp64 values of bf16 Q, K, V [N, d]).
     ``router`` ROUTER_MASS uses ``tau`` (steps 4-5); ROUTER_PRICE uses
-    ``price`` and the tiers of ``low`` (steps 4'-5')."""
+    ``price`` and the tiers of ``low`` (steps 4'-5'); ROUTER_ENTROPY uses
+    ``kappa`` and ``tau`` (steps 4''-5'')."""
     N, d = Qh.shape
     if scale == 0.0:
         scale = 1.0 / math.sqrt(d)
@@ -217,15 +259,18 @@ def route_head(Qh, Kh, Vh, tau, block_q: int, block_k: int, scale: float = 0.0,
     flags = np.empty((nqb, nkb), dtype=bool)
     counts = np.empty((nqb, 4), dtype=np.int32)
     lists = np.empty((nqb, nkb), dtype=np.int32)
+    keep = np.full(nqb, nkb, dtype=np.int64)
     for i in range(nqb):
         diag = diag_blocks(i, block_q, block_k, N) if keep_diag_full else ()
         if router == ROUTER_PRICE:
             tiers[i], flags[i] = assign_tiers_price(M[i], delta[i], price, low, diag)
+        elif router == ROUTER_ENTROPY:
+            tiers[i], flags[i], keep[i] = assign_tiers_entropy(M[i], tau, kappa, diag)
         else:
             tiers[i], flags[i] = assign_tiers(M[i], tau, diag)
         counts[i], lists[i] = row_lists(tiers[i], M[i])
     return {"qbar": qbar, "kbar": kbar, "vbar": vbar, "n_k": n_k, "M": M,
-            "kvar": kvar, "delta": delta,
+            "kvar": kvar, "delta": delta, "keep": keep,
             "kbar_b": bf16_rne(kbar), "vbar_b": bf16_rne(vbar), "scale": scale,
             "tiers": tiers, "flags": flags, "counts": counts, "lists": lists}
 
