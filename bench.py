@@ -445,6 +445,8 @@ def main():
               "N": cfg.N, "d": cfg.d, "grid_txyx": list(cfg.grid),
               "tile": [cfg.block_q, cfg.block_k], "low_tier": LOW_NAMES[cfg.low],
               **({"router": "single price", "price": cfg.price} if getattr(cfg, "router", 0) == 1
+                 else {"router": "entropy retention", "kappa": cfg.kappa, "tau": list(cfg.tau)}
+                 if getattr(cfg, "router", 0) == 2
                  else {"router": "cumulative pooled mass", "tau": list(cfg.tau)}),
               "logit_std": cfg.logit_std,
               "l2": f"inputs larger than L2 (Q+K+V {3 * cfg.B * cfg.H * cfg.N * cfg.d * 2 / 1e9:.2f} GB per GPU)",

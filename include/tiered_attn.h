@@ -68,8 +68,11 @@ typedef enum {
 /* How tiers are chosen (see tiered_attn_plan). */
 typedef enum {
   TA_ROUTER_MASS = 0,        /* cumulative pooled-mass thresholds tau         */
-  TA_ROUTER_PRICE = 1        /* per tile, the tier of least predicted error +
+  TA_ROUTER_PRICE = 1,       /* per tile, the tier of least predicted error +
                                 price * compute cost ("Triage" abstract)       */
+  TA_ROUTER_ENTROPY = 2      /* per query block, keep the ceil(retention *
+                                exp(H)) heaviest key blocks, H the entropy of the
+                                pooled pattern ("HierPAS" abstract)            */
 } ta_router;
 
 /* Tier codes stored in the tier map. */
@@ -91,7 +94,9 @@ typedef struct {
   int32_t router;            /* ta_router                                     */
   double  price;             /* TA_ROUTER_PRICE: error per unit of compute the
                                 router pays for a more accurate tier (finite,
-                                >= 0); unused by TA_ROUTER_MASS                */
+                                >= 0); unused by the other routers             */
+  double  retention;         /* TA_ROUTER_ENTROPY: kappa, the kept blocks per
+                                effective block (finite, > 0); unused otherwise */
 } ta_params;
 
 /* Test hook: the attention producer never loads the first K tile, so the
@@ -159,7 +164,11 @@ size_t tiered_attn_workspace_bytes(const ta_params* p);
  *    block; its cost is the tier's tensor-pipe time relative to an NVFP4 tile
  *    (skip 0, NVFP4 1, FP8 2, NVFP4 + residual 3, bf16 4); the tile takes the
  *    tier of least error + price * cost among those `low` provides (the
- *    cheaper tier on a tie).  tau is then unused but must still be valid.
+ *    cheaper tier on a tie).  tau is then unused but must still be valid;
+ *  - TA_ROUTER_ENTROPY: per query block i, H_i = -sum_j M_ij ln M_ij and the
+ *    row keeps k_i = min(nKb, max(1, ceil(retention * exp(H_i)))) key blocks,
+ *    the first k_i in (-M, j) order, with the precision of the mass rule (the
+ *    least precise kept tier where that rule would skip); the rest are skipped.
  * Either way the diagonal blocks are forced full when keep_diag_full, and each
  * row's list holds full, residual, low, then skip blocks, each in (-M, j)
  * order.  Three kernel launches on `stream`.  ws_dev must hold

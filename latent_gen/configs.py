@@ -45,8 +45,9 @@ class Workload:
     noise: float = 0.3                  # std of the i.i.d. noise added to Q and K
     n_features: int = 32                # cos/sin Fourier features per token
     keep_diag_full: int = 1
-    router: int = 0                     # 0: pooled-mass thresholds tau; 1: single price
+    router: int = 0                     # 0: pooled-mass thresholds tau; 1: single price; 2: entropy
     price: float = 0.0                  # the price of router 1
+    kappa: float = 1.0                  # the retention scale of router 2
     extra: Dict[str, float] = field(default_factory=dict)
 
     @property
@@ -88,6 +89,16 @@ def _price() -> float:
         return float(json.load(f)["price"])
 
 
+def _kappa() -> float:
+    """The entropy-router workload's retention scale (written by
+    oracle/calibrate_entropy.py)."""
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "kappa.json")
+    if not os.path.exists(path):
+        return 1.0
+    with open(path) as f:
+        return float(json.load(f)["kappa"])
+
+
 def _build() -> Dict[str, Workload]:
     c: Dict[str, Workload] = {}
     c["tiny"] = Workload("tiny", 1, 2, 64, (4, 16, 16), 64, 64, 3.0, LOW_FP8,
@@ -105,6 +116,12 @@ def _build() -> Dict[str, Workload]:
     c["480p-price"] = Workload("480p-price", 1, 40, 128, (21, 30, 52), 128, 128, 4.0,
                                LOW_NVFP4_RES, (0.5, 0.675, 0.85), p_offset_log2=11,
                                router=1, price=_price())
+    # The 480p layer with the kept blocks of each query block chosen from the
+    # entropy of its pooled pattern; kappa calibrated on the oracle for half
+    # of the tiles skipped.
+    c["480p-entropy"] = Workload("480p-entropy", 1, 40, 128, (21, 30, 52), 128, 128, 4.0,
+                                 LOW_NVFP4, (0.6, 0.9), p_offset_log2=11, router=2,
+                                 kappa=_kappa())
     # Sparsity sweep on the 480p shape with an FP8 low tier; the 0% point runs
     # every tile in bf16 (thresholds above every cumulative mass).
     sweep = _sweep_tau()

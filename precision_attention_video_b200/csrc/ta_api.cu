@@ -62,7 +62,10 @@ ta_status validate(const ta_params* p) {
   if (p->p_offset_log2 < 0 || p->p_offset_log2 > 15) return TA_ERR_INVALID_ARG;
   if (!std::isfinite(p->softmax_scale) || p->softmax_scale < 0.0f) return TA_ERR_INVALID_ARG;
   if (p->keep_diag_full != 0 && p->keep_diag_full != 1) return TA_ERR_INVALID_ARG;
-  if (p->router != TA_ROUTER_MASS && p->router != TA_ROUTER_PRICE) return TA_ERR_INVALID_ARG;
+  if (p->router != TA_ROUTER_MASS && p->router != TA_ROUTER_PRICE && p->router != TA_ROUTER_ENTROPY)
+    return TA_ERR_INVALID_ARG;
+  if (p->router == TA_ROUTER_ENTROPY && !(std::isfinite(p->retention) && p->retention > 0.0))
+    return TA_ERR_INVALID_ARG;
   if (p->router == TA_ROUTER_PRICE && !(std::isfinite(p->price) && p->price >= 0.0))
     return TA_ERR_INVALID_ARG;
   const Shape s = shape_of(p);
@@ -191,6 +194,7 @@ void fill_plan_args(const ta_params* p, const void* Q, const void* K, const void
   a.keep_diag = p->keep_diag_full;
   a.router = p->router;
   a.price = p->price;
+  a.retention = p->retention;
   a.scale = p->softmax_scale > 0.0f ? (double)p->softmax_scale : 1.0 / std::sqrt((double)p->d);
   a.status = at<int>(ws, L.status);
   a.qbar = at<double>(ws, L.qbar);

@@ -26,6 +26,7 @@ struct PlanArgs {
   int keep_diag;
   int router;                   // ta_router
   double price;                 // TA_ROUTER_PRICE's price
+  double retention;             // TA_ROUTER_ENTROPY's kappa
   double scale;                 // softmax scale (fp64 in the router)
   int* status;
   double* qbar;

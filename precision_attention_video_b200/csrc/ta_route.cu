@@ -13,6 +13,9 @@
 //   key blocks meeting query block i's token range become full;
 //   list = full blocks, then residual, low, skip; within a tier in (-M, j)
 //   order, so a query block meets its heaviest key blocks first.
+// The entropy router ("HierPAS" abstract: retention ratios from an entropy
+// analysis of a cheap pattern estimate) keeps, per query block, the
+// ceil(kappa exp(H)) heaviest key blocks, H the entropy of the pooled row.
 // The price router ("Triage" abstract: move a tile to a more accurate tier
 // only when its predicted error reduction is worth the extra compute at a
 // single price) gives each tile the tier of least M * eps_t + price * cost_t,
@@ -156,6 +159,17 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs 
     part += w;
   }
   const double total = warp_sum(part);
+  // entropy router: keep the ceil(kappa exp(H)) heaviest blocks of the row
+  int keep = nKb;
+  if (a.router == TA_ROUTER_ENTROPY) {
+    double hp = 0.0;
+    for (int j = lane; j < nKb; j += 32) {
+      const double m = key[j] / total;
+      if (m > 0.0) hp -= m * log(m);
+    }
+    const double want = a.retention * exp(warp_sum(hp));
+    keep = (int)fmin((double)nKb, fmax(1.0, ceil(want)));
+  }
   for (int j = lane; j < sortn; j += 32) {
     if (j < nKb) {
       const double m = key[j] / total;
@@ -216,12 +230,14 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs 
     codes[2] = TA_TIER_LOW;
   }
   if (a.router != TA_ROUTER_PRICE) {
+    const int kept_low = codes[a.n_tau - 1];   // least precise kept tier
     for (int r = lane * per; r < (lane + 1) * per; ++r) {
       const int j = idx[r];
       if (j < nKb) {
         int t = TA_TIER_SKIP;
         for (int q = a.n_tau - 1; q >= 0; --q)
           if (C < a.tau[q]) t = codes[q];
+        if (a.router == TA_ROUTER_ENTROPY) t = (r >= keep) ? TA_TIER_SKIP : (t == TA_TIER_SKIP ? kept_low : t);
         tier[j] = (uint8_t)t;
       }
       C += fmax(key[r], 0.0);

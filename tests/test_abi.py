@@ -66,13 +66,17 @@ def test_workspace_bytes_and_validation(pav):
         dict(d=96), dict(block_q=32), dict(N=0), dict(low=7), dict(tau=(0.9, 0.6)),
         dict(low=3), dict(low=0), dict(p_offset_log2=40), dict(N=200000),
         dict(strides=(2 * 1000 * 64, 1000 * 64, 60)),
-        dict(router=2), dict(router=-1), dict(router=1, price=-1e-3),
+        dict(router=3), dict(router=-1), dict(router=1, price=-1e-3),
         dict(router=1, price=float("nan")), dict(router=1, price=float("inf")),
+        dict(router=2, retention=0.0), dict(router=2, retention=-1.0),
+        dict(router=2, retention=float("nan")),
     ]
     for kw in bad:
         assert pav.workspace_bytes(_params(pav, **kw)) == 0, kw
-    # the price router adds its block statistics to the workspace
+    # the price router adds its block statistics to the workspace; the
+    # entropy router needs none
     assert pav.workspace_bytes(_params(pav, router=1, price=1e-3)) > n
+    assert pav.workspace_bytes(_params(pav, router=2, retention=0.5)) == n
 
 
 def test_calls_reject_bad_arguments_before_launch(pav):

@@ -289,3 +289,27 @@ def test_plan_reuse_parity(cuda_ok):
         for i in rows:
             Oref[i * cfg.block_q:(i + 1) * cfg.block_q] = np.nan
         assert_out_close(to64(O[0, h]), Oref, f"plan reuse head {h}")
+
+
+@pytest.mark.parametrize("name,grid,kappa", [
+    ("480p", (3, 10, 21), 0.5),          # NVFP4 low tier
+    ("720p", (3, 9, 20), 1.0),           # four tiers
+    ("sweep70", (3, 10, 21), 0.5),       # native FP8 low tier
+    ("small", None, 0.5),                # FP8 low tier on bf16 images
+])
+def test_entropy_router_parity(cuda_ok, name, grid, kappa):
+    over = {"H": 2, "router": 2, "kappa": kappa}
+    if grid is not None:
+        over["grid"] = grid
+    cfg, Q, K, V = inputs(name, **over)
+    _, views, O, st = run_gpu(cfg, Q, K, V)
+    assert st == 0
+    t = views["tier_map"].numpy()
+    assert len(np.unique(t)) >= 3
+    _plan_parity(cfg, Q, K, V, views, [(0, h) for h in range(cfg.H)])
+    for h in range(cfg.H):
+        rt, qt, Oref = oracle_head(cfg, Q, K, V, 0, h)
+        _, rows = compare_tiers(views["tier_map"][h].numpy(), rt)
+        for i in rows:
+            Oref[i * cfg.block_q:(i + 1) * cfg.block_q] = np.nan
+        assert_out_close(to64(O[0, h]), Oref, f"entropy router {name} head {h}")
