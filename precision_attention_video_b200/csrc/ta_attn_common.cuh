@@ -120,17 +120,6 @@ __device__ __forceinline__ void gather_row_sf(unsigned char* dst, const uint8_t*
   }
 }
 
-// a / 6 for the ue4m3 block scale: a product with RN(1/6) corrected once by
-// its residual, which one FMA gives exactly (Markstein's correction step).
-// The result is the correctly rounded fp32 quotient for every a >= 2^-125
-// (checked over all floats); below that, the quotient lies far under the
-// smallest e4m3 subnormal, so the scale code it rounds to is 0 either way.
-__device__ __forceinline__ float div6(float a) {
-  const float r = 1.0f / 6.0f;
-  const float q0 = __fmul_rn(a, r);
-  return __fmaf_rn(__fmaf_rn(-6.0f, q0, a), r, q0);
-}
-
 // NVFP4 of 32 non-negative P' values, two groups of 16 keys: sc =
 // ue4m3_rn(fp32(amax / 6)), code = e2m1_rn_satfinite(fp32(x * fp32(1 / sc)))
 // (code 0 when sc = 0).  Codes go to p[0..3] (element i of a word in nibble

@@ -378,6 +378,17 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t codes16) {
 __device__ __forceinline__ float e4m3_to_float(uint32_t code) {
   return e4m3x2_to_float2(code & 0xFF).x;
 }
+// a / 6 for the ue4m3 block scale: a product with RN(1/6) corrected once by
+// its residual, which one FMA gives exactly (Markstein's correction step).
+// The result is the correctly rounded fp32 quotient for every a >= 2^-125
+// (checked over all floats); below that, the quotient lies far under the
+// smallest e4m3 subnormal, so the scale code it rounds to is 0 either way.
+__device__ __forceinline__ float div6(float a) {
+  const float r = 1.0f / 6.0f;
+  const float q0 = __fmul_rn(a, r);
+  return __fmaf_rn(__fmaf_rn(-6.0f, q0, a), r, q0);
+}
+
 // Pack two floats to e2m1 (RNE, satfinite): `lo` in the low nibble.
 __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
   uint32_t r;

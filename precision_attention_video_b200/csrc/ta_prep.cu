@@ -41,16 +41,17 @@ __device__ __forceinline__ float fp8_pow2_scale(float amax) {
 
 // NVFP4 of one group of 16 values: packed codes (element 2i in the low nibble
 // of byte i) and the ue4m3 scale code; the scale value comes back in `sc`.
+// `inv_tab[c]` is the correctly rounded reciprocal of ue4m3 code c's value.
 __device__ __forceinline__ void nvfp4_group(const float (&x)[16], uint32_t (&packed)[2],
-                                            uint32_t& sc_code, float& sc) {
+                                            uint32_t& sc_code, float& sc, const float* inv_tab) {
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
-  sc_code = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xFFu;
+  sc_code = cvt_e4m3x2(div6(amax), 0.0f) & 0xFFu;
   sc = e4m3_to_float(sc_code);
   packed[0] = packed[1] = 0u;
   if (sc == 0.0f) return;
-  const float inv = __frcp_rn(sc);
+  const float inv = inv_tab[sc_code];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t c = cvt_e2m1x2(__fmul_rn(x[2 * i], inv), __fmul_rn(x[2 * i + 1], inv));
@@ -80,7 +81,12 @@ __global__ void __launch_bounds__(kThreads, 3) prep_kernel(const PlanArgs a) {
   float* red = reinterpret_cast<float*>(rtile + R * LD);
   float* tile_scale = red + kThreads;
 
+  __shared__ float inv_tab[128];   // ue4m3 code -> correctly rounded 1 / value
   const int tid = threadIdx.x;
+  if (tid < 128) {
+    const float v = (tid == 0x7F) ? 0.0f : e4m3_to_float(tid);
+    inv_tab[tid] = v > 0.0f ? __frcp_rn(v) : 0.0f;
+  }
   const int bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
   const int r0 = blockIdx.x * R;
@@ -208,55 +214,58 @@ __global__ void __launch_bounds__(kThreads, 3) prep_kernel(const PlanArgs a) {
             make_uint4(w[0], w[1], w[2], w[3]);
       }
     } else {
-      // ---- NVFP4 (+ residual) ----
+      // ---- NVFP4 (+ residual); no bf16 images of these copies are kept ----
       const bool res = (a.low == TA_LOW_NVFP4_RES);
       uint8_t* rcodes = which == 0 ? a.rq_codes : which == 1 ? a.rk_codes : a.rv_codes;
       uint8_t* scales = reinterpret_cast<uint8_t*>(which == 0 ? a.q_scales
                                                    : which == 1 ? a.k_scales
                                                                 : a.v_scales);
       uint8_t* rscales = which == 0 ? a.rq_scales : which == 1 ? a.rk_scales : a.rv_scales;
-      __nv_bfloat16* rdeq_out = which == 0 ? a.drq : which == 1 ? a.drk : a.drv;
       if (which < 2) {
         // groups of 16 along d; codes [BH, N, D/2], scales [BH, N, D/16]
         for (int idx = tid; idx < R * (D / 16); idx += kThreads) {
           const int r = idx / (D / 16), g = idx % (D / 16);
           if (r >= nrows) continue;
-          __nv_bfloat16* px = tile + r * LD + g * 16;
+          const uint4* pv = reinterpret_cast<const uint4*>(tile + r * LD + g * 16);
           float x[16], dqv[16], sc;
           uint32_t pk[2], scc;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) x[i] = bf2f(px[i]);
-          nvfp4_group(x, pk, scc, sc);
+          for (int v = 0; v < 2; ++v) {
+            const uint4 w = pv[v];
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              x[v * 8 + e * 2] = __uint_as_float(ws[e] << 16);
+              x[v * 8 + e * 2 + 1] = __uint_as_float(ws[e] & 0xFFFF0000u);
+            }
+          }
+          nvfp4_group(x, pk, scc, sc, inv_tab);
           const int64_t row = bhN + r0 + r;
           *reinterpret_cast<uint2*>(codes + row * (D / 2) + g * 8) = make_uint2(pk[0], pk[1]);
           scales[row * (D / 16) + g] = (uint8_t)scc;
-          if (deq_out != nullptr || res) nvfp4_dequant(pk, sc, dqv);
-          if (deq_out != nullptr) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) px[i] = __float2bfloat16_rn(dqv[i]);
-          }
           if (res) {
-            float rr[16], rdq[16], rsc;
+            float rr[16], rsc;
+            nvfp4_dequant(pk, sc, dqv);
 #pragma unroll
             for (int i = 0; i < 16; ++i) rr[i] = __fsub_rn(x[i], dqv[i]);
-            nvfp4_group(rr, pk, scc, rsc);
-            if (rdeq_out != nullptr) nvfp4_dequant(pk, rsc, rdq);
+            nvfp4_group(rr, pk, scc, rsc, inv_tab);
             *reinterpret_cast<uint2*>(rcodes + row * (D / 2) + g * 8) = make_uint2(pk[0], pk[1]);
             rscales[row * (D / 16) + g] = (uint8_t)scc;
-            if (rdeq_out != nullptr) {
-              __nv_bfloat16* pr = rtile + r * LD + g * 16;
-#pragma unroll
-              for (int i = 0; i < 16; ++i) pr[i] = __float2bfloat16_rn(rdq[i]);
-            }
           }
         }
       } else {
         // V: groups of 16 tokens per column; codes [BH, D, Np/2] (transposed),
-        // scales [BH, Np/16, D].  Thread map: column slow, group fast.
-        // every group of 16 tokens below the padded pitch Np: groups past N come
-        // out as zero codes with a zero scale
-        for (int idx = tid; idx < D * (R / 16); idx += kThreads) {
-          const int c = idx / (R / 16), g = idx % (R / 16);
+        // scales [BH, Np/16, D].  Threads walk the columns fastest, so that a
+        // warp reads one 64-byte run of a staged row at a time (no bank
+        // conflicts); the codes go column-major to shared memory (the residual
+        // tile area, unused here; group-major with a padded row of D + 1, so
+        // that both the writes here and the reads below avoid bank conflicts)
+        // and leave 64 bytes per column.  Groups past
+        // N come out as zero codes with a zero scale, up to the pitch Np.
+        const int G = R / 16;
+        uint2* vst = reinterpret_cast<uint2*>(rtile);   // [copy][G][D + 1]
+        for (int idx = tid; idx < D * G; idx += kThreads) {
+          const int c = idx % D, g = idx / D;
           if (r0 + g * 16 >= a.Np) continue;
           float x[16], dqv[16], sc;
           uint32_t pk[2], scc;
@@ -265,45 +274,28 @@ __global__ void __launch_bounds__(kThreads, 3) prep_kernel(const PlanArgs a) {
             const int r = g * 16 + i;
             x[i] = (r < nrows) ? bf2f(tile[r * LD + c]) : 0.0f;
           }
-          nvfp4_group(x, pk, scc, sc);
-          if (deq_out != nullptr || res) nvfp4_dequant(pk, sc, dqv);
+          nvfp4_group(x, pk, scc, sc, inv_tab);
           const int64_t tok = r0 + g * 16;
-          *reinterpret_cast<uint2*>(codes + ((int64_t)bh * D + c) * (a.Np / 2) + tok / 2) =
-              make_uint2(pk[0], pk[1]);
+          vst[g * (D + 1) + c] = make_uint2(pk[0], pk[1]);
           scales[((int64_t)bh * (a.Np / 16) + tok / 16) * D + c] = (uint8_t)scc;
-          if (deq_out != nullptr) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int r = g * 16 + i;
-              if (r < nrows) tile[r * LD + c] = __float2bfloat16_rn(dqv[i]);
-            }
-          }
           if (res) {
-            float rr[16], rdq[16], rsc;
+            float rr[16], rsc;
+            nvfp4_dequant(pk, sc, dqv);
 #pragma unroll
             for (int i = 0; i < 16; ++i) rr[i] = __fsub_rn(x[i], dqv[i]);
-            nvfp4_group(rr, pk, scc, rsc);
-            if (rdeq_out != nullptr) nvfp4_dequant(pk, rsc, rdq);
-            *reinterpret_cast<uint2*>(rcodes + ((int64_t)bh * D + c) * (a.Np / 2) + tok / 2) =
-                make_uint2(pk[0], pk[1]);
+            nvfp4_group(rr, pk, scc, rsc, inv_tab);
+            vst[(G + g) * (D + 1) + c] = make_uint2(pk[0], pk[1]);
             rscales[((int64_t)bh * (a.Np / 16) + tok / 16) * D + c] = (uint8_t)scc;
-            if (rdeq_out != nullptr) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const int r = g * 16 + i;
-                if (r < nrows) rtile[r * LD + c] = __float2bfloat16_rn(rdq[i]);
-              }
-            }
           }
         }
-      }
-      __syncthreads();
-      if (res && rdeq_out != nullptr) {
-        for (int idx = tid; idx < R * (D / 8); idx += kThreads) {
-          const int r = idx / (D / 8), c8 = idx % (D / 8);
-          if (r < nrows)
-            *reinterpret_cast<uint4*>(rdeq_out + (bhN + r0 + r) * D + c8 * 8) =
-                *reinterpret_cast<const uint4*>(rtile + r * LD + c8 * 8);
+        __syncthreads();
+        const int gv = min(G, (a.Np - r0) / 16);   // groups below the pitch
+        const int copies = res ? 2 : 1;
+        for (int idx = tid; idx < copies * D * gv; idx += kThreads) {
+          const int copy = idx / (D * gv), rem = idx % (D * gv);
+          const int c = rem / gv, g = rem % gv;
+          uint8_t* dst = (copy ? rcodes : codes) + ((int64_t)bh * D + c) * (a.Np / 2) + r0 / 2 + g * 8;
+          *reinterpret_cast<uint2*>(dst) = vst[(copy * G + g) * (D + 1) + c];
         }
       }
     }

@@ -313,3 +313,18 @@ def test_entropy_router_parity(cuda_ok, name, grid, kappa):
         for i in rows:
             Oref[i * cfg.block_q:(i + 1) * cfg.block_q] = np.nan
         assert_out_close(to64(O[0, h]), Oref, f"entropy router {name} head {h}")
+
+
+def test_forward_parity_batch_of_two(cuda_ok):
+    # B = 2: every (b, h) routed and attended independently, strides over b
+    cfg, Q, K, V = inputs("480p", grid=(2, 10, 16), H=2, B=2)   # N = 320 = 2*128 + 64
+    _, views, O, st = run_gpu(cfg, Q, K, V)
+    assert st == 0
+    _plan_parity(cfg, Q, K, V, views, [(b, h) for b in range(2) for h in range(2)])
+    for b in range(2):
+        for h in range(2):
+            rt, qt, Oref = oracle_head(cfg, Q, K, V, b, h)
+            _, rows = compare_tiers(views["tier_map"][b * cfg.H + h].numpy(), rt)
+            for i in rows:
+                Oref[i * cfg.block_q:(i + 1) * cfg.block_q] = np.nan
+            assert_out_close(to64(O[b, h]), Oref, f"batch {b} head {h}")
