@@ -129,16 +129,62 @@ __device__ __forceinline__ double warp_sum(double v) {
   return v;
 }
 
-__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs a, int sortn) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+// Bitonic sort of 32*E (key, idx) pairs held by one warp, element e = k*32 +
+// lane in register k of lane `lane`, into (-key, idx) order.  Partners less
+// than 32 apart are in other lanes (shuffles); farther ones are in this lane's
+// registers.  Fully unrolled, so every register index is a constant.
+template <int E>
+__device__ __forceinline__ void warp_sort(double (&key)[E], int (&idx)[E], int lane) {
+  constexpr int n = 32 * E;
+#pragma unroll
+  for (int size = 2; size <= n; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride >= 32) {
+        const int ks = stride / 32;
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+          const int kp = k ^ ks;
+          if (kp > k) {
+            const bool up = (((k * 32 + lane) & size) == 0);
+            const bool sw = up ? before(key[kp], idx[kp], key[k], idx[k])
+                               : before(key[k], idx[k], key[kp], idx[kp]);
+            if (sw) {
+              const double tk = key[k];
+              key[k] = key[kp];
+              key[kp] = tk;
+              const int ti = idx[k];
+              idx[k] = idx[kp];
+              idx[kp] = ti;
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+          const double ok = __shfl_xor_sync(0xffffffffu, key[k], stride);
+          const int oi = __shfl_xor_sync(0xffffffffu, idx[k], stride);
+          const bool lower = (lane & stride) == 0;
+          const bool up = (((k * 32 + lane) & size) == 0);
+          // the lower position of an ascending pair keeps the element that
+          // comes first; of a descending pair, the one that comes second
+          const bool mine_first = before(key[k], idx[k], ok, oi);
+          if ((lower == up) != mine_first) {
+            key[k] = ok;
+            idx[k] = oi;
+          }
+        }
+      }
+    }
+  }
+}
+
+template <int E>
+__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs a) {
+  constexpr int sortn = 32 * E;
+  __shared__ uint8_t tier_s[kRouteWarps][sortn];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  double* key = reinterpret_cast<double*>(smem_raw) + (size_t)warp * sortn;
-  int* idx = reinterpret_cast<int*>(reinterpret_cast<double*>(smem_raw) + (size_t)kRouteWarps * sortn) +
-             (size_t)warp * sortn;
-  uint8_t* tier = reinterpret_cast<uint8_t*>(reinterpret_cast<int*>(reinterpret_cast<double*>(smem_raw) +
-                                                                    (size_t)kRouteWarps * sortn) +
-                                             (size_t)kRouteWarps * sortn) +
-                  (size_t)warp * sortn;
+  uint8_t* tier = tier_s[warp];
 
   const int64_t g = (int64_t)blockIdx.x * kRouteWarps + warp;  // global row
   const int64_t nrows = (int64_t)a.B * a.H * a.nQb;
@@ -147,77 +193,63 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs 
   const int nKb = a.nKb;
   const double* lrow = a.logits + g * nKb;
 
-  // pooled block softmax weighted by key counts
+  // pooled block softmax weighted by key counts; element e = k*32 + lane
+  double key[E];
+  int idx[E];
   double mx = -INFINITY;
-  for (int j = lane; j < nKb; j += 32) mx = fmax(mx, lrow[j]);
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    const int j = k * 32 + lane;
+    key[k] = j < nKb ? lrow[j] : -INFINITY;
+    mx = fmax(mx, key[k]);
+  }
   mx = warp_max(mx);
   double part = 0.0;
-  for (int j = lane; j < nKb; j += 32) {
-    const int nj = min(a.bk, a.N - j * a.bk);
-    const double w = (double)nj * exp(lrow[j] - mx);
-    key[j] = w;
-    part += w;
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    const int j = k * 32 + lane;
+    if (j < nKb) {
+      const int nj = min(a.bk, a.N - j * a.bk);
+      key[k] = (double)nj * exp(key[k] - mx);
+      part += key[k];
+    }
   }
   const double total = warp_sum(part);
   // entropy router: keep the ceil(kappa exp(H)) heaviest blocks of the row
   int keep = nKb;
   if (a.router == TA_ROUTER_ENTROPY) {
     double hp = 0.0;
-    for (int j = lane; j < nKb; j += 32) {
-      const double m = key[j] / total;
-      if (m > 0.0) hp -= m * log(m);
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const int j = k * 32 + lane;
+      if (j < nKb) {
+        const double m = key[k] / total;
+        if (m > 0.0) hp -= m * log(m);
+      }
     }
     const double want = a.retention * exp(warp_sum(hp));
     keep = (int)fmin((double)nKb, fmax(1.0, ceil(want)));
   }
-  for (int j = lane; j < sortn; j += 32) {
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    const int j = k * 32 + lane;
     if (j < nKb) {
-      const double m = key[j] / total;
-      key[j] = m;
-      idx[j] = j;
+      const double m = key[k] / total;
+      key[k] = m;
+      idx[k] = j;
       a.mass[g * nKb + j] = m;
       if (a.router == TA_ROUTER_PRICE)
         tier[j] = (uint8_t)price_tier(m, a.spread[g * nKb + j], a.price, a.low);
     } else {
-      key[j] = -1.0;
-      idx[j] = 0x7fffffff - (sortn - j);
-    }
-  }
-  __syncwarp();
-
-  // bitonic sort into (-M, j) order
-  for (int k = 2; k <= sortn; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int t = lane; t < sortn; t += 32) {
-        const int u = t ^ jj;
-        if (u > t) {
-          const double kt = key[t], ku = key[u];
-          const int it = idx[t], iu = idx[u];
-          const bool up = (t & k) == 0;
-          const bool sw = up ? before(ku, iu, kt, it) : before(kt, it, ku, iu);
-          if (sw) {
-            key[t] = ku;
-            key[u] = kt;
-            idx[t] = iu;
-            idx[u] = it;
-          }
-        }
-      }
-      __syncwarp();
+      key[k] = -1.0;
+      idx[k] = 0x7fffffff - (sortn - j);
     }
   }
 
-  // exclusive prefix of the sorted masses, then tiers by rank
-  const int per = sortn / 32;
-  double lsum = 0.0;
-  for (int r = lane * per; r < (lane + 1) * per; ++r) lsum += fmax(key[r], 0.0);
-  double incl = lsum;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  double C = incl - lsum;
+  // sort into (-M, j) order: rank r = k*32 + lane holds (key[k], idx[k])
+  warp_sort<E>(key, idx, lane);
+
+  // tiers by rank: exclusive prefix of the sorted masses, rank r = k*32 + lane
   int codes[3];
   if (a.n_tau == 1) {
     codes[0] = TA_TIER_FULL;
@@ -231,8 +263,19 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs 
   }
   if (a.router != TA_ROUTER_PRICE) {
     const int kept_low = codes[a.n_tau - 1];   // least precise kept tier
-    for (int r = lane * per; r < (lane + 1) * per; ++r) {
-      const int j = idx[r];
+    double base = 0.0;                          // masses of all ranks before this row of 32
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const double mk = fmax(key[k], 0.0);
+      double incl = mk;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const double C = base + (incl - mk);
+      base += __shfl_sync(0xffffffffu, incl, 31);
+      const int j = idx[k], r = k * 32 + lane;
       if (j < nKb) {
         int t = TA_TIER_SKIP;
         for (int q = a.n_tau - 1; q >= 0; --q)
@@ -240,7 +283,6 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs 
         if (a.router == TA_ROUTER_ENTROPY) t = (r >= keep) ? TA_TIER_SKIP : (t == TA_TIER_SKIP ? kept_low : t);
         tier[j] = (uint8_t)t;
       }
-      C += fmax(key[r], 0.0);
     }
   }
   __syncwarp();
@@ -258,8 +300,9 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs 
   for (int q = 0; q < 4; ++q) {
     const int t = order[q];
     int cnt = 0;
-    for (int r0 = 0; r0 < sortn; r0 += 32) {
-      const int j = idx[r0 + lane];
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const int j = idx[k];
       const bool p = (j < nKb) && tier[j] == t;
       const unsigned bal = __ballot_sync(0xffffffffu, p);
       if (p) a.row_lists[g * nKb + base + cnt + __popc(bal & ((1u << lane) - 1u))] = j;
@@ -279,12 +322,17 @@ cudaError_t launch_route(const PlanArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   int sortn = 32;
   while (sortn < a.nKb) sortn <<= 1;
-  const size_t smem = (size_t)kRouteWarps * sortn * (sizeof(double) + sizeof(int) + 1);
-  e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   const int64_t rows = (int64_t)a.B * a.H * a.nQb;
   dim3 g2((unsigned)((rows + kRouteWarps - 1) / kRouteWarps));
-  route_kernel<<<g2, kRouteWarps * 32, smem, s>>>(a, sortn);
+  switch (sortn) {
+    case 32: route_kernel<1><<<g2, kRouteWarps * 32, 0, s>>>(a); break;
+    case 64: route_kernel<2><<<g2, kRouteWarps * 32, 0, s>>>(a); break;
+    case 128: route_kernel<4><<<g2, kRouteWarps * 32, 0, s>>>(a); break;
+    case 256: route_kernel<8><<<g2, kRouteWarps * 32, 0, s>>>(a); break;
+    case 512: route_kernel<16><<<g2, kRouteWarps * 32, 0, s>>>(a); break;
+    case 1024: route_kernel<32><<<g2, kRouteWarps * 32, 0, s>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 
