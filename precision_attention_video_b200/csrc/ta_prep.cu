@@ -15,7 +15,8 @@
 //     groups aligned to token 0) a ue4m3 scale sc = e4m3_rn(amax / 6), codes
 //     e2m1_rn_satfinite(x * rcp_rn(sc)); residual copies quantise
 //     fp32(x - dequant(x)) the same way;
-//   * the dequantised values of each copy, in bf16 (exact: at most 6
+//   * for an FP8 low tier that the attention kernel runs on bf16 images (d =
+//     64 or 64-row tiles), the dequantised values in bf16 (exact: at most 4
 //     significant bits), row-major like the input.
 // One CTA per (chunk of R = max(bq, bk) tokens, head, operand Q / K / V); the
 // chunk is staged in shared memory with 16-byte coalesced loads and written
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(kThreads, 3) prep_kernel(const PlanArgs a) {
   constexpr int LD = D + 8;  // padded row stride (elements)
   const int R = a.R;
   __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(smem_raw);
-  __nv_bfloat16* rtile = tile + R * LD;  // residual dequantised values (NVFP4_RES)
+  __nv_bfloat16* rtile = tile + R * LD;  // staging of the transposed NVFP4 V codes
   float* red = reinterpret_cast<float*>(rtile + R * LD);
   float* tile_scale = red + kThreads;
 
