@@ -328,3 +328,29 @@ def test_forward_parity_batch_of_two(cuda_ok):
             for i in rows:
                 Oref[i * cfg.block_q:(i + 1) * cfg.block_q] = np.nan
             assert_out_close(to64(O[b, h]), Oref, f"batch {b} head {h}")
+
+
+def test_head_interleaved_layout_matches_contiguous(cuda_ok):
+    # Q, K, V, O stored [B, N, H, d] (heads interleaved per token) and passed
+    # with their strides: the same plan and output, bit for bit, as the
+    # contiguous [B, H, N, d] run
+    import precision_attention_video_b200 as pav
+    cfg, Q, K, V = inputs("480p", grid=(3, 10, 21), H=3)
+    _, views1, O1, st1 = run_gpu(cfg, Q, K, V)
+    assert st1 == 0
+    dev = torch.device("cuda:0")
+    Qs, Ks, Vs = (x.permute(0, 2, 1, 3).contiguous().to(dev).permute(0, 2, 1, 3) for x in (Q, K, V))
+    assert Qs.stride() == (cfg.N * cfg.H * cfg.d, cfg.d, cfg.H * cfg.d, 1)
+    p = pav.params_for(cfg, strides=Qs.stride()[:3])
+    ws = pav.alloc_workspace(p, dev)
+    pav.plan(p, Qs, Ks, Vs, ws)
+    Os = torch.empty_like(Qs)
+    assert Os.stride() == Qs.stride()
+    pav.forward(p, Qs, Ks, Vs, ws, Os)
+    torch.cuda.synchronize()
+    assert pav.get_status(ws) == 0
+    views = {k: v.cpu() for k, v in pav.plan_views(p, ws).items()}
+    for k in ("tier_map", "row_counts", "row_lists", "qbar", "kbar", "q_codes", "k_codes", "v_codes",
+              "q_scales", "k_scales", "v_scales"):
+        assert torch.equal(views[k], views1[k]), k
+    assert torch.equal(Os.cpu(), O1)
