@@ -141,9 +141,12 @@ typedef struct {
   /* TA_ROUTER_PRICE only (NULL otherwise): f64 [BH, nKb, d] the variance of
    * each coordinate over a key block's keys (mean of (k_c - kbar_c)^2), and
    * f64 [BH, nQb, nKb] the skip tier's predicted relative error
-   * delta = scale * sqrt(sum_c qbar_c^2 kvar_c) */
+   * delta = scale * sqrt(sum_c (qbar_c^2 + qvar_c) kvar_c) */
   double* kvar;
   double* spread;
+  /* TA_ROUTER_PRICE only: f64 [BH, nQb, d] the same variances over a query
+   * block's queries */
+  double* qvar;
 } ta_plan_views;
 
 /* Bytes of workspace that tiered_attn_plan / tiered_attn_forward need for
@@ -162,8 +165,8 @@ size_t tiered_attn_workspace_bytes(const ta_params* p);
  *  - TA_ROUTER_PRICE: each tile's error under tier t is predicted as
  *    M * eps_t, eps the tier's unit roundoff (bf16 2^-8, FP8 2^-4, NVFP4 2^-2,
  *    NVFP4 + residual 2^-4) and, for skip, delta = scale * sqrt(sum_c
- *    qbar_c^2 kvar_c) with kvar_c the variance of coordinate c over the key
- *    block; its cost is the tier's tensor-pipe time relative to an NVFP4 tile
+ *    (qbar_c^2 + qvar_c) kvar_c) with kvar_c (qvar_c) the variance of
+ *    coordinate c over the key (query) block; its cost is the tier's tensor-pipe time relative to an NVFP4 tile
  *    (skip 0, NVFP4 1, FP8 2, NVFP4 + residual 3, bf16 4); the tile takes the
  *    tier of least error + price * cost among those `low` provides (the
  *    cheaper tier on a tie).  tau is then unused but must still be valid;

@@ -48,7 +48,8 @@ def head_stats(cfg):
         qbar, _ = pool_means(Qh, cfg.block_q)
         kbar, n_k = pool_means(Kh, cfg.block_k)
         M = pooled_mass(qbar, kbar, n_k, scale)
-        delta = scale * np.sqrt((qbar * qbar) @ block_spread(Kh, cfg.block_k).T)
+        qvar = block_spread(Qh, cfg.block_q)
+        delta = scale * np.sqrt((qbar * qbar + qvar) @ block_spread(Kh, cfg.block_k).T)
         out.append((M, delta))
         print("head", h, flush=True)
     return out

@@ -37,12 +37,13 @@ error reduction is worth the extra compute at a single price.  Reading:
 4'. Predicted error of tile (i, j) under tier t: e_t = M_ij * eps_t, with eps
     the unit roundoff of the tier's arithmetic (bf16 2^-8; FP8 e4m3 2^-4;
     NVFP4 e2m1 2^-2; NVFP4 plus its residual 2^-4, the square of e2m1's) and,
-    for skip, eps_skip = delta_ij = scale * sqrt(sum_c qbar_ic^2 var_jc), where
-    var_jc is the variance of coordinate c over block j's keys (the mean of
-    (k_c - kbar_jc)^2): the spread of the pooled query's logits across the
-    block were the block's key coordinates uncorrelated, which is what
-    replacing the block by its means ignores (0 when the block's keys are
-    equal, and then skipping is exact).  Cost of tier t: its tensor-pipe time
+    for skip, eps_skip = delta_ij = scale * sqrt(sum_c (qbar_ic^2 + qvar_ic)
+    kvar_jc), where kvar_jc (qvar_ic) is the variance of coordinate c over key
+    block j's keys (query block i's queries), the mean of (x_c - xbar_c)^2:
+    the RMS over the tile's (query, key) pairs of how far a query's logit
+    moves from the one it has with the block's mean key, were the
+    coordinates uncorrelated; that is what replacing the block by its means
+    ignores (0 when the block's keys are equal, and then skipping is exact).  Cost of tier t: its tensor-pipe time
     relative to an NVFP4 tile at the nominal rates (skip 0, NVFP4 1, FP8 2,
     NVFP4 + residual 3, bf16 4).  The tile takes the tier of least
     e_t + price * cost_t among the tiers the low format provides; on a tie the
@@ -253,7 +254,8 @@ def route_head(Qh, Kh, Vh, tau, block_q: int, block_k: int, scale: float = 0.0,
     vbar, _ = pool_means(Vh, block_k)
     M = pooled_mass(qbar, kbar, n_k, scale)
     kvar = block_spread(Kh, block_k)
-    delta = scale * np.sqrt((qbar * qbar) @ kvar.T)
+    qvar = block_spread(Qh, block_q)
+    delta = scale * np.sqrt((qbar * qbar + qvar) @ kvar.T)
     nqb, nkb = M.shape
     tiers = np.empty((nqb, nkb), dtype=np.uint8)
     flags = np.empty((nqb, nkb), dtype=bool)
@@ -270,7 +272,7 @@ def route_head(Qh, Kh, Vh, tau, block_q: int, block_k: int, scale: float = 0.0,
             tiers[i], flags[i] = assign_tiers(M[i], tau, diag)
         counts[i], lists[i] = row_lists(tiers[i], M[i])
     return {"qbar": qbar, "kbar": kbar, "vbar": vbar, "n_k": n_k, "M": M,
-            "kvar": kvar, "delta": delta, "keep": keep,
+            "kvar": kvar, "qvar": qvar, "delta": delta, "keep": keep,
             "kbar_b": bf16_rne(kbar), "vbar_b": bf16_rne(vbar), "scale": scale,
             "tiers": tiers, "flags": flags, "counts": counts, "lists": lists}
 

@@ -47,7 +47,7 @@ _VIEW_FIELDS = [
     "status", "qbar", "kbar", "kbar_b", "vbar_b", "n_k", "logits", "mass", "tier_map",
     "row_counts", "row_lists", "q_codes", "k_codes", "v_codes", "q_scales", "k_scales",
     "v_scales", "rq_codes", "rk_codes", "rv_codes", "rq_scales", "rk_scales", "rv_scales",
-    "dq", "dk", "dv", "drq", "drk", "drv", "kvar", "spread",
+    "dq", "dk", "dv", "drq", "drk", "drv", "kvar", "spread", "qvar",
 ]
 
 
@@ -213,7 +213,7 @@ def plan_views(p: ta_params, ws: torch.Tensor) -> Dict[str, torch.Tensor]:
         "row_lists": (i32, (BH, nqb, nkb)),
         "dq": (b16, (BH, N, d)), "dk": (b16, (BH, N, d)), "dv": (b16, (BH, N, d)),
         "drq": (b16, (BH, N, d)), "drk": (b16, (BH, N, d)), "drv": (b16, (BH, N, d)),
-        "kvar": (f64, (BH, nkb, d)), "spread": (f64, (BH, nqb, nkb)),
+        "kvar": (f64, (BH, nkb, d)), "spread": (f64, (BH, nqb, nkb)), "qvar": (f64, (BH, nqb, d)),
     }
     if p.low == TA_LOW_FP8_E4M3:
         shapes.update({"q_codes": (u8, (BH, N, d)), "k_codes": (u8, (BH, N, d)),

@@ -86,7 +86,7 @@ bool native_fp8(const ta_params* p) {
 // Workspace layout: byte offsets of every array (kAbsent when not produced).
 struct Layout {
   size_t status, n_k, qbar, kbar, kbar_b, vbar_b, logits, mass, tier_map, row_counts, row_lists;
-  size_t kvar, spread;
+  size_t kvar, spread, qvar;
   size_t q_codes, k_codes, v_codes, q_scales, k_scales, v_scales;
   size_t rq_codes, rk_codes, rv_codes, rq_scales, rk_scales, rv_scales;
   size_t dq, dk, dv, drq, drk, drv;
@@ -117,6 +117,7 @@ Layout layout_of(const ta_params* p) {
   if (p->router == TA_ROUTER_PRICE) {
     L.kvar = take((size_t)s.BH * s.nKb * s.d * 8);
     L.spread = take((size_t)s.BH * s.nQb * s.nKb * 8);
+    L.qvar = take((size_t)s.BH * s.nQb * s.d * 8);
   }
   const size_t tok = (size_t)s.BH * s.N * s.d;  // elements of one [BH, N, d] tensor
   if (p->low == TA_LOW_FP8_E4M3) {
@@ -206,6 +207,7 @@ void fill_plan_args(const ta_params* p, const void* Q, const void* K, const void
   a.mass = at<double>(ws, L.mass);
   a.kvar = at<double>(ws, L.kvar);
   a.spread = at<double>(ws, L.spread);
+  a.qvar = at<double>(ws, L.qvar);
   a.tier_map = at<uint8_t>(ws, L.tier_map);
   a.row_counts = at<int>(ws, L.row_counts);
   a.row_lists = at<int>(ws, L.row_lists);
@@ -343,6 +345,7 @@ ta_status tiered_attn_plan_views(const ta_params* p, void* ws, ta_plan_views* ou
   out->drv = at<uint16_t>(ws, L.drv);
   out->kvar = at<double>(ws, L.kvar);
   out->spread = at<double>(ws, L.spread);
+  out->qvar = at<double>(ws, L.qvar);
   return TA_OK;
 }
 

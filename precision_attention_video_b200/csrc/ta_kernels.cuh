@@ -37,6 +37,7 @@ struct PlanArgs {
   double* logits;
   double* mass;
   double* kvar;                 // [BH, nKb, d] key-block coordinate variances (price router)
+  double* qvar;                 // [BH, nQb, d] query-block coordinate variances (price router)
   double* spread;               // [BH, nQb, nKb] skip error factor delta (price router)
   uint8_t* tier_map;
   int* row_counts;

@@ -8,7 +8,8 @@
 // exactly once and produces all of them:
 //   * fp64 block sums -> qbar (per query block), kbar (per key block), and the
 //     bf16 (round-to-nearest-even) kbar_b / vbar_b used by the skip tier;
-//     for the price router also each key block's coordinate variances;
+//     for the price router also each query and key block's coordinate
+//     variances;
 //   * FP8 e4m3: one power-of-two scale per tile (the smallest 2^k with
 //     amax <= 448 * 2^k), codes = e4m3_rn_satfinite(x * 2^-k);
 //   * NVFP4: per 16 elements along d (Q, K rows) or along tokens (V columns,
@@ -152,6 +153,15 @@ __global__ void __launch_bounds__(kThreads, 3) prep_kernel(const PlanArgs a) {
         const double mean = s / (double)(re - rs);
         if (which == 0) {
           a.qbar[((int64_t)bh * a.nQb + gb) * D + c] = mean;
+          if (a.qvar) {
+            // variance of coordinate c over the block's queries (second pass)
+            double ss = 0.0;
+            for (int r = rs; r < re; ++r) {
+              const double dv = (double)bf2f(tile[r * LD + c]) - mean;
+              ss += dv * dv;
+            }
+            a.qvar[((int64_t)bh * a.nQb + gb) * D + c] = ss / (double)(re - rs);
+          }
         } else if (which == 1) {
           a.kbar[((int64_t)bh * a.nKb + gb) * D + c] = mean;
           a.kbar_b[((int64_t)bh * a.nKb + gb) * D + c] = bf16_from_double(mean);

@@ -32,19 +32,21 @@ namespace {
 // ---------------------------------------------------------------------------
 // Pooled logits: logits[bh, i, j] = scale * sum_c qbar[bh, i, c] kbar[bh, j, c]
 // and, for the price router, the skip tier's error factor
-// spread[bh, i, j] = scale * sqrt(sum_c qbar[bh, i, c]^2 kvar[bh, j, c]).
+// spread[bh, i, j] = scale * sqrt(sum_c (qbar[bh, i, c]^2 + qvar[bh, i, c]) kvar[bh, j, c]).
 // 32 x 32 output tile per CTA, 2 x 2 per thread, d staged 32 at a time.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) logits_kernel(const PlanArgs a) {
   __shared__ double qs[32][33];
   __shared__ double ks[32][33];
   __shared__ double vs[32][33];
+  __shared__ double qw[32][33];   // qbar^2 + qvar (price router)
   const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
   const int bh = blockIdx.z, i0 = blockIdx.x * 32, j0 = blockIdx.y * 32;
   const int D = a.d;
   const double* qb = a.qbar + (int64_t)bh * a.nQb * D;
   const double* kb = a.kbar + (int64_t)bh * a.nKb * D;
   const double* kvb = a.kvar ? a.kvar + (int64_t)bh * a.nKb * D : nullptr;
+  const double* qvb = a.qvar ? a.qvar + (int64_t)bh * a.nQb * D : nullptr;
   double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
   double spr[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
   for (int c0 = 0; c0 < D; c0 += 32) {
@@ -52,7 +54,10 @@ __global__ void __launch_bounds__(256) logits_kernel(const PlanArgs a) {
       const int r = e / 32, c = e % 32;
       qs[r][c] = (i0 + r < a.nQb) ? qb[(int64_t)(i0 + r) * D + c0 + c] : 0.0;
       ks[r][c] = (j0 + r < a.nKb) ? kb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
-      if (kvb) vs[r][c] = (j0 + r < a.nKb) ? kvb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
+      if (kvb) {
+        vs[r][c] = (j0 + r < a.nKb) ? kvb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
+        qw[r][c] = (i0 + r < a.nQb) ? qs[r][c] * qs[r][c] + qvb[(int64_t)(i0 + r) * D + c0 + c] : 0.0;
+      }
     }
     __syncthreads();
 #pragma unroll 8
@@ -67,12 +72,12 @@ __global__ void __launch_bounds__(256) logits_kernel(const PlanArgs a) {
     if (kvb) {
 #pragma unroll 8
       for (int c = 0; c < 32; ++c) {
-        const double q0 = qs[ty * 2][c], q1 = qs[ty * 2 + 1][c];
+        const double w0 = qw[ty * 2][c], w1 = qw[ty * 2 + 1][c];
         const double v0 = vs[tx * 2][c], v1 = vs[tx * 2 + 1][c];
-        spr[0][0] += q0 * q0 * v0;
-        spr[0][1] += q0 * q0 * v1;
-        spr[1][0] += q1 * q1 * v0;
-        spr[1][1] += q1 * q1 * v1;
+        spr[0][0] += w0 * v0;
+        spr[0][1] += w0 * v1;
+        spr[1][0] += w1 * v0;
+        spr[1][1] += w1 * v1;
       }
     }
     __syncthreads();

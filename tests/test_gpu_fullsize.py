@@ -40,6 +40,7 @@ def _check_head(cfg, Q, K, V, views, O, h, qblocks):
     rt = Rt.route_head(Qh, Kh, Vh, cfg.tau, cfg.block_q, cfg.block_k, **router_kwargs(cfg))
     if getattr(cfg, "router", 0) == Rt.ROUTER_PRICE:
         np.testing.assert_allclose(views["kvar"][h].cpu().numpy(), rt["kvar"], rtol=1e-12, atol=0)
+        np.testing.assert_allclose(views["qvar"][h].cpu().numpy(), rt["qvar"], rtol=1e-12, atol=0)
         np.testing.assert_allclose(views["spread"][h].cpu().numpy(), rt["delta"], rtol=1e-12, atol=0)
     tiers = views["tier_map"][h].cpu().numpy()
     _, rows = compare_tiers(tiers, rt)

@@ -38,19 +38,22 @@ def test_block_spread_closed_form():
     assert (R.block_spread(np.concatenate([X, base[:1]]), blk)[-1] == 0.0).all()
 
 
-def test_delta_is_the_logit_spread_when_key_coordinates_are_independent():
-    # keys with independent +-a_c signs per coordinate: the variance of q . k
-    # over the block is exactly sum_c q_c^2 a_c^2, the router's delta^2 / scale^2
+def test_delta_is_the_rms_logit_spread_when_key_coordinates_are_independent():
+    # keys with independent +-a_c signs per coordinate (all 2^d patterns): for
+    # each query q the variance of q . k over the block is exactly
+    # sum_c q_c^2 a_c^2, so the mean over the block's queries is
+    # sum_c (qbar_c^2 + qvar_c) a_c^2, the router's delta^2 / scale^2
     rng = np.random.default_rng(9)
     d, blk = 8, 256
     a = rng.uniform(0.1, 1.0, size=d)
     signs = np.array([[1 if (r >> c) & 1 else -1 for c in range(d)] for r in range(blk)])
     Kb = signs * a
-    Q = rng.normal(size=(blk, d))
+    Q = rng.normal(size=(blk, d)) + 0.5
     rt = R.route_head(Q, Kb, Kb, None, blk, blk, router=R.ROUTER_PRICE, price=0.0,
                       low=Qz.LOW_NVFP4, keep_diag_full=False)
-    logits = Kb @ rt["qbar"][0] * rt["scale"]
-    assert abs(rt["delta"][0, 0] - logits.std()) <= 1e-12 * logits.std()
+    per_query_var = ((Q @ Kb.T) * rt["scale"]).var(axis=1)
+    want = np.sqrt(per_query_var.mean())
+    assert abs(rt["delta"][0, 0] - want) <= 1e-12 * want
 
 
 def _blocky(N, d, bk, seed):
@@ -71,7 +74,7 @@ def test_equal_keys_are_skipped_and_skip_is_exact(N, bq, bk, d, price):
     Q, K, V = _blocky(N, d, bk, seed=N + d)
     low = Qz.LOW_NVFP4_RES
     rt = R.route_head(Q, K, V, None, bq, bk, router=R.ROUTER_PRICE, price=price, low=low)
-    assert (rt["kvar"] == 0.0).all()
+    assert (rt["kvar"] == 0.0).all() and (rt["delta"] == 0.0).all()
     for i in range(rt["tiers"].shape[0]):
         diag = set(R.diag_blocks(i, bq, bk, N))
         for j in range(rt["tiers"].shape[1]):
