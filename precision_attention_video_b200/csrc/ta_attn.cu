@@ -157,8 +157,17 @@ __device__ __forceinline__ bool softmax_tail(const SoftmaxTail q, float& psum) {
   constexpr bool smem_p = (PK == PK_FP4 || PK == PK_RES || PK == PK_F8);
   const int s = q.t & 1;
   float* x = q.x;
+  {
+    // arguments two at a time (packed fp32 FMA), then the exponentials
+    const uint64_t c2t2 = pack2(q.c2t, q.c2t), nmc2 = pack2(-q.mc, -q.mc);
 #pragma unroll
-  for (int c = 0; c < HB; ++c) x[c] = fast_exp2(fmaf(x[c], q.c2t, -q.mc));
+    for (int c = 0; c < HB; c += 2) {
+      float a0, a1;
+      unpack2(fma2(pack2(x[c], x[c + 1]), c2t2, nmc2), a0, a1);
+      x[c] = fast_exp2(a0);
+      x[c + 1] = fast_exp2(a1);
+    }
+  }
   if constexpr (PK == PK_SKIP) {
     // pooled keys weigh n_j
 #pragma unroll
@@ -169,10 +178,19 @@ __device__ __forceinline__ bool softmax_tail(const SoftmaxTail q, float& psum) {
       }
     }
   }
-  float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  {
+    // four running sums (keys c = 0, 1, 2, 3 mod 4) as two packed pairs
+    uint64_t sa = pack2(0.0f, 0.0f), sb = pack2(0.0f, 0.0f);
 #pragma unroll
-  for (int c = 0; c < HB; ++c) ps[c & 3] += x[c];
-  psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+    for (int c = 0; c < HB; c += 4) {
+      sa = add2(sa, pack2(x[c], x[c + 1]));
+      sb = add2(sb, pack2(x[c + 2], x[c + 3]));
+    }
+    float s0, s1, s2, s3;
+    unpack2(sa, s0, s1);
+    unpack2(sb, s2, s3);
+    psum = (s0 + s1) + (s2 + s3);
+  }
 
   // round P' as the tier demands
   uint32_t p[(PK == PK_RES) ? 13 : (HB / 2)];
@@ -218,8 +236,14 @@ __device__ __forceinline__ bool softmax_tail(const SoftmaxTail q, float& psum) {
     for (int c0 = 0; c0 < HD; c0 += 32) {
       uint32_t raw[32];
       tmem_ld32(q.tO + q.part * HD + c0, raw);
+      const uint64_t al2 = pack2(q.alpha, q.alpha);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) raw[c] = __float_as_uint(__uint_as_float(raw[c]) * q.alpha);
+      for (int c = 0; c < 32; c += 2) {
+        float o0, o1;
+        unpack2(mul2(pack2(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), al2), o0, o1);
+        raw[c] = __float_as_uint(o0);
+        raw[c + 1] = __float_as_uint(o1);
+      }
       tmem_st32(q.tO + q.part * HD + c0, raw);
     }
   }
@@ -803,9 +827,13 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           uint32_t raw[32];
           tmem_ld32(tO + lane_off + part * HD + c0, raw);
           uint32_t w[16];
+          const uint64_t il2 = pack2(inv_l, inv_l);
 #pragma unroll
-          for (int c = 0; c < 32; c += 2)
-            w[c / 2] = pack_bf16(__uint_as_float(raw[c]) * inv_l, __uint_as_float(raw[c + 1]) * inv_l);
+          for (int c = 0; c < 32; c += 2) {
+            float o0, o1;
+            unpack2(mul2(pack2(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1])), il2), o0, o1);
+            w[c / 2] = pack_bf16(o0, o1);
+          }
           if (valid) {
 #pragma unroll
             for (int v = 0; v < 4; ++v)

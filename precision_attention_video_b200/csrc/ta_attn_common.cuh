@@ -38,6 +38,32 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Pairs of fp32 values in one 64-bit register and the packed fp32x2
+// arithmetic of sm_100: each lane is rounded exactly as the scalar form.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -137,11 +163,13 @@ __device__ __forceinline__ uint32_t nvfp4_quant32(const float* x, const float2* 
     const uint32_t scc = cvt_e4m3x2(div6(amax), 0.0f) & 0xFFu;
     const float inv = sc_tab[scc].y;
     scw |= scc << (8 * g);
+    const uint64_t inv2 = pack2(inv, inv);
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
       float y[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(x[g * 16 + w * 8 + i], inv);
+      for (int i = 0; i < 8; i += 2)
+        unpack2(mul2(pack2(x[g * 16 + w * 8 + i], x[g * 16 + w * 8 + i + 1]), inv2), y[i], y[i + 1]);
       p[g * 2 + w] = cvt_e2m1x8(y);
     }
   }
