@@ -185,6 +185,10 @@ __device__ __forceinline__ uint32_t nvfp4_residual32(const float* x, const uint3
 #pragma unroll
   for (int g = 0; g < 2; ++g) {
     const float sc1 = sc_tab[(scw >> (8 * g)) & 0xFFu].x;
+    // x - code * sc1 in one rounding: code * sc1 is exact in fp32 (at most
+    // 2 + 4 significant bits), so a fused multiply-add rounds like the
+    // subtraction of that exact product
+    const uint64_t nsc1 = pack2(-sc1, -sc1);
     float rr[16];
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
@@ -192,8 +196,7 @@ __device__ __forceinline__ uint32_t nvfp4_residual32(const float* x, const uint3
       for (int bb = 0; bb < 4; ++bb) {
         const float2 f = __half22float2(e2m1x2_to_half2(p[g * 2 + w] >> (8 * bb)));
         const int c = w * 8 + 2 * bb;
-        rr[c] = __fsub_rn(x[g * 16 + c], __fmul_rn(f.x, sc1));
-        rr[c + 1] = __fsub_rn(x[g * 16 + c + 1], __fmul_rn(f.y, sc1));
+        unpack2(fma2(pack2(f.x, f.y), nsc1, pack2(x[g * 16 + c], x[g * 16 + c + 1])), rr[c], rr[c + 1]);
       }
     }
     float am = 0.0f;
@@ -202,11 +205,13 @@ __device__ __forceinline__ uint32_t nvfp4_residual32(const float* x, const uint3
     const uint32_t scc2 = cvt_e4m3x2(div6(am), 0.0f) & 0xFFu;
     const float inv2 = sc_tab[scc2].y;
     scw2 |= scc2 << (8 * g);
+    const uint64_t inv22 = pack2(inv2, inv2);
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
       float y[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(rr[w * 8 + i], inv2);
+      for (int i = 0; i < 8; i += 2)
+        unpack2(mul2(pack2(rr[w * 8 + i], rr[w * 8 + i + 1]), inv22), y[i], y[i + 1]);
       p2[g * 2 + w] = cvt_e2m1x8(y);
     }
   }
