@@ -30,7 +30,17 @@ namespace {
 
 constexpr int kThreads = 256;
 
-__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+// The two bf16 values of a 32-bit word as fp32 (exact), element 0 in the low half.
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// 16 bytes global -> shared without a register round trip; src_bytes = 0
+// writes zeros (and reads nothing).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
 
 // Smallest power of two s with amax <= 448 s (1 when amax == 0).
 __device__ __forceinline__ float fp8_pow2_scale(float amax) {
@@ -41,306 +51,333 @@ __device__ __forceinline__ float fp8_pow2_scale(float amax) {
   return ldexpf(1.0f, k);
 }
 
-// NVFP4 of one group of 16 values: packed codes (element 2i in the low nibble
-// of byte i) and the ue4m3 scale code; the scale value comes back in `sc`.
-// `inv_tab[c]` is the correctly rounded reciprocal of ue4m3 code c's value.
-__device__ __forceinline__ void nvfp4_group(const float (&x)[16], uint32_t (&packed)[2],
-                                            uint32_t& sc_code, float& sc, const float* inv_tab) {
-  float amax = 0.0f;
+// NVFP4 of one group of 16 values: returns the ue4m3 scale code
+// sc = e4m3_rn(amax / 6); the codes e2m1_rn_satfinite(x * rcp_rn(sc)) go to
+// `packed`, element i in nibble i (a zero scale gives zero codes).
+// `tab[c]` = (value, correctly rounded 1 / value) of ue4m3 code c.
+__device__ __forceinline__ uint32_t nvfp4_group(const float (&x)[16], uint32_t (&packed)[2],
+                                                const float2* tab) {
+  float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
-  sc_code = cvt_e4m3x2(div6(amax), 0.0f) & 0xFFu;
-  sc = e4m3_to_float(sc_code);
-  packed[0] = packed[1] = 0u;
-  if (sc == 0.0f) return;
-  const float inv = inv_tab[sc_code];
+  for (int i = 0; i < 16; ++i) am[i & 3] = fmaxf(am[i & 3], fabsf(x[i]));
+  const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
+  const uint32_t scc = cvt_e4m3x2(div6(amax), 0.0f) & 0xFFu;
+  const float inv = tab[scc].y;
+  const uint64_t inv2 = pack2(inv, inv);
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2)
+      unpack2(mul2(pack2(x[w * 8 + i], x[w * 8 + i + 1]), inv2), y[i], y[i + 1]);
+    const uint32_t c = cvt_e2m1x8(y);
+    packed[w] = scc ? c : 0u;
+  }
+  return scc;
+}
+
+// The residual of a quantised group, r = fp32(x - code * sc).  code * sc is
+// exact in fp32 (at most 2 + 4 significant bits), so one fused multiply-add
+// per pair rounds like the subtraction of that exact product.
+__device__ __forceinline__ void nvfp4_residual(const float (&x)[16], const uint32_t (&packed)[2],
+                                               float sc, float (&r)[16]) {
+  const uint64_t nsc = pack2(-sc, -sc);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t c = cvt_e2m1x2(__fmul_rn(x[2 * i], inv), __fmul_rn(x[2 * i + 1], inv));
-    packed[i >> 2] |= c << (8 * (i & 3));
+    const float2 f = __half22float2(e2m1x2_to_half2(packed[i >> 2] >> (8 * (i & 3))));
+    unpack2(fma2(pack2(f.x, f.y), nsc, pack2(x[2 * i], x[2 * i + 1])), r[2 * i], r[2 * i + 1]);
   }
 }
 
-// The values a packed group stands for: code value times the scale (exact in
-// fp32: at most 3 + 4 significant bits).
-__device__ __forceinline__ void nvfp4_dequant(const uint32_t (&packed)[2], float sc,
-                                              float (&deq)[16]) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t c = (packed[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-    deq[2 * i] = e2m1_value(c & 0xFu) * sc;
-    deq[2 * i + 1] = e2m1_value(c >> 4) * sc;
-  }
-}
+// Shared memory of one CTA: the staged chunk [R][D] bf16, then a region that
+// first holds the partial column sums (fp64) and maxima (fp32) [SEG][D] and
+// later the V codes in transit [2 copies][R / 16][D + 2] uint2, then the FP8
+// tile scales.
+template <int D, int R>
+struct PrepSmem {
+  static constexpr int CP = D / 2;            // column pairs
+  static constexpr int SEG = kThreads / CP;   // row segments of the column sums
+  static constexpr int RS = R / SEG;          // rows per segment
+  static constexpr int G = R / 16;            // 16-token groups of a V column
+  static constexpr int VP = D + 2;            // uint2 pitch of a group's V codes
+  static constexpr size_t oTile = 0;
+  static constexpr size_t oPsum = oTile + (size_t)R * D * 2;
+  static constexpr size_t oRed = oPsum + (size_t)SEG * D * 8;
+  static constexpr size_t oVst = oPsum;
+  static constexpr size_t kSums = (size_t)SEG * D * 12, kVst = (size_t)2 * G * VP * 8;
+  static constexpr size_t oScale = oPsum + (kSums > kVst ? kSums : kVst);
+  static constexpr size_t kBytes = oScale + 8 * sizeof(float);
+  static_assert(kThreads % CP == 0 && R % SEG == 0 && 64 % RS == 0,
+                "a row segment must lie inside one block");
+};
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 3) prep_kernel(const PlanArgs a) {
+template <int D, int R>
+__global__ void __launch_bounds__(kThreads, 4) prep_kernel(const PlanArgs a) {
+  using L = PrepSmem<D, R>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  constexpr int LD = D + 8;  // padded row stride (elements)
-  const int R = a.R;
-  __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(smem_raw);
-  __nv_bfloat16* rtile = tile + R * LD;  // staging of the transposed NVFP4 V codes
-  float* red = reinterpret_cast<float*>(rtile + R * LD);
-  float* tile_scale = red + kThreads;
+  __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(smem_raw + L::oTile);
+  const uint32_t* tile32 = reinterpret_cast<const uint32_t*>(tile);
+  double* psum = reinterpret_cast<double*>(smem_raw + L::oPsum);
+  float* red = reinterpret_cast<float*>(smem_raw + L::oRed);
+  uint2* vst = reinterpret_cast<uint2*>(smem_raw + L::oVst);
+  float* tile_scale = reinterpret_cast<float*>(smem_raw + L::oScale);
 
-  __shared__ float inv_tab[128];   // ue4m3 code -> correctly rounded 1 / value
+  __shared__ float2 sc_tab[128];   // ue4m3 code -> (value, correctly rounded 1 / value)
   const int tid = threadIdx.x;
   if (tid < 128) {
     const float v = (tid == 0x7F) ? 0.0f : e4m3_to_float(tid);
-    inv_tab[tid] = v > 0.0f ? __frcp_rn(v) : 0.0f;
+    sc_tab[tid] = make_float2(v, v > 0.0f ? __frcp_rn(v) : 0.0f);
   }
+  const int which = blockIdx.z;
   const int bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
   const int r0 = blockIdx.x * R;
   const int nrows = min(R, a.N - r0);
-  const int64_t in_off = (int64_t)b * a.sb + (int64_t)h * a.sh;
   const int64_t bhN = (int64_t)bh * a.N;
-  double* psum = reinterpret_cast<double*>(tile_scale + 8);   // [kThreads] partial block sums
+  const __nv_bfloat16* src =
+      (which == 0 ? a.Q : which == 1 ? a.K : a.V) + (int64_t)b * a.sb + (int64_t)h * a.sh;
 
+  // ---- stage the chunk; rows past N are zeros ----
+  for (int idx = tid; idx < R * (D / 8); idx += kThreads) {
+    const int r = idx / (D / 8), c8 = idx % (D / 8);
+    const bool in = r < nrows;
+    cp_async16(tile + r * D + c8 * 8, src + (int64_t)(r0 + (in ? r : 0)) * a.sn + c8 * 8,
+               in ? 16u : 0u);
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+
+  // ---- block sums in fp64 and column maxima.  A sum of bf16 values is exact
+  // in fp64 while a block's values span at most 38 binades (53 - 8 - 7 bits),
+  // and then the order of the additions does not matter.  Each thread takes
+  // two adjacent columns over one segment of RS rows (zero rows add nothing) ----
+  const int blk = (which == 0) ? a.bq : a.bk;
+  const int nb = R / blk;
   {
-    const int which = blockIdx.z;
-    const __nv_bfloat16* src = (which == 0 ? a.Q : which == 1 ? a.K : a.V) + in_off;
-    // ---- stage the chunk (rows past N read as zero) ----
-    for (int idx = tid; idx < R * (D / 8); idx += kThreads) {
-      const int r = idx / (D / 8), c8 = idx % (D / 8);
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < nrows) v = *reinterpret_cast<const uint4*>(src + (int64_t)(r0 + r) * a.sn + c8 * 8);
-      *reinterpret_cast<uint4*>(tile + r * LD + c8 * 8) = v;
+    const int cp = tid % L::CP, seg = tid / L::CP;
+    const uint32_t* col = tile32 + seg * L::RS * L::CP + cp;
+    double s0 = 0.0, s1 = 0.0;
+    float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll 8
+    for (int r = 0; r < L::RS; ++r) {
+      const uint32_t w = col[r * L::CP];
+      const float lo = bf_lo(w), hi = bf_hi(w);
+      s0 += (double)lo;
+      s1 += (double)hi;
+      m0 = fmaxf(m0, fabsf(lo));
+      m1 = fmaxf(m1, fabsf(hi));
     }
-    __syncthreads();
+    *reinterpret_cast<double2*>(psum + seg * D + 2 * cp) = make_double2(s0, s1);
+    *reinterpret_cast<float2*>(red + seg * D + 2 * cp) = make_float2(m0, m1);
+  }
+  __syncthreads();
+  // nb * D <= 256 = kThreads: one (block, column) per thread
+  const bool mine = tid < nb * D;
+  double s = 0.0;
+  float amax_c = 0.0f;
+  if (mine) {
+    const int jb = tid / D, c = tid % D;
+    const int spb = L::SEG / nb;   // segments per block
+    for (int k = 0; k < spb; ++k) {
+      s += psum[(jb * spb + k) * D + c];
+      amax_c = fmaxf(amax_c, red[(jb * spb + k) * D + c]);
+    }
+  }
+  __syncthreads();
+  if (mine) {
+    const int w = tid;
+    const int jb = w / D, c = w % D;
+    const int rs = jb * blk, re = min(rs + blk, nrows);
+    red[w] = amax_c;
+    if (re > rs) {
+      const int gb = r0 / blk + jb;
+      const double mean = s / (double)(re - rs);
+      if (which == 0) {
+        a.qbar[((int64_t)bh * a.nQb + gb) * D + c] = mean;
+        if (a.qvar) {
+          // variance of coordinate c over the block's queries (second pass)
+          double ss = 0.0;
+          for (int r = rs; r < re; ++r) {
+            const double dv = (double)__bfloat162float(tile[r * D + c]) - mean;
+            ss += dv * dv;
+          }
+          a.qvar[((int64_t)bh * a.nQb + gb) * D + c] = ss / (double)(re - rs);
+        }
+      } else if (which == 1) {
+        a.kbar[((int64_t)bh * a.nKb + gb) * D + c] = mean;
+        a.kbar_b[((int64_t)bh * a.nKb + gb) * D + c] = bf16_from_double(mean);
+        if (bh == 0 && c == 0) a.n_k[gb] = re - rs;
+        if (a.kvar) {
+          // variance of coordinate c over the block's keys (second pass over
+          // the staged rows, deviations from the fp64 mean)
+          double ss = 0.0;
+          for (int r = rs; r < re; ++r) {
+            const double dv = (double)__bfloat162float(tile[r * D + c]) - mean;
+            ss += dv * dv;
+          }
+          a.kvar[((int64_t)bh * a.nKb + gb) * D + c] = ss / (double)(re - rs);
+        }
+      } else {
+        a.vbar_b[((int64_t)bh * a.nKb + gb) * D + c] = bf16_from_double(mean);
+      }
+    }
+  }
+  __syncthreads();
+  if (a.low == TA_LOW_NONE) return;
 
-    // ---- block sums (fp64: exact for bf16 inputs, so the order of the
-    // additions does not matter) and per-column amax; kSeg threads share a
-    // (block, column) and each sums a run of its rows ----
-    const int blk = (which == 0) ? a.bq : a.bk;
-    const int nb = R / blk;
-    const int kSeg = kThreads / (nb * D) > 0 ? kThreads / (nb * D) : 1;
-    for (int w0 = tid; w0 < nb * D * kSeg; w0 += kThreads) {
-      const int w = w0 % (nb * D), seg = w0 / (nb * D);
-      const int jb = w / D, c = w % D;
-      const int rs = jb * blk, re = min(rs + blk, nrows);
-      const int len = (blk + kSeg - 1) / kSeg;
-      const int s0 = rs + seg * len, s1 = min(s0 + len, re);
-      double sum = 0.0;
+  uint8_t* codes = which == 0 ? a.q_codes : which == 1 ? a.k_codes : a.v_codes;
+  __nv_bfloat16* deq_out = which == 0 ? a.dq : which == 1 ? a.dk : a.dv;
+
+  if (a.low == TA_LOW_FP8_E4M3) {
+    // ---- FP8: one power-of-two scale per tile of `blk` rows ----
+    if (tid < nb) {
       float amax = 0.0f;
-      for (int r = s0; r < s1; ++r) {
-        const float x = bf2f(tile[r * LD + c]);
-        sum += (double)x;
-        amax = fmaxf(amax, fabsf(x));
-      }
-      psum[w0] = sum;
-      red[w0] = amax;
-    }
-    __syncthreads();
-    // nb * D <= 256 = kThreads: one (block, column) per thread
-    const bool mine = tid < nb * D;
-    double s = 0.0;
-    float amax_c = 0.0f;
-    if (mine) {
-      for (int seg = 0; seg < kSeg; ++seg) {
-        s += psum[seg * nb * D + tid];
-        amax_c = fmaxf(amax_c, red[seg * nb * D + tid]);
+      for (int c = 0; c < D; ++c) amax = fmaxf(amax, red[tid * D + c]);
+      const float sc = fp8_pow2_scale(amax);
+      tile_scale[tid] = sc;
+      const int gb = r0 / blk + tid;
+      if (tid * blk < nrows) {
+        float* scp = reinterpret_cast<float*>(which == 0 ? a.q_scales
+                                              : which == 1 ? a.k_scales
+                                                           : a.v_scales);
+        scp[(int64_t)bh * (which == 0 ? a.nQb : a.nKb) + gb] = sc;
       }
     }
     __syncthreads();
-    if (mine) {
-      const int w = tid;
-      const int jb = w / D, c = w % D;
-      const int rs = jb * blk, re = min(rs + blk, nrows);
-      red[w] = amax_c;
-      if (re > rs) {
-        const int gb = r0 / blk + jb;
-        const double mean = s / (double)(re - rs);
-        if (which == 0) {
-          a.qbar[((int64_t)bh * a.nQb + gb) * D + c] = mean;
-          if (a.qvar) {
-            // variance of coordinate c over the block's queries (second pass)
-            double ss = 0.0;
-            for (int r = rs; r < re; ++r) {
-              const double dv = (double)bf2f(tile[r * LD + c]) - mean;
-              ss += dv * dv;
-            }
-            a.qvar[((int64_t)bh * a.nQb + gb) * D + c] = ss / (double)(re - rs);
-          }
-        } else if (which == 1) {
-          a.kbar[((int64_t)bh * a.nKb + gb) * D + c] = mean;
-          a.kbar_b[((int64_t)bh * a.nKb + gb) * D + c] = bf16_from_double(mean);
-          if (bh == 0 && c == 0) a.n_k[gb] = re - rs;
-          if (a.kvar) {
-            // variance of coordinate c over the block's keys (second pass
-            // over the staged rows, deviations from the fp64 mean)
-            double ss = 0.0;
-            for (int r = rs; r < re; ++r) {
-              const double dv = (double)bf2f(tile[r * LD + c]) - mean;
-              ss += dv * dv;
-            }
-            a.kvar[((int64_t)bh * a.nKb + gb) * D + c] = ss / (double)(re - rs);
-          }
-        } else {
-          a.vbar_b[((int64_t)bh * a.nKb + gb) * D + c] = bf16_from_double(mean);
-        }
+    for (int idx = tid; idx < R * (D / 16); idx += kThreads) {
+      const int r = idx / (D / 16), g = idx % (D / 16);
+      if (r >= nrows) continue;
+      const float sc = tile_scale[r / blk];
+      const float inv = 1.0f / sc;  // exact: sc is a power of two
+      __nv_bfloat16* px = tile + r * D + g * 16;
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t c2 = cvt_e4m3x2(__bfloat162float(px[2 * i]) * inv,
+                                       __bfloat162float(px[2 * i + 1]) * inv);
+        if (i & 1)
+          w[i >> 1] |= c2 << 16;
+        else
+          w[i >> 1] = c2;
+        const float2 f = e4m3x2_to_float2(c2);
+        px[2 * i] = __float2bfloat16_rn(f.x * sc);
+        px[2 * i + 1] = __float2bfloat16_rn(f.y * sc);
       }
+      *reinterpret_cast<uint4*>(codes + (bhN + r0 + r) * D + g * 16) =
+          make_uint4(w[0], w[1], w[2], w[3]);
     }
-    __syncthreads();
-    if (a.low == TA_LOW_NONE) return;
-
-    uint8_t* codes = which == 0 ? a.q_codes : which == 1 ? a.k_codes : a.v_codes;
-    __nv_bfloat16* deq_out = which == 0 ? a.dq : which == 1 ? a.dk : a.dv;
-
-    if (a.low == TA_LOW_FP8_E4M3) {
-      // ---- FP8: one power-of-two scale per tile of `blk` rows ----
-      if (tid < nb) {
-        float amax = 0.0f;
-        for (int c = 0; c < D; ++c) amax = fmaxf(amax, red[tid * D + c]);
-        const float s = fp8_pow2_scale(amax);
-        tile_scale[tid] = s;
-        const int gb = r0 / blk + tid;
-        if (tid * blk < nrows) {
-          float* sc = reinterpret_cast<float*>(which == 0 ? a.q_scales
-                                               : which == 1 ? a.k_scales
-                                                            : a.v_scales);
-          sc[(int64_t)bh * (which == 0 ? a.nQb : a.nKb) + gb] = s;
-        }
-      }
-      __syncthreads();
+  } else {
+    // ---- NVFP4 (+ residual); no bf16 images of these copies are kept ----
+    const bool res = (a.low == TA_LOW_NVFP4_RES);
+    uint8_t* rcodes = which == 0 ? a.rq_codes : which == 1 ? a.rk_codes : a.rv_codes;
+    uint8_t* scales = reinterpret_cast<uint8_t*>(which == 0 ? a.q_scales
+                                                 : which == 1 ? a.k_scales
+                                                              : a.v_scales);
+    uint8_t* rscales = which == 0 ? a.rq_scales : which == 1 ? a.rk_scales : a.rv_scales;
+    if (which < 2) {
+      // groups of 16 along d; codes [BH, N, D/2], scales [BH, N, D/16]
       for (int idx = tid; idx < R * (D / 16); idx += kThreads) {
         const int r = idx / (D / 16), g = idx % (D / 16);
         if (r >= nrows) continue;
-        const float s = tile_scale[r / blk];
-        const float inv = 1.0f / s;  // exact: s is a power of two
-        __nv_bfloat16* px = tile + r * LD + g * 16;
-        uint32_t w[4];
+        const uint4* pv = reinterpret_cast<const uint4*>(tile + r * D + g * 16);
+        float x[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t c2 = cvt_e4m3x2(bf2f(px[2 * i]) * inv, bf2f(px[2 * i + 1]) * inv);
-          if (i & 1)
-            w[i >> 1] |= c2 << 16;
-          else
-            w[i >> 1] = c2;
-          const float2 f = e4m3x2_to_float2(c2);
-          px[2 * i] = __float2bfloat16_rn(f.x * s);
-          px[2 * i + 1] = __float2bfloat16_rn(f.y * s);
+        for (int v = 0; v < 2; ++v) {
+          const uint4 q = pv[v];
+          const uint32_t ws[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            x[v * 8 + e * 2] = bf_lo(ws[e]);
+            x[v * 8 + e * 2 + 1] = bf_hi(ws[e]);
+          }
         }
-        *reinterpret_cast<uint4*>(codes + (bhN + r0 + r) * D + g * 16) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+        uint32_t pk[2];
+        const uint32_t scc = nvfp4_group(x, pk, sc_tab);
+        const int64_t row = bhN + r0 + r;
+        *reinterpret_cast<uint2*>(codes + row * (D / 2) + g * 8) = make_uint2(pk[0], pk[1]);
+        scales[row * (D / 16) + g] = (uint8_t)scc;
+        if (res) {
+          float rr[16];
+          nvfp4_residual(x, pk, sc_tab[scc].x, rr);
+          const uint32_t scc2 = nvfp4_group(rr, pk, sc_tab);
+          *reinterpret_cast<uint2*>(rcodes + row * (D / 2) + g * 8) = make_uint2(pk[0], pk[1]);
+          rscales[row * (D / 16) + g] = (uint8_t)scc2;
+        }
       }
     } else {
-      // ---- NVFP4 (+ residual); no bf16 images of these copies are kept ----
-      const bool res = (a.low == TA_LOW_NVFP4_RES);
-      uint8_t* rcodes = which == 0 ? a.rq_codes : which == 1 ? a.rk_codes : a.rv_codes;
-      uint8_t* scales = reinterpret_cast<uint8_t*>(which == 0 ? a.q_scales
-                                                   : which == 1 ? a.k_scales
-                                                                : a.v_scales);
-      uint8_t* rscales = which == 0 ? a.rq_scales : which == 1 ? a.rk_scales : a.rv_scales;
-      if (which < 2) {
-        // groups of 16 along d; codes [BH, N, D/2], scales [BH, N, D/16]
-        for (int idx = tid; idx < R * (D / 16); idx += kThreads) {
-          const int r = idx / (D / 16), g = idx % (D / 16);
-          if (r >= nrows) continue;
-          const uint4* pv = reinterpret_cast<const uint4*>(tile + r * LD + g * 16);
-          float x[16], dqv[16], sc;
-          uint32_t pk[2], scc;
+      // V: groups of 16 tokens per column; codes [BH, D, Np/2] (transposed),
+      // scales [BH, Np/16, D].  A thread takes two adjacent columns of one
+      // group (a warp reads 128 contiguous bytes of a staged row per token);
+      // the codes go to shared memory group-major and leave 64 bytes per
+      // column.  Groups past N come out as zero codes with a zero scale, up to
+      // the pitch Np.
+      for (int idx = tid; idx < L::CP * L::G; idx += kThreads) {
+        const int cp = idx % L::CP, g = idx / L::CP;
+        if (r0 + g * 16 >= a.Np) continue;
+        float x0[16], x1[16];
 #pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const uint4 w = pv[v];
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              x[v * 8 + e * 2] = __uint_as_float(ws[e] << 16);
-              x[v * 8 + e * 2 + 1] = __uint_as_float(ws[e] & 0xFFFF0000u);
-            }
-          }
-          nvfp4_group(x, pk, scc, sc, inv_tab);
-          const int64_t row = bhN + r0 + r;
-          *reinterpret_cast<uint2*>(codes + row * (D / 2) + g * 8) = make_uint2(pk[0], pk[1]);
-          scales[row * (D / 16) + g] = (uint8_t)scc;
-          if (res) {
-            float rr[16], rsc;
-            nvfp4_dequant(pk, sc, dqv);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) rr[i] = __fsub_rn(x[i], dqv[i]);
-            nvfp4_group(rr, pk, scc, rsc, inv_tab);
-            *reinterpret_cast<uint2*>(rcodes + row * (D / 2) + g * 8) = make_uint2(pk[0], pk[1]);
-            rscales[row * (D / 16) + g] = (uint8_t)scc;
-          }
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t w = tile32[(g * 16 + i) * L::CP + cp];
+          x0[i] = bf_lo(w);
+          x1[i] = bf_hi(w);
         }
-      } else {
-        // V: groups of 16 tokens per column; codes [BH, D, Np/2] (transposed),
-        // scales [BH, Np/16, D].  Threads walk the columns fastest, so that a
-        // warp reads one 64-byte run of a staged row at a time (no bank
-        // conflicts); the codes go column-major to shared memory (the residual
-        // tile area, unused here; group-major with a padded row of D + 1, so
-        // that both the writes here and the reads below avoid bank conflicts)
-        // and leave 64 bytes per column.  Groups past
-        // N come out as zero codes with a zero scale, up to the pitch Np.
-        const int G = R / 16;
-        uint2* vst = reinterpret_cast<uint2*>(rtile);   // [copy][G][D + 1]
-        for (int idx = tid; idx < D * G; idx += kThreads) {
-          const int c = idx % D, g = idx / D;
-          if (r0 + g * 16 >= a.Np) continue;
-          float x[16], dqv[16], sc;
-          uint32_t pk[2], scc;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int r = g * 16 + i;
-            x[i] = (r < nrows) ? bf2f(tile[r * LD + c]) : 0.0f;
-          }
-          nvfp4_group(x, pk, scc, sc, inv_tab);
-          const int64_t tok = r0 + g * 16;
-          vst[g * (D + 1) + c] = make_uint2(pk[0], pk[1]);
-          scales[((int64_t)bh * (a.Np / 16) + tok / 16) * D + c] = (uint8_t)scc;
-          if (res) {
-            float rr[16], rsc;
-            nvfp4_dequant(pk, sc, dqv);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) rr[i] = __fsub_rn(x[i], dqv[i]);
-            nvfp4_group(rr, pk, scc, rsc, inv_tab);
-            vst[(G + g) * (D + 1) + c] = make_uint2(pk[0], pk[1]);
-            rscales[((int64_t)bh * (a.Np / 16) + tok / 16) * D + c] = (uint8_t)scc;
-          }
-        }
-        __syncthreads();
-        const int gv = min(G, (a.Np - r0) / 16);   // groups below the pitch
-        const int copies = res ? 2 : 1;
-        for (int idx = tid; idx < copies * D * gv; idx += kThreads) {
-          const int copy = idx / (D * gv), rem = idx % (D * gv);
-          const int c = rem / gv, g = rem % gv;
-          uint8_t* dst = (copy ? rcodes : codes) + ((int64_t)bh * D + c) * (a.Np / 2) + r0 / 2 + g * 8;
-          *reinterpret_cast<uint2*>(dst) = vst[(copy * G + g) * (D + 1) + c];
+        uint32_t p0[2], p1[2];
+        const uint32_t s0 = nvfp4_group(x0, p0, sc_tab);
+        const uint32_t s1 = nvfp4_group(x1, p1, sc_tab);
+        const int64_t srow = ((int64_t)bh * (a.Np / 16) + (r0 + g * 16) / 16) * D + 2 * cp;
+        *reinterpret_cast<uint4*>(vst + g * L::VP + 2 * cp) = make_uint4(p0[0], p0[1], p1[0], p1[1]);
+        *reinterpret_cast<uint16_t*>(scales + srow) = (uint16_t)(s0 | (s1 << 8));
+        if (res) {
+          float rr[16];
+          nvfp4_residual(x0, p0, sc_tab[s0].x, rr);
+          const uint32_t t0 = nvfp4_group(rr, p0, sc_tab);
+          nvfp4_residual(x1, p1, sc_tab[s1].x, rr);
+          const uint32_t t1 = nvfp4_group(rr, p1, sc_tab);
+          *reinterpret_cast<uint4*>(vst + (L::G + g) * L::VP + 2 * cp) =
+              make_uint4(p0[0], p0[1], p1[0], p1[1]);
+          *reinterpret_cast<uint16_t*>(rscales + srow) = (uint16_t)(t0 | (t1 << 8));
         }
       }
+      __syncthreads();
+      const int gv = min(L::G, (a.Np - r0) / 16);   // groups below the pitch
+      const int copies = res ? 2 : 1;
+      for (int idx = tid; idx < copies * D * gv; idx += kThreads) {
+        const int copy = idx / (D * gv), rem = idx % (D * gv);
+        const int c = rem / gv, g = rem % gv;
+        uint8_t* dst = (copy ? rcodes : codes) + ((int64_t)bh * D + c) * (a.Np / 2) + r0 / 2 + g * 8;
+        *reinterpret_cast<uint2*>(dst) = vst[(copy * L::G + g) * L::VP + c];
+      }
     }
-    __syncthreads();
-    // ---- dequantised copy, coalesced (only where a tile path reads it) ----
-    if (deq_out != nullptr)
+  }
+  __syncthreads();
+  // ---- dequantised copy, coalesced (only where a tile path reads it) ----
+  if (deq_out != nullptr)
     for (int idx = tid; idx < R * (D / 8); idx += kThreads) {
       const int r = idx / (D / 8), c8 = idx % (D / 8);
       if (r < nrows)
         *reinterpret_cast<uint4*>(deq_out + (bhN + r0 + r) * D + c8 * 8) =
-            *reinterpret_cast<const uint4*>(tile + r * LD + c8 * 8);
+            *reinterpret_cast<const uint4*>(tile + r * D + c8 * 8);
     }
-    __syncthreads();
-  }
 }
 
-template <int D>
-cudaError_t launch_prep_d(const PlanArgs& a, cudaStream_t s) {
-  const int chunks = (a.N + a.R - 1) / a.R;
-  const size_t smem = (size_t)2 * a.R * (D + 8) * sizeof(__nv_bfloat16) +
-                      (size_t)(kThreads + 8) * sizeof(float) + (size_t)kThreads * sizeof(double);
-  auto k = prep_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <int D, int R>
+cudaError_t launch_prep_dr(const PlanArgs& a, cudaStream_t s) {
+  using L = PrepSmem<D, R>;
+  const int chunks = (a.N + R - 1) / R;
+  auto k = prep_kernel<D, R>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(chunks, a.B * a.H, 3);
-  k<<<grid, kThreads, smem, s>>>(a);
+  k<<<grid, kThreads, L::kBytes, s>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_prep(const PlanArgs& a, cudaStream_t s) {
-  if (a.d == 64) return launch_prep_d<64>(a, s);
-  return launch_prep_d<128>(a, s);
+  // R = max(bq, bk), which the parameter check keeps to 64 or 128
+  if (a.d == 64) return a.R == 64 ? launch_prep_dr<64, 64>(a, s) : launch_prep_dr<64, 128>(a, s);
+  return a.R == 64 ? launch_prep_dr<128, 64>(a, s) : launch_prep_dr<128, 128>(a, s);
 }
 
 }  // namespace ta
