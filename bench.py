@@ -47,7 +47,7 @@ L2_BYTES = 126 * 2 ** 20
 # profiles/attn_kernel_480p_h8.md (8 heads, scaled to 40 by heads: traffic
 # grows with the (head, query block) rows); valid only for the kernel source it
 # was measured on and for that workload.
-ATTN_TRAFFIC = {"source_sha1": "54131e6e7b7a5ac4cdaebbb79673b36058173f14", "bytes_per_launch": 1592325120}
+ATTN_TRAFFIC = {"source_sha1": "1e216b4f03bb22d4745498d1ab6211ddf3b634c9", "bytes_per_launch": 1592325120}
 
 
 def _env_int(name, default):
