@@ -355,3 +355,25 @@ def test_head_interleaved_layout_matches_contiguous(cuda_ok):
               "q_scales", "k_scales", "v_scales"):
         assert torch.equal(views[k], views1[k]), k
     assert torch.equal(Os.cpu(), O1)
+
+
+@pytest.mark.parametrize("name,N", [("tiny", 1), ("tiny", 17), ("tiny", 100), ("480p", 1),
+                                    ("480p", 17), ("480p", 100), ("720p", 40)])
+def test_sequences_shorter_than_one_tile(cuda_ok, name, N):
+    # sequences shorter than one 128-token tile: N = 1 (a single key, and one
+    # NVFP4 V group holding one token), N = 17 (one group and one token of the
+    # next), N = 100 and 40 (a block short of its 128 rows; with 64-token
+    # blocks, N = 100 is a full block and a 36-token tail); the inputs are the
+    # first N tokens of the seeded ragged-grid inputs
+    grid = {"tiny": (4, 16, 16), "480p": (3, 10, 21), "720p": (3, 9, 20)}[name]
+    base, Q, K, V = inputs(name, grid=grid, H=2)
+    cfg = base.with_(grid=(1, 1, N))
+    Qs, Ks, Vs = (x[:, :, :N].contiguous() for x in (Q, K, V))
+    _, views, O, st = run_gpu(cfg, Qs, Ks, Vs)
+    assert st == 0
+    _plan_parity(cfg, Qs, Ks, Vs, views, [(0, h) for h in range(cfg.H)])
+    for h in range(cfg.H):
+        rt, _, Oref = oracle_head(cfg, Qs, Ks, Vs, 0, h)
+        n_diff, _ = compare_tiers(views["tier_map"][h].numpy(), rt)
+        assert n_diff == 0
+        assert_out_close(to64(O[0, h]), Oref, f"{name} N={N} head {h}")
