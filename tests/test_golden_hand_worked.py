@@ -4,10 +4,11 @@ Each fixture states its inputs, cites the passage its rule follows, and works
 every expected value by hand in its comments (no expected value was produced
 by running code).  The router rows pin pooling, the n_j-weighted pooled
 softmax, the (-M, j) sort with its tie rule, the exclusive prefix against the
-thresholds, the forced diagonal and the list order.  The attention case pins
-the power-of-two offset of P', the NVFP4 rounding of P' in groups of 16 keys
-and of V in groups of 16 tokens per column, and a denominator that sums P'
-before rounding.
+thresholds, the forced diagonal and the list order.  The low-tier attention
+case pins the power-of-two offset of P', the NVFP4 rounding of P' in groups of
+16 keys and of V in groups of 16 tokens per column, and a denominator that
+sums P' before rounding; the refine-tier case pins the residual copies (with
+e4m3 subnormal scales) and the three-term product that drops A2 B2.
 """
 
 import math
@@ -19,7 +20,7 @@ import pytest
 
 from oracle import route as R
 from oracle.attention import tiered_attention
-from oracle.quant import LOW_NVFP4
+from oracle.quant import LOW_NVFP4, LOW_NVFP4_RES
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
@@ -49,7 +50,11 @@ def _read(name):
 
 
 def _nums(text):
-    return [float(Fraction(t)) for t in text.split()]
+    out = []
+    for t in text.split():
+        num, _, den = t.partition("/")
+        out.append(float(Fraction(num) / Fraction(den or "1")))
+    return out
 
 
 def _ints(text):
@@ -85,8 +90,8 @@ def test_router_rows_hand_worked(case):
         np.testing.assert_array_equal(rt["lists"][i], _ints(lst.split(None, 1)[1]))
 
 
-def _attention_case():
-    sec = _read("nvfp4_tier_attention.txt")[""]
+def _attention_case(name="nvfp4_tier_attention.txt"):
+    sec = _read(name)[""]
     N, d, block = int(sec["N"]), int(sec["d"]), int(sec["block"])
     Q = np.zeros((1, 1, N, d))
     K = np.ones((1, 1, N, d))
@@ -113,4 +118,18 @@ def test_nvfp4_tier_attention_hand_worked(exact):
         rows = O[qb * block:(qb + 1) * block]
         # dyadic values: the fp64 pass reproduces them up to the rounding of
         # exp(0) - 1 = 0 and of a few exact products, i.e. exactly
+        np.testing.assert_allclose(rows, np.broadcast_to(want, rows.shape), rtol=0, atol=1e-15)
+
+
+def test_nvfp4_residual_tier_attention_hand_worked():
+    sec, Q, K, V, block = _attention_case("nvfp4_residual_attention.txt")
+    out = tiered_attention(Q, K, V, _nums(sec["tau"]), LOW_NVFP4_RES, block, block,
+                           int(sec["p_offset_log2"]))[(0, 0)]
+    tiers = out["route"]["tiers"]
+    np.testing.assert_array_equal(tiers[0], _ints(sec["tiers_qblock0"]))
+    np.testing.assert_array_equal(tiers[1], _ints(sec["tiers_qblock1"]))
+    for qb in range(2):
+        want = np.zeros(Q.shape[-1])
+        want[:2] = _nums(sec[f"O_qblock{qb}"])
+        rows = out["O"][qb * block:(qb + 1) * block]
         np.testing.assert_allclose(rows, np.broadcast_to(want, rows.shape), rtol=0, atol=1e-15)
