@@ -8,7 +8,9 @@ thresholds, the forced diagonal and the list order.  The low-tier attention
 case pins the power-of-two offset of P', the NVFP4 rounding of P' in groups of
 16 keys and of V in groups of 16 tokens per column, and a denominator that
 sums P' before rounding; the refine-tier case pins the residual copies (with
-e4m3 subnormal scales) and the three-term product that drops A2 B2.
+e4m3 subnormal scales) and the three-term product that drops A2 B2.  The
+price and entropy rows pin the price rule's objectives and spread and the
+entropy rule's k = ceil(kappa e^H) with its lift of kept blocks to NVFP4.
 """
 
 import math
@@ -133,3 +135,41 @@ def test_nvfp4_residual_tier_attention_hand_worked():
         want[:2] = _nums(sec[f"O_qblock{qb}"])
         rows = out["O"][qb * block:(qb + 1) * block]
         np.testing.assert_allclose(rows, np.broadcast_to(want, rows.shape), rtol=0, atol=1e-15)
+
+
+PRICE_ENTROPY = _read("router_price_entropy_rows.txt")
+
+
+def _check_rows(rt, rows):
+    assert len(rows) == rt["tiers"].shape[0]
+    for text in rows:
+        head, tiers, counts, lst = [p.strip() for p in text.split("|")]
+        i = int(head)
+        np.testing.assert_array_equal(rt["tiers"][i], _ints(tiers.split(None, 1)[1]))
+        np.testing.assert_array_equal(rt["counts"][i], _ints(counts.split(None, 1)[1]))
+        np.testing.assert_array_equal(rt["lists"][i], _ints(lst.split(None, 1)[1]))
+
+
+@pytest.mark.parametrize("case", sorted(PRICE_ENTROPY))
+def test_price_and_entropy_router_rows_hand_worked(case):
+    sec = PRICE_ENTROPY[case]
+    N, block = 320, 64
+    w = [8.0, 4.0, 2.0, 1.0, 1.0]
+    b = _nums(sec["b"])
+    Q = np.ones((N, 1))
+    K = np.empty((N, 1))
+    for j in range(len(w)):
+        rows = np.arange(j * block, (j + 1) * block)
+        K[rows, 0] = math.log(w[j]) + np.where(rows % 2 == 0, b[j], -b[j])
+    np.testing.assert_allclose(R.block_spread(K, block)[:, 0], np.square(b), rtol=1e-12, atol=1e-15)
+    if case == "price":
+        rt = R.route_head(Q, K, np.zeros((N, 1)), (0.5, 0.9), block, block, scale=1.0,
+                          router=R.ROUTER_PRICE, price=float(sec["price"]), low=LOW_NVFP4)
+        np.testing.assert_allclose(rt["delta"][0], b, rtol=1e-12, atol=1e-15)
+    else:
+        rt = R.route_head(Q, K, np.zeros((N, 1)), _nums(sec["tau"]), block, block, scale=1.0,
+                          router=R.ROUTER_ENTROPY, kappa=float(sec["kappa"]), low=LOW_NVFP4)
+        np.testing.assert_array_equal(rt["keep"], int(sec["keep"]))
+    np.testing.assert_allclose(rt["M"][0], np.array(w) / 16.0, rtol=1e-12)
+    assert not rt["flags"].any()
+    _check_rows(rt, sec["row"])
