@@ -2,8 +2,9 @@
 
 The compute path is libtiered_attn.so (hand-written sm_100a CUDA kernels
 behind a C ABI, see include/tiered_attn.h); this package is its thin Python
-binding.  Importing it requires the built library (``python -m
-precision_attention_video_b200.build``).
+binding.  The library is built in-tree by ``python -m
+precision_attention_video_b200.build`` and loaded on the first call; a call
+without it raises ImportError (there is no fallback path).
 """
 
 from .binding import (  # noqa: F401

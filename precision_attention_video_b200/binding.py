@@ -82,15 +82,21 @@ def _load():
     return lib
 
 
-_lib = _load()
+_lib = None
 
 
 def lib() -> ctypes.CDLL:
+    """The loaded library; loaded on first use, so that the package (and its
+    build module) imports before the library exists.  Every call into the
+    compute path goes through here and raises if the library is missing."""
+    global _lib
+    if _lib is None:
+        _lib = _load()
     return _lib
 
 
 def status_string(code: int) -> str:
-    return _lib.tiered_attn_status_string(code).decode()
+    return lib().tiered_attn_status_string(code).decode()
 
 
 class TieredAttnError(RuntimeError):
@@ -141,7 +147,7 @@ def _stream(stream) -> int:
 
 
 def workspace_bytes(p: ta_params) -> int:
-    return int(_lib.tiered_attn_workspace_bytes(ctypes.byref(p)))
+    return int(lib().tiered_attn_workspace_bytes(ctypes.byref(p)))
 
 
 def alloc_workspace(p: ta_params, device="cuda") -> torch.Tensor:
@@ -153,51 +159,51 @@ def alloc_workspace(p: ta_params, device="cuda") -> torch.Tensor:
 
 def plan(p: ta_params, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, ws: torch.Tensor,
          stream=None) -> None:
-    _check("tiered_attn_plan", _lib.tiered_attn_plan(
+    _check("tiered_attn_plan", lib().tiered_attn_plan(
         ctypes.byref(p), Q.data_ptr(), K.data_ptr(), V.data_ptr(), ws.data_ptr(),
         ws.numel(), _stream(stream)))
 
 
 def prep(p, Q, K, V, ws, stream=None) -> None:
-    _check("tiered_attn_prep", _lib.tiered_attn_prep(
+    _check("tiered_attn_prep", lib().tiered_attn_prep(
         ctypes.byref(p), Q.data_ptr(), K.data_ptr(), V.data_ptr(), ws.data_ptr(),
         ws.numel(), _stream(stream)))
 
 
 def route(p, ws, stream=None) -> None:
-    _check("tiered_attn_route", _lib.tiered_attn_route(
+    _check("tiered_attn_route", lib().tiered_attn_route(
         ctypes.byref(p), ws.data_ptr(), ws.numel(), _stream(stream)))
 
 
 def route_noalloc(p: ta_params, Q, K, V, tier_map, row_counts, row_lists, stream=None) -> None:
     """Tier map, row counts and row lists without any workspace: the router's
     intermediates live in the library's fixed device array (see the header)."""
-    _check("tiered_attn_route_noalloc", _lib.tiered_attn_route_noalloc(
+    _check("tiered_attn_route_noalloc", lib().tiered_attn_route_noalloc(
         ctypes.byref(p), Q.data_ptr(), K.data_ptr(), V.data_ptr(), tier_map.data_ptr(),
         row_counts.data_ptr(), row_lists.data_ptr(), _stream(stream)))
 
 
 def forward(p: ta_params, Q, K, V, ws, O, stream=None) -> None:
-    _check("tiered_attn_forward", _lib.tiered_attn_forward(
+    _check("tiered_attn_forward", lib().tiered_attn_forward(
         ctypes.byref(p), Q.data_ptr(), K.data_ptr(), V.data_ptr(), ws.data_ptr(), ws.numel(),
         O.data_ptr(), _stream(stream)))
 
 
 def layer_from_host(p, Qh, Kh, Vh, Oh, Qd, Kd, Vd, Od, ws, stream=None) -> None:
-    _check("tiered_attn_layer_from_host", _lib.tiered_attn_layer_from_host(
+    _check("tiered_attn_layer_from_host", lib().tiered_attn_layer_from_host(
         ctypes.byref(p), Qh.data_ptr(), Kh.data_ptr(), Vh.data_ptr(), Oh.data_ptr(),
         Qd.data_ptr(), Kd.data_ptr(), Vd.data_ptr(), Od.data_ptr(), ws.data_ptr(), ws.numel(),
         _stream(stream)))
 
 
 def get_status(ws: torch.Tensor, stream=None) -> int:
-    return int(_lib.tiered_attn_get_status(ws.data_ptr(), _stream(stream)))
+    return int(lib().tiered_attn_get_status(ws.data_ptr(), _stream(stream)))
 
 
 def plan_views(p: ta_params, ws: torch.Tensor) -> Dict[str, torch.Tensor]:
     """Typed tensor views of a planned workspace (no copies)."""
     v = ta_plan_views()
-    _check("tiered_attn_plan_views", _lib.tiered_attn_plan_views(
+    _check("tiered_attn_plan_views", lib().tiered_attn_plan_views(
         ctypes.byref(p), ws.data_ptr(), ctypes.byref(v)))
     BH = p.B * p.H
     N, d = p.N, p.d
@@ -240,4 +246,4 @@ def plan_views(p: ta_params, ws: torch.Tensor) -> Dict[str, torch.Tensor]:
 
 
 def version() -> int:
-    return int(_lib.tiered_attn_version())
+    return int(lib().tiered_attn_version())
