@@ -33,7 +33,8 @@ def _run(Q, K, V, tau, low, bq, bk, o=8, exact=True, keep_diag=True):
     return tiered_attention_head(Q, K, V, rt, qt, low, bq, bk, o, rt["scale"], exact), rt
 
 
-@pytest.mark.parametrize("N,bq,bk,d", [(200, 64, 64, 32), (256, 128, 64, 64), (300, 64, 128, 16)])
+@pytest.mark.parametrize("N,bq,bk,d", [(200, 64, 64, 32), (256, 128, 64, 64), (300, 64, 128, 16),
+                                    (300, 128, 32, 16)])
 def test_all_full_equals_dense(N, bq, bk, d):
     rng = np.random.default_rng(N)
     Q, K, V = (F.bf16_rne(rng.normal(size=(N, d)) * 2) for _ in range(3))
@@ -168,3 +169,31 @@ def test_tiers_mix_reasonable_on_generator_input():
     assert (t == R.TIER_FULL).any() and (t == R.TIER_LOW).any() and (t == R.TIER_SKIP).any()
     D = oracle.dense_attention(Q[0, 1], K[0, 1], V[0, 1])
     assert _rel(r["O"], D) < 0.3          # an approximation, but not garbage
+
+
+def test_fine_grained_key_blocks_of_32():
+    # FG-Attn ("FG-Attn" searcharxiv author page, abstract) skips at M x N
+    # granularity with M >= 16, N >= 1; the tiered method at N = 32 keys and
+    # M = 128 queries is the same pass over 32-key blocks.  Three exact cases:
+    rng = np.random.default_rng(12)
+    N, d, bq, bk = 296, 32, 128, 32               # 9 full key blocks and an 8-key tail
+    # (1) constant 32-key blocks: skipping them is exact
+    nb = -(-N // bk)
+    K = np.repeat(F.bf16_rne(rng.normal(size=(nb, d))), bk, axis=0)[:N]
+    V = np.repeat(F.bf16_rne(rng.normal(size=(nb, d))), bk, axis=0)[:N]
+    Q = F.bf16_rne(rng.normal(size=(N, d)))
+    O, rt = _run(Q, K, V, (0.0, 0.0), Qz.LOW_FP8, bq, bk)
+    assert (rt["tiers"] == R.TIER_SKIP).sum() > 0
+    assert rt["n_k"][-1] == N - (nb - 1) * bk
+    assert _rel(O, oracle.dense_attention(Q, K, V)) <= 1e-12
+    # (2) operands on the NVFP4 grid, every tile low: a 32-key tile holds two
+    # whole 16-token V groups and two 16-key P groups, so exact=True is dense
+    N2 = 256
+    Q2, K2 = _nvfp4_grid_rows(rng, N2, d), _nvfp4_grid_rows(rng, N2, d)
+    V2 = _nvfp4_grid_rows(rng, d, N2).T.copy()
+    O2, rt2 = _run(Q2, K2, V2, (0.0, 2.0), Qz.LOW_NVFP4, bq, bk, o=11, keep_diag=False)
+    assert (rt2["tiers"] == R.TIER_LOW).all()
+    assert _rel(O2, oracle.dense_attention(Q2, K2, V2)) <= 1e-12
+    # (3) the diagonal of a 128-row query block covers four 32-key blocks
+    assert R.diag_blocks(1, bq, bk, N) == [4, 5, 6, 7]
+    assert all((rt["tiers"][1, 4:8] == R.TIER_FULL))
