@@ -1,5 +1,7 @@
 """Host-side logic of the benchmark: the algorithmic FLOP count per tier that
-the roofline line divides by, checked against a hand count on a small plan."""
+the roofline line divides by, checked against a hand count on a small plan,
+and the summary of the clock samples taken during the timed region (median
+SM clock, throttle reasons) that decides whether a run is kept."""
 
 import importlib.util
 import os
@@ -35,3 +37,28 @@ def test_algorithmic_flops_by_tier():
     want_low = 4 * d * (q[0] * k[1] + q[2] * k[0])
     want_skip = 4 * d * (q[1] * 1 + q[2] * 1)
     assert (full, res, low, skip) == (want_full, want_res, want_low, want_skip)
+
+
+def test_clock_summary_from_nvidia_smi_lines():
+    # lines as `nvidia-smi --query-gpu=... --format=csv,noheader,nounits` prints them:
+    # index, clocks.sm, clocks.max.sm, power.draw, reasons.active, hw_slowdown,
+    # hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap
+    bench = _bench()
+    cs = bench.ClockSampler(0)
+    cs.lines = [
+        "0, 1965, 1965, 612.40, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1845, 1965, 998.10, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1900, 1965, 990.00, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, [N/A], 1965, [N/A], [N/A], [N/A], [N/A], [N/A], [N/A]",   # unreadable sample
+        "garbled",
+    ]
+    s = cs.summary()
+    assert s["samples"] == 3
+    assert s["sm_mhz"] == 1900.0            # median of 1965, 1845, 1900
+    assert s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
+    cs.lines.append("0, 1200, 1965, 700.0, 0x0000000000000048, Active, Active, Not Active, Not Active")
+    assert bench.ClockSampler.summary(cs)["reasons"] == ["hw_slowdown", "hw_thermal_slowdown",
+                                                         "sw_power_cap"]
+    cs.lines = []
+    assert cs.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
