@@ -370,10 +370,10 @@ def run_gpu_arm(args, rank, world, local_rank):
 
 def cpu_baseline(cfg, budget_s: float = 20.0, threads: int = 0):
     """The oracle, as it stands, on a bounded sample of the workload: whole
-    heads are routed and quantised, then query blocks of those heads (spread
-    over the sequence) are attended until the time budget is used.  The unit
-    is dense-equivalent TFLOPS of the query rows attended; input generation is
-    not timed."""
+    heads are routed (with the workload's router) and quantised, then query
+    blocks of those heads (spread over the sequence) are attended until the
+    time budget is used.  The unit is dense-equivalent TFLOPS of the query
+    rows attended; input generation is not timed."""
     import oracle
     from latent_gen.generator import make_head
     from oracle import quant as Qz
@@ -387,7 +387,9 @@ def cpu_baseline(cfg, budget_s: float = 20.0, threads: int = 0):
         q, k, v = make_head(cfg, 0, heads)
         Qh, Kh, Vh = (torch.from_numpy(x).to(torch.bfloat16).double().numpy() for x in (q, k, v))
         t = time.time()
-        rt = Rt.route_head(Qh, Kh, Vh, cfg.tau, cfg.block_q, cfg.block_k)
+        rt = Rt.route_head(Qh, Kh, Vh, cfg.tau, cfg.block_q, cfg.block_k,
+                           router=getattr(cfg, "router", 0), price=getattr(cfg, "price", 0.0),
+                           low=cfg.low, kappa=getattr(cfg, "kappa", 1.0))
         qt = Qz.quantize_head(Qh, Kh, Vh, cfg.low, cfg.block_q, cfg.block_k)
         spent += time.time() - t
         done = 0
