@@ -118,3 +118,51 @@ def test_residual_reduces_error():
     r = F.fp32_rne(X - qt["dq"])
     c, s = Qz.quant_nvfp4_rows(r)
     np.testing.assert_array_equal(c, qt["rq_codes"])
+
+
+def _nearest_even(v, grid_vals, grid_codes):
+    """Brute force: the grid value nearest to v; on an exact tie the one whose
+    code is even (the encoding's last mantissa bit 0)."""
+    d = np.abs(grid_vals - v)
+    best = np.nonzero(d == d.min())[0]
+    if len(best) > 1:
+        best = [b for b in best if grid_codes[b] % 2 == 0]
+    return grid_codes[best[0]], grid_vals[best[0]]
+
+
+def test_nvfp4_groups_match_brute_force_nearest():
+    # The whole group rule restated by exhaustive search over the two grids,
+    # with no bit manipulation: sc = the ue4m3 value nearest fp32(amax / 6)
+    # (ties to the even code, saturating at 448), then each element's e2m1
+    # value nearest fp32(x * fp32(1 / sc)) (ties to even, saturating at 6,
+    # sign kept), and every code 0 when sc = 0.
+    rng = np.random.default_rng(21)
+    e4 = [(c, F.e4m3_decode(np.array([c], dtype=np.uint8))[0]) for c in range(0x7F)]
+    e4_codes = np.array([c for c, _ in e4])
+    e4_vals = np.array([v for _, v in e4])
+    e2_vals = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    e2_codes = np.arange(8)
+    f32 = lambda v: float(np.float32(v))
+    groups = []
+    for _ in range(3000):
+        mag = 2.0 ** rng.uniform(-14, 12)                    # subnormal to saturated scales
+        g = rng.normal(size=16) * mag
+        g[rng.random(16) < 0.2] = 0.0
+        groups.append(F.bf16_rne(g))
+    groups.append(np.zeros(16))
+    G = np.stack(groups)
+    codes, sc_code = Qz.nvfp4_quant_groups(G)
+    for k in range(G.shape[0]):
+        x = G[k]
+        q = f32(f32(np.abs(x).max()) / 6.0)
+        want_sc, sc = _nearest_even(min(q, 448.0), e4_vals, e4_codes)
+        assert int(sc_code[k]) == want_sc, (k, q)
+        if sc == 0.0:
+            assert not codes[k].any()
+            continue
+        inv = f32(1.0 / sc)
+        for i in range(16):
+            y = f32(x[i] * inv)
+            c, _ = _nearest_even(min(abs(y), 6.0), e2_vals, e2_codes)
+            want = c | (8 if y < 0 or (y == 0 and np.signbit(y)) else 0)
+            assert int(codes[k, i]) == want, (k, i, x[i], y)
