@@ -166,3 +166,26 @@ def test_nvfp4_groups_match_brute_force_nearest():
             c, _ = _nearest_even(min(abs(y), 6.0), e2_vals, e2_codes)
             want = c | (8 if y < 0 or (y == 0 and np.signbit(y)) else 0)
             assert int(codes[k, i]) == want, (k, i, x[i], y)
+
+
+def test_fp8_tiles_match_brute_force_nearest():
+    # One tile: s = the smallest power of two with amax <= 448 s (found by
+    # stepping through powers of two), codes = the e4m3 value nearest x / s
+    # (exact: s is a power of two), ties to the even code, sign kept.
+    rng = np.random.default_rng(22)
+    e4 = [(c, F.e4m3_decode(np.array([c], dtype=np.uint8))[0]) for c in range(0x7F)]
+    e4_codes = np.array([c for c, _ in e4])
+    e4_vals = np.array([v for _, v in e4])
+    for t in range(200):
+        X = F.bf16_rne(rng.normal(size=(8, 16)) * 2.0 ** rng.uniform(-20, 20))
+        codes, scales = Qz.quant_fp8_tiles(X, 8)
+        amax = np.abs(X).max()
+        k = -200
+        while amax > 448.0 * 2.0 ** k:
+            k += 1
+        assert scales[0] == 2.0 ** k
+        for idx in np.ndindex(X.shape):
+            y = X[idx] / 2.0 ** k
+            c, _ = _nearest_even(abs(y), e4_vals, e4_codes)
+            want = c | (0x80 if y < 0 else 0)
+            assert int(codes[idx]) == want, (t, idx, y)
