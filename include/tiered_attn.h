@@ -79,7 +79,9 @@ typedef enum {
 enum { TA_TIER_SKIP = 0, TA_TIER_LOW = 1, TA_TIER_RES = 2, TA_TIER_FULL = 3 };
 
 typedef struct {
-  int32_t B, H, N, d;        /* batch, heads, tokens, head dim (d in {64,128}) */
+  int32_t B, H, N, d;        /* batch, heads, tokens (N >= 1; the last query and
+                                key blocks may be partial, down to one token),
+                                head dim (d in {64,128})                       */
   int32_t block_q, block_k;  /* tile rows / keys, each in {64,128}            */
   int32_t low;               /* ta_low_format                                 */
   int32_t n_thresholds;      /* 1 (full only), 2 (full, low), 3 (full, res, low) */
