@@ -173,3 +173,25 @@ def test_price_and_entropy_router_rows_hand_worked(case):
     np.testing.assert_allclose(rt["M"][0], np.array(w) / 16.0, rtol=1e-12)
     assert not rt["flags"].any()
     _check_rows(rt, sec["row"])
+
+
+def test_fp8_tier_attention_hand_worked():
+    from oracle.quant import LOW_FP8
+    sec = _read("fp8_tier_attention.txt")[""]
+    N, d, block = int(sec["N"]), int(sec["d"]), int(sec["block"])
+    Q = np.zeros((1, 1, N, d))
+    K = np.ones((1, 1, N, d))
+    V = np.zeros((1, 1, N, d))
+    V[0, 0, :4, 0] = 1.0
+    V[0, 0, 4:, 1] = float(sec["v_block1"])
+    out = tiered_attention(Q, K, V, _nums(sec["tau"]), LOW_FP8, block, block,
+                           int(sec["p_offset_log2"]))[(0, 0)]
+    tiers = out["route"]["tiers"]
+    np.testing.assert_array_equal(tiers[0], _ints(sec["tiers_qblock0"]))
+    np.testing.assert_array_equal(tiers[1], _ints(sec["tiers_qblock1"]))
+    np.testing.assert_array_equal(out["quant"]["v_scale"], [2.0 ** -8, 2.0 ** -10])
+    for qb in range(2):
+        want = np.zeros(d)
+        want[:2] = _nums(sec[f"O_qblock{qb}"])
+        rows = out["O"][qb * block:(qb + 1) * block]
+        np.testing.assert_allclose(rows, np.broadcast_to(want, rows.shape), rtol=0, atol=1e-15)
