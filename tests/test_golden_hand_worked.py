@@ -11,6 +11,9 @@ sums P' before rounding; the refine-tier case pins the residual copies (with
 e4m3 subnormal scales) and the three-term product that drops A2 B2.  The
 price and entropy rows pin the price rule's objectives and spread and the
 entropy rule's k = ceil(kappa e^H) with its lift of kept blocks to NVFP4.
+The FP8 case pins the power-of-two tile scales and e4m3 rounding; the skip
+case pins the n_j weight of a ragged skipped block and the bf16 rounding of
+its pseudo-value.
 """
 
 import math
@@ -195,3 +198,25 @@ def test_fp8_tier_attention_hand_worked():
         want[:2] = _nums(sec[f"O_qblock{qb}"])
         rows = out["O"][qb * block:(qb + 1) * block]
         np.testing.assert_allclose(rows, np.broadcast_to(want, rows.shape), rtol=0, atol=1e-15)
+
+
+def test_skip_tier_attention_hand_worked():
+    from oracle.quant import LOW_FP8
+    sec = _read("skip_tier_attention.txt")[""]
+    N, d, block = int(sec["N"]), int(sec["d"]), int(sec["block"])
+    Q = np.zeros((1, 1, N, d))
+    K = np.ones((1, 1, N, d))
+    V = np.zeros((1, 1, N, d))
+    V[0, 0, :4, 0] = 1.0
+    V[0, 0, 4:6, 1] = 1.0
+    V[0, 0, 6, 1] = 0.75
+    out = tiered_attention(Q, K, V, _nums(sec["tau"]), LOW_FP8, block, block,
+                           int(sec["p_offset_log2"]))[(0, 0)]
+    tiers = out["route"]["tiers"]
+    np.testing.assert_array_equal(tiers[0], _ints(sec["tiers_qblock0"]))
+    np.testing.assert_array_equal(tiers[1], _ints(sec["tiers_qblock1"]))
+    for qb in range(2):
+        want = np.zeros(d)
+        want[:2] = _nums(sec[f"O_qblock{qb}"])
+        rows = out["O"][qb * block:min(N, (qb + 1) * block)]
+        np.testing.assert_allclose(rows, np.broadcast_to(want, rows.shape), rtol=1e-15, atol=1e-15)
