@@ -43,10 +43,10 @@ UNIT = "TFLOPS"
 L2_BYTES = 126 * 2 ** 20
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one forward
-# launch of the 480p-video-like layer, from the ncu capture summarised in
-# profiles/attn_kernel_480p_h8.md (8 heads, scaled to 40 by heads: traffic
-# grows with the (head, query block) rows); valid only for the kernel source it
-# was measured on and for that workload.
+# launch of the 480p-video-like layer, from the ncu capture of this kernel on
+# 8 heads of that layer, scaled to 40 by heads (traffic grows with the (head,
+# query block) rows); valid only for the kernel source it was measured on and
+# for that workload.
 ATTN_TRAFFIC = {"source_sha1": "1e216b4f03bb22d4745498d1ab6211ddf3b634c9", "bytes_per_launch": 1592325120}
 
 
@@ -64,6 +64,20 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def bf16_peak(peaks, clocks):
+    """The bf16 tensor peak that applies to this run: the burst figure (a
+    short matmul at full clock) when the sampled SM clock stayed at its
+    maximum with no power cap, else the sustained one (a seconds-long matmul
+    whose clock sank under the power cap).  Returns (TFLOP/s, which)."""
+    burst = float(peaks.get("bf16_tflops", 0.0) or 0.0)
+    sustained = float(peaks.get("bf16_tflops_sustained", burst) or burst)
+    sm, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    full_clock = sm is not None and mx and sm >= 0.97 * mx
+    if burst and full_clock and "sw_power_cap" not in clocks.get("reasons", []):
+        return burst, f"burst bf16_tflops (SM clock {sm:.0f} of {mx:.0f} MHz, no power cap)"
+    return sustained, "sustained bf16_tflops_sustained (SM clock below max or power-capped)"
 
 
 def attn_source_sha1():
@@ -501,7 +515,7 @@ def main():
     fwd_ms = statistics.mean(r["fwd_ms"])
     step_ms, fwd_ms, e2e_ms = max_over_ranks([step_ms, fwd_ms, r["e2e_ms"]], world)
     peaks, peak_src = load_peaks()
-    p_bf16 = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    p_bf16, peak_kind = bf16_peak(peaks, r["clocks"])
     # Full tiles and skip chunks run on the bf16 pipe; NVFP4 tiles (low and
     # residual) on the FP4 pipe and native FP8 tiles (d = 128, 128 x 128) on
     # the FP8 pipe, whose peaks are taken as 4x and 2x the measured bf16 one
@@ -529,9 +543,10 @@ def main():
             "roofline": {"kernel": "tiered_attn_forward (attn_kernel<128,128>)", "bound": "tensor",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": (f"blend of {peak_src} bf16_tflops_sustained "
+                         "peak_source": (f"blend of {peak_src} bf16 {peak_kind} "
                                          f"{p_bf16:.1f}, nvfp4 = 4x and native fp8 = 2x "
-                                         "that, weighted by the launch's FLOPs per tier"),
+                                         "that (nominal ratios), weighted by the launch's "
+                                         "FLOPs per tier"),
                          "flops_per_launch": executed,
                          "flops_by_tier": {"full": r["full_flops"], "res": r["res_flops"],
                                            "low": r["low_flops"], "skip": r["skip_flops"]}},

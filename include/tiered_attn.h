@@ -119,8 +119,9 @@ typedef struct {
   double*  mass;             /* f64 [BH, nQb, nKb] pooled block mass M        */
   uint8_t* tier_map;         /* u8  [BH, nQb, nKb] TA_TIER_* per tile          */
   int32_t* row_counts;       /* i32 [BH, nQb, 4] tiles per tier: full, res, low, skip */
-  int32_t* row_lists;        /* i32 [BH, nQb, nKb] key blocks: full ascending,
-                                then res, low, skip (each ascending)           */
+  int32_t* row_lists;        /* i32 [BH, nQb, nKb] key blocks by tier: full,
+                                then res, low, skip; within a tier by
+                                descending pooled mass M, ties by ascending j */
   /* FP8 copies: codes u8 [BH, N, d] (row-major like the input), scales f32
    * per tile [BH, nQb] for Q and [BH, nKb] for K and V.
    * NVFP4 copies: Q, K codes packed two per byte along d, u8 [BH, N, d/2]
@@ -249,12 +250,15 @@ ta_status tiered_attn_route(const ta_params* p, void* ws_dev, size_t ws_bytes, v
  * or a latency-critical path where cudaMalloc would synchronise the device.
  * From Q, K, V it writes the tier map (u8 [B*H, nQb, nKb]), the per-row tier
  * counts (i32 [B*H, nQb, 4]) and the per-row lists (i32 [B*H, nQb, nKb]) into
- * caller buffers, exactly as tiered_attn_plan does; it makes no low-precision
- * copies.  Its intermediate block means, pooled logits and masses live in one
- * fixed array of TA_ROUTE_NOALLOC_SCRATCH_BYTES in the library's device memory,
- * which every GPU that loads the library holds until the process exits.
+ * caller buffers, exactly as tiered_attn_plan does with the same params (every
+ * router: mass, price and entropy); it makes no low-precision copies.  Its
+ * intermediate block means, pooled logits and masses (and, for the price
+ * router, the block variances and skip spreads) live in one fixed array of
+ * TA_ROUTE_NOALLOC_SCRATCH_BYTES in the library's device memory, which every
+ * GPU that loads the library holds until the process exits.
  *  - Problems whose intermediates exceed that size (about B*H*nQb*nKb*16 +
- *    B*H*(nQb+nKb)*d*8 + B*H*nKb*d*4 bytes) return TA_ERR_WORKSPACE.
+ *    B*H*(nQb+nKb)*d*8 + B*H*nKb*d*4 bytes; the price router adds
+ *    B*H*nQb*nKb*8 + B*H*(nQb+nKb)*d*8) return TA_ERR_WORKSPACE.
  *  - The first call on a device looks up the array's device address (with that
  *    device current); make that first call before any stream capture.
  *  - All calls share the one array: calls whose work overlaps on the GPU (two

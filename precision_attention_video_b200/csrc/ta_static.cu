@@ -56,18 +56,24 @@ extern "C" ta_status tiered_attn_route_noalloc(const ta_params* p, const void* Q
   const int64_t BH = (int64_t)p->B * p->H;
   const int64_t nQb = (p->N + p->block_q - 1) / p->block_q;
   const int64_t nKb = (p->N + p->block_k - 1) / p->block_k;
-  // scratch sections: status, n_k, qbar, kbar, kbar_b, vbar_b, logits, mass
-  size_t off[9];
+  const bool price = p->router == TA_ROUTER_PRICE;
+  // scratch sections: status, n_k, qbar, kbar, kbar_b, vbar_b, logits, mass;
+  // for the price router also kvar, qvar (block coordinate variances) and
+  // spread (the skip tier's error factor)
+  constexpr int kSections = 11;
+  size_t off[kSections];
   size_t at = 0;
-  const size_t sizes[8] = {16, (size_t)nKb * 4, (size_t)(BH * nQb * p->d * 8),
-                           (size_t)(BH * nKb * p->d * 8), (size_t)(BH * nKb * p->d * 2),
-                           (size_t)(BH * nKb * p->d * 2), (size_t)(BH * nQb * nKb * 8),
-                           (size_t)(BH * nQb * nKb * 8)};
-  for (int i = 0; i < 8; ++i) {
+  const size_t sizes[kSections] = {16, (size_t)nKb * 4, (size_t)(BH * nQb * p->d * 8),
+                                   (size_t)(BH * nKb * p->d * 8), (size_t)(BH * nKb * p->d * 2),
+                                   (size_t)(BH * nKb * p->d * 2), (size_t)(BH * nQb * nKb * 8),
+                                   (size_t)(BH * nQb * nKb * 8),
+                                   price ? (size_t)(BH * nKb * p->d * 8) : 0,
+                                   price ? (size_t)(BH * nQb * p->d * 8) : 0,
+                                   price ? (size_t)(BH * nQb * nKb * 8) : 0};
+  for (int i = 0; i < kSections; ++i) {
     off[i] = at;
     at = up256(at + sizes[i]);
   }
-  off[8] = at;
   if (at > kScratchBytes) return TA_ERR_WORKSPACE;  // problem too large for the fixed scratch
 
   unsigned char* base = static_cast<unsigned char*>(scratch_on_current_device());
@@ -88,7 +94,7 @@ extern "C" ta_status tiered_attn_route_noalloc(const ta_params* p, const void* Q
   a.d = p->d;
   a.bq = p->block_q;
   a.bk = p->block_k;
-  a.low = TA_LOW_NONE;  // block means only: no low-precision copies
+  a.low = TA_LOW_NONE;  // prep: block means (and variances) only, no low-precision copies
   a.R = p->block_q > p->block_k ? p->block_q : p->block_k;
   a.nQb = (int)nQb;
   a.nKb = (int)nKb;
@@ -96,6 +102,9 @@ extern "C" ta_status tiered_attn_route_noalloc(const ta_params* p, const void* Q
   a.n_tau = p->n_thresholds;
   for (int i = 0; i < 3; ++i) a.tau[i] = i < p->n_thresholds ? p->tau[i] : 0.0;
   a.keep_diag = p->keep_diag_full;
+  a.router = p->router;
+  a.price = p->price;
+  a.retention = p->retention;
   a.scale = p->softmax_scale > 0.0f ? (double)p->softmax_scale : 1.0 / std::sqrt((double)p->d);
   a.status = reinterpret_cast<int*>(base + off[0]);
   a.n_k = reinterpret_cast<int*>(base + off[1]);
@@ -105,6 +114,11 @@ extern "C" ta_status tiered_attn_route_noalloc(const ta_params* p, const void* Q
   a.vbar_b = reinterpret_cast<__nv_bfloat16*>(base + off[5]);
   a.logits = reinterpret_cast<double*>(base + off[6]);
   a.mass = reinterpret_cast<double*>(base + off[7]);
+  if (price) {
+    a.kvar = reinterpret_cast<double*>(base + off[8]);
+    a.qvar = reinterpret_cast<double*>(base + off[9]);
+    a.spread = reinterpret_cast<double*>(base + off[10]);
+  }
   a.tier_map = tier_map;
   a.row_counts = row_counts;
   a.row_lists = row_lists;
@@ -113,6 +127,8 @@ extern "C" ta_status tiered_attn_route_noalloc(const ta_params* p, const void* Q
   // other section is fully rewritten by the kernels below
   if (cudaMemsetAsync(a.status, 0, 16, s) != cudaSuccess) return TA_ERR_CUDA;
   if (ta::launch_prep(a, s) != cudaSuccess) return TA_ERR_CUDA;
+  // the price router chooses among the tiers the low format provides
+  a.low = p->low;
   if (ta::launch_route(a, s) != cudaSuccess) return TA_ERR_CUDA;
   return TA_OK;
 }

@@ -62,3 +62,19 @@ def test_clock_summary_from_nvidia_smi_lines():
                                                          "sw_power_cap"]
     cs.lines = []
     assert cs.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def test_bf16_peak_follows_the_sampled_clock():
+    # burst peak when the timed region ran at the maximum SM clock with no
+    # power cap; sustained peak otherwise (clock sank, or power-capped)
+    bench = _bench()
+    peaks = {"bf16_tflops": 1606.7, "bf16_tflops_sustained": 1365.0}
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.bf16_peak(peaks, full)[0] == 1606.7
+    assert "burst" in bench.bf16_peak(peaks, full)[1]
+    capped = dict(full, reasons=["sw_power_cap"])
+    assert bench.bf16_peak(peaks, capped)[0] == 1365.0
+    slow = dict(full, sm_mhz=1305.0)
+    assert bench.bf16_peak(peaks, slow)[0] == 1365.0
+    none = {"sm_mhz": None, "sm_max_mhz": None, "reasons": []}
+    assert "sustained" in bench.bf16_peak(peaks, none)[1]

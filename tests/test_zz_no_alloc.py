@@ -4,8 +4,9 @@ tiered_attn_route_noalloc serves callers that cannot allocate device memory
 (code inside a host framework that owns the GPU's memory, or a latency-critical
 path where cudaMalloc would synchronise the device): its intermediates live in
 a fixed array inside the library.  It must produce the same tier map, row
-counts and row lists as tiered_attn_plan, and keep doing so on back-to-back
-calls that reuse the array.  This file is collected last on purpose.
+counts and row lists as tiered_attn_plan with the same params, for every
+router, and keep doing so on back-to-back calls that reuse the array.  This
+file is collected last on purpose.
 """
 
 import numpy as np
@@ -17,10 +18,22 @@ from gpu_helpers import inputs
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name", ["tiny", "small"])
-def test_noalloc_router_matches_plan_twice(cuda_ok, name):
+CASES = [
+    ("tiny", {}),                                            # mass router, FP8
+    ("small", {}),                                           # 128 x 64 tiles
+    ("480p", {"H": 2, "grid": (3, 10, 21)}),                 # ragged N = 630, NVFP4
+    ("720p", {"H": 2, "grid": (3, 9, 20)}),                  # ragged N = 540, four tiers
+    ("480p-price", {"H": 2, "grid": (3, 10, 21), "price": 0.028}),   # price router
+    ("small", {"H": 3, "router": 1, "price": 0.002}),        # price router, FP8 tiers
+    ("480p", {"H": 2, "grid": (3, 10, 21), "router": 2, "kappa": 0.5}),  # entropy router
+    ("720p", {"H": 2, "grid": (3, 9, 20), "router": 2, "kappa": 1.0}),   # entropy, four tiers
+]
+
+
+@pytest.mark.parametrize("name,over", CASES, ids=[f"{n}-{i}" for i, (n, _) in enumerate(CASES)])
+def test_noalloc_router_matches_plan_twice(cuda_ok, name, over):
     import precision_attention_video_b200 as pav
-    cfg, Q, K, V = inputs(name)
+    cfg, Q, K, V = inputs(name, **over)
     dev = torch.device("cuda:0")
     Qd, Kd, Vd = (x.to(dev) for x in (Q, K, V))
     p = pav.params_for(cfg)
@@ -37,8 +50,10 @@ def test_noalloc_router_matches_plan_twice(cuda_ok, name):
         lst = torch.full((BH, cfg.n_qb, cfg.n_kb), -1, dtype=torch.int32, device=dev)
         pav.route_noalloc(p, Qd, Kd, Vd, tmap, cnt, lst)
         torch.cuda.synchronize()
+        c = cnt.cpu().numpy()
+        assert (c.sum(axis=-1) == cfg.n_kb).all(), f"call {call}: counts do not cover every block"
         np.testing.assert_array_equal(tmap.cpu().numpy(), want_t, err_msg=f"call {call}")
-        np.testing.assert_array_equal(cnt.cpu().numpy(), want_c, err_msg=f"call {call}")
+        np.testing.assert_array_equal(c, want_c, err_msg=f"call {call}")
         np.testing.assert_array_equal(lst.cpu().numpy(), want_l, err_msg=f"call {call}")
 
 
