@@ -99,7 +99,24 @@ typedef struct {
                                 >= 0); unused by the other routers             */
   double  retention;         /* TA_ROUTER_ENTROPY: kappa, the kept blocks per
                                 effective block (finite, > 0); unused otherwise */
+  double  tier_cost[4];      /* TA_ROUTER_PRICE: compute cost of a tile in each
+                                tier, indexed by tier code (skip, low, res,
+                                full), in units of one bf16 tile (finite,
+                                >= 0).  All zero selects the costs measured on
+                                this library's attention kernel
+                                (TA_TIER_COST_* below); unused by the other
+                                routers */
 } ta_params;
+
+/* Default tier costs of the price router: per-tile time of each tier on this
+ * library's fused attention kernel (B200, d = 128, 128 x 128 tiles), relative
+ * to a bf16 tile.  A skipped block costs one column of a 128-block skip
+ * chunk.  The low tier's cost depends on its format. */
+#define TA_TIER_COST_SKIP 0.008
+#define TA_TIER_COST_FP8 1.0
+#define TA_TIER_COST_NVFP4 1.1
+#define TA_TIER_COST_NVFP4_RES 2.2
+#define TA_TIER_COST_FULL 1.0
 
 /* Test hook: the attention producer never loads the first K tile, so the
  * kernel's bounded wait runs out and the status word reports TA_ERR_TIMEOUT. */

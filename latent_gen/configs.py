@@ -48,6 +48,7 @@ class Workload:
     router: int = 0                     # 0: pooled-mass thresholds tau; 1: single price; 2: entropy
     price: float = 0.0                  # the price of router 1
     kappa: float = 1.0                  # the retention scale of router 2
+    tier_cost: Tuple[float, ...] = (0.0, 0.0, 0.0, 0.0)   # router 1's costs by tier code; 0s: defaults
     extra: Dict[str, float] = field(default_factory=dict)
 
     @property

@@ -6,7 +6,9 @@ TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``): run once to write
 The workload is the 480p-video-like layer (B=1, H=40, N=32760, d=128,
 128 x 128 tiles) with all four tiers (bf16, NVFP4 + residual, NVFP4, skip)
 chosen by the price rule of ``oracle.route`` ("Triage" abstract: a single
-price sets the trade-off between predicted error and compute).  Reading: one
+price sets the trade-off between predicted error and compute), with the
+rule's default tier costs (each tier's per-tile time on the fused kernel
+relative to a bf16 tile).  Reading: one
 global price, found by bisection on the oracle's fp64 pooled masses and skip
 spreads of all heads, so that half of all tiles are skipped (the forced
 diagonal counts as kept), the share the pooled-mass 480p workload skips.
@@ -32,8 +34,8 @@ from latent_gen import get_config  # noqa: E402
 from latent_gen.generator import make_head  # noqa: E402
 from oracle.quant import LOW_NVFP4_RES  # noqa: E402
 from oracle.route import (TIER_FULL, TIER_LOW, TIER_RES, TIER_SKIP,  # noqa: E402
-                          assign_tiers_price, block_spread, diag_blocks, pool_means,
-                          pooled_mass)
+                          assign_tiers_price, block_spread, default_tier_cost, diag_blocks,
+                          pool_means, pooled_mass)
 
 TARGET_SKIP = 0.5
 
@@ -79,6 +81,7 @@ def main():
     f = fractions(stats, cfg, price)
     out = {"workload": "480p-video-like, price router, NVFP4 + residual", "target_skip": TARGET_SKIP,
            "method": "bisection on the oracle's fp64 pooled masses and skip spreads (all 40 heads)",
+           "tier_cost": list(default_tier_cost(LOW_NVFP4_RES)),
            "price": price,
            "achieved": {"full": f[TIER_FULL], "res": f[TIER_RES], "low": f[TIER_LOW], "skip": f[TIER_SKIP]}}
     print(out, flush=True)

@@ -43,9 +43,13 @@ error reduction is worth the extra compute at a single price.  Reading:
     the RMS over the tile's (query, key) pairs of how far a query's logit
     moves from the one it has with the block's mean key, were the
     coordinates uncorrelated; that is what replacing the block by its means
-    ignores (0 when the block's keys are equal, and then skipping is exact).  Cost of tier t: its tensor-pipe time
-    relative to an NVFP4 tile at the nominal rates (skip 0, NVFP4 1, FP8 2,
-    NVFP4 + residual 3, bf16 4).  The tile takes the tier of least
+    ignores (0 when the block's keys are equal, and then skipping is exact).
+    Cost of tier t: the compute the tier spends, a parameter (tier_cost, by
+    tier code).  By default each tier's measured per-tile time on the fused
+    kernel relative to a bf16 tile (skip 0.008, FP8 1.0, NVFP4 1.1, NVFP4 +
+    residual 2.2, bf16 1.0): the abstract moves a tile up only when the
+    error reduction justifies the extra compute, and the compute a tier
+    costs is what the kernel spends on it.  The tile takes the tier of least
     e_t + price * cost_t among the tiers the low format provides; on a tie the
     cheaper tier.  The forced diagonal (step 4's last sentence) still applies,
     and step 6 orders the lists as before.
@@ -191,26 +195,38 @@ def block_spread(X: np.ndarray, block: int) -> np.ndarray:
     return np.stack(out)
 
 
-def price_tiers(low: int):
+def default_tier_cost(low: int):
+    """Step 4' costs when none are given, by tier code (skip, low, res, full):
+    each tier's per-tile time on the fused attention kernel, relative to a
+    bf16 tile (a skipped block: one column of a 128-block skip chunk)."""
+    return (0.008, 1.0 if low == LOW_FP8 else 1.1, 2.2, 1.0)
+
+
+def price_tiers(low: int, tier_cost=None):
     """(tier, eps, cost) of the tiers the low format provides, cheapest first;
-    eps None marks skip, whose error factor is the tile's delta (step 4')."""
-    skip, full = (TIER_SKIP, None, 0.0), (TIER_FULL, 2.0 ** -8, 4.0)
+    eps None marks skip, whose error factor is the tile's delta (step 4').
+    ``tier_cost`` by tier code (skip, low, res, full); None or all zero: the
+    defaults."""
+    if tier_cost is None or not any(tier_cost):
+        tier_cost = default_tier_cost(low)
+    c = [float(x) for x in tier_cost]
+    skip, full = (TIER_SKIP, None, c[TIER_SKIP]), (TIER_FULL, 2.0 ** -8, c[TIER_FULL])
     if low == LOW_NONE:
         return [skip, full]
     if low == LOW_FP8:
-        return [skip, (TIER_LOW, 2.0 ** -4, 2.0), full]
+        return [skip, (TIER_LOW, 2.0 ** -4, c[TIER_LOW]), full]
     if low == LOW_NVFP4:
-        return [skip, (TIER_LOW, 2.0 ** -2, 1.0), full]
+        return [skip, (TIER_LOW, 2.0 ** -2, c[TIER_LOW]), full]
     if low == LOW_NVFP4_RES:
-        return [skip, (TIER_LOW, 2.0 ** -2, 1.0), (TIER_RES, 2.0 ** -4, 3.0), full]
+        return [skip, (TIER_LOW, 2.0 ** -2, c[TIER_LOW]), (TIER_RES, 2.0 ** -4, c[TIER_RES]), full]
     raise ValueError("unknown low format")
 
 
 def assign_tiers_price(M_row: np.ndarray, delta_row: np.ndarray, price: float, low: int,
-                       diag=()):
+                       diag=(), tier_cost=None):
     """Tiers (uint8 [nKb]) and flags (bool [nKb]) of one row by the price rule."""
     n = M_row.shape[0]
-    table = price_tiers(low)
+    table = price_tiers(low, tier_cost)
     tiers = np.empty(n, dtype=np.uint8)
     flags = np.zeros(n, dtype=bool)
     for j in range(n):
@@ -241,7 +257,7 @@ def row_lists(tiers_row: np.ndarray, M_row: np.ndarray):
 
 def route_head(Qh, Kh, Vh, tau, block_q: int, block_k: int, scale: float = 0.0,
                keep_diag_full: bool = True, router: int = ROUTER_MASS, price: float = 0.0,
-               low: int = LOW_NVFP4, kappa: float = 1.0) -> dict:
+               low: int = LOW_NVFP4, kappa: float = 1.0, tier_cost=None) -> dict:
     """Router output for one head (fp64 values of bf16 Q, K, V [N, d]).
     ``router`` ROUTER_MASS uses ``tau`` (steps 4-5); ROUTER_PRICE uses
     ``price`` and the tiers of ``low`` (steps 4'-5'); ROUTER_ENTROPY uses
@@ -265,7 +281,7 @@ def route_head(Qh, Kh, Vh, tau, block_q: int, block_k: int, scale: float = 0.0,
     for i in range(nqb):
         diag = diag_blocks(i, block_q, block_k, N) if keep_diag_full else ()
         if router == ROUTER_PRICE:
-            tiers[i], flags[i] = assign_tiers_price(M[i], delta[i], price, low, diag)
+            tiers[i], flags[i] = assign_tiers_price(M[i], delta[i], price, low, diag, tier_cost)
         elif router == ROUTER_ENTROPY:
             tiers[i], flags[i], keep[i] = assign_tiers_entropy(M[i], tau, kappa, diag)
         else:

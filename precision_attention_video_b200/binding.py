@@ -40,6 +40,7 @@ class ta_params(ctypes.Structure):
         ("softmax_scale", ctypes.c_float), ("debug_flags", ctypes.c_int32),
         ("stride_b", ctypes.c_int64), ("stride_h", ctypes.c_int64), ("stride_n", ctypes.c_int64),
         ("router", ctypes.c_int32), ("price", ctypes.c_double), ("retention", ctypes.c_double),
+        ("tier_cost", ctypes.c_double * 4),
     ]
 
 
@@ -114,7 +115,8 @@ def make_params(B: int, H: int, N: int, d: int, block_q: int, block_k: int, low:
                 tau: Sequence[float], p_offset_log2: int, keep_diag_full: int = 1,
                 softmax_scale: float = 0.0, debug_flags: int = 0,
                 strides: Optional[Sequence[int]] = None, router: int = 0,
-                price: float = 0.0, retention: float = 1.0) -> ta_params:
+                price: float = 0.0, retention: float = 1.0,
+                tier_cost: Sequence[float] = (0.0, 0.0, 0.0, 0.0)) -> ta_params:
     """ta_params for a [B, H, N, d] layout (contiguous unless ``strides`` = (sb, sh, sn))."""
     p = ta_params()
     p.B, p.H, p.N, p.d = B, H, N, d
@@ -127,6 +129,8 @@ def make_params(B: int, H: int, N: int, d: int, block_q: int, block_k: int, low:
     sb, sh, sn = strides if strides is not None else (H * N * d, N * d, d)
     p.stride_b, p.stride_h, p.stride_n = sb, sh, sn
     p.router, p.price, p.retention = router, float(price), float(retention)
+    for i in range(4):
+        p.tier_cost[i] = float(tier_cost[i])   # by tier code; all zero: the library's defaults
     return p
 
 
@@ -135,7 +139,8 @@ def params_for(cfg, **overrides) -> ta_params:
     kw = dict(B=cfg.B, H=cfg.H, N=cfg.N, d=cfg.d, block_q=cfg.block_q, block_k=cfg.block_k,
               low=cfg.low, tau=cfg.tau, p_offset_log2=cfg.p_offset_log2,
               keep_diag_full=cfg.keep_diag_full, router=getattr(cfg, "router", 0),
-              price=getattr(cfg, "price", 0.0), retention=getattr(cfg, "kappa", 1.0))
+              price=getattr(cfg, "price", 0.0), retention=getattr(cfg, "kappa", 1.0),
+              tier_cost=getattr(cfg, "tier_cost", (0.0, 0.0, 0.0, 0.0)))
     kw.update(overrides)
     return make_params(**kw)
 

@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libtiered_attn.so")
 
-SOURCES = ["ta_api.cu", "ta_prep.cu", "ta_route.cu", "ta_attn.cu", "ta_static.cu"]
+SOURCES = ["ta_api.cu", "ta_prep.cu", "ta_route.cu", "ta_attn.cu", "ta_attn2.cu", "ta_static.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", INCLUDE, "-I", CSRC]

@@ -68,6 +68,9 @@ ta_status validate(const ta_params* p) {
     return TA_ERR_INVALID_ARG;
   if (p->router == TA_ROUTER_PRICE && !(std::isfinite(p->price) && p->price >= 0.0))
     return TA_ERR_INVALID_ARG;
+  if (p->router == TA_ROUTER_PRICE)
+    for (int i = 0; i < 4; ++i)
+      if (!(std::isfinite(p->tier_cost[i]) && p->tier_cost[i] >= 0.0)) return TA_ERR_INVALID_ARG;
   const Shape s = shape_of(p);
   if (s.nKb > ta::kMaxKeyBlocks) return TA_ERR_UNSUPPORTED;
   if ((int64_t)p->B * p->H > 65535 || s.nQb > 2147483647) return TA_ERR_UNSUPPORTED;
@@ -169,6 +172,25 @@ ta_status check_tensor(const void* ptr) {
   return (ptr && aligned(ptr, 16)) ? TA_OK : TA_ERR_INVALID_ARG;
 }
 
+}  // namespace
+
+// The price router's tier costs: the caller's, or the measured defaults when
+// all four are zero.
+void ta_resolve_tier_cost(const ta_params* p, double* cost) {
+  bool given = false;
+  for (int i = 0; i < 4; ++i) given = given || p->tier_cost[i] != 0.0;
+  if (given) {
+    for (int i = 0; i < 4; ++i) cost[i] = p->tier_cost[i];
+    return;
+  }
+  cost[TA_TIER_SKIP] = TA_TIER_COST_SKIP;
+  cost[TA_TIER_LOW] = p->low == TA_LOW_FP8_E4M3 ? TA_TIER_COST_FP8 : TA_TIER_COST_NVFP4;
+  cost[TA_TIER_RES] = TA_TIER_COST_NVFP4_RES;
+  cost[TA_TIER_FULL] = TA_TIER_COST_FULL;
+}
+
+namespace {
+
 void fill_plan_args(const ta_params* p, const void* Q, const void* K, const void* V, void* ws,
                     ta::PlanArgs& a) {
   const Shape s = shape_of(p);
@@ -195,6 +217,7 @@ void fill_plan_args(const ta_params* p, const void* Q, const void* K, const void
   a.keep_diag = p->keep_diag_full;
   a.router = p->router;
   a.price = p->price;
+  ta_resolve_tier_cost(p, a.cost);
   a.retention = p->retention;
   a.scale = p->softmax_scale > 0.0f ? (double)p->softmax_scale : 1.0 / std::sqrt((double)p->d);
   a.status = at<int>(ws, L.status);
@@ -427,6 +450,7 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
   a.row_counts = at<int>(ws, L.row_counts);
   a.row_lists = at<int>(ws, L.row_lists);
   a.O = static_cast<__nv_bfloat16*>(O);
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
   a.Np = (int)s.Np;
   a.q_sf = fp4 ? at<uint8_t>(ws, L.q_scales) : nullptr;
   a.k_sf = fp4 ? at<uint8_t>(ws, L.k_scales) : nullptr;

@@ -869,6 +869,9 @@ cudaError_t launch_d(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s)
 }  // namespace
 
 cudaError_t launch_attn(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
+  // d = 128 with 128 x 128 tiles runs on the two-group kernel (ta_attn2.cu)
+  const cudaError_t e2 = launch_attn2(a, maps, s);
+  if (e2 != cudaErrorNotSupported) return e2;
   if (a.d == 64 && a.bk == 64) return launch_d<64, 64, LM_IMAGE>(a, maps, s);
   if (a.d == 64 && a.bk == 128) return launch_d<64, 128, LM_IMAGE>(a, maps, s);
   if (a.d == 128 && a.bk == 64) return launch_d<128, 64, LM_IMAGE>(a, maps, s);

@@ -38,6 +38,34 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^x for two floats on the FMA pipe, leaving the MUFU unit to ex2.approx:
+// x = j + f with j = rint(x) from the magic-number addition (x + 1.5 * 2^23
+// rounds to an integer in the low mantissa bits), 2^f for f in [-1/2, 1/2]
+// by the cubic 1 + f (c1 + f (c2 + f c3)), and j added into the exponent
+// field of the result.  The coefficients are a minimax fit of our own
+// (Lawson's iteratively reweighted least squares on the relative error, with
+// p(0) = 1 so that integer arguments give exact powers of two): relative
+// error <= 1.02e-4 in fp32.  x is clamped below at -125 (masked columns
+// arrive as -inf and come out as 2^-125, which no sum or rounding of P'
+// against a row maximum of 2^o notices).
+__device__ __forceinline__ void exp2_poly2(float a0, float a1, float& y0, float& y1) {
+  constexpr float kMagic = 12582912.0f;
+  const float x0 = fmaxf(a0, -125.0f), x1 = fmaxf(a1, -125.0f);
+  const uint64_t x = pack2(x0, x1);
+  const uint64_t t = add2(x, pack2(kMagic, kMagic));
+  const uint64_t j = add2(t, pack2(-kMagic, -kMagic));
+  const uint64_t f = fma2(j, pack2(-1.0f, -1.0f), x);
+  uint64_t p = fma2(f, pack2(0.055008940398693085f, 0.055008940398693085f),
+                    pack2(0.2422109991312027f, 0.2422109991312027f));
+  p = fma2(f, p, pack2(0.6932829022407532f, 0.6932829022407532f));
+  p = fma2(f, p, pack2(1.0f, 1.0f));
+  float p0, p1, t0, t1;
+  unpack2(p, p0, p1);
+  unpack2(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -109,6 +137,29 @@ __device__ __forceinline__ uint32_t nvfp4_quant32(const float* x, const float2* 
     for (int i = 0; i < 16; ++i) am[i & 3] = fmaxf(am[i & 3], x[g * 16 + i]);
     const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
     const uint32_t scc = cvt_e4m3x2(div6(amax), 0.0f) & 0xFFu;
+    const float inv = sc_tab[scc].y;
+    scw |= scc << (8 * g);
+    const uint64_t inv2 = pack2(inv, inv);
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      float y[8];
+#pragma unroll
+      for (int i = 0; i < 8; i += 2)
+        unpack2(mul2(pack2(x[g * 16 + w * 8 + i], x[g * 16 + w * 8 + i + 1]), inv2), y[i], y[i + 1]);
+      p[g * 2 + w] = cvt_e2m1x8(y);
+    }
+  }
+  return scw;
+}
+
+// The same, with each group's amax given (the P' of its largest S, taken
+// from the maximum pass): no maximum over the 16 values here.
+__device__ __forceinline__ uint32_t nvfp4_quant32_am(const float* x, float am0, float am1,
+                                                     const float2* sc_tab, uint32_t* p) {
+  uint32_t scw = 0u;
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const uint32_t scc = cvt_e4m3x2(div6(g ? am1 : am0), 0.0f) & 0xFFu;
     const float inv = sc_tab[scc].y;
     scw |= scc << (8 * g);
     const uint64_t inv2 = pack2(inv, inv);

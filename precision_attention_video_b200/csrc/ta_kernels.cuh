@@ -26,6 +26,7 @@ struct PlanArgs {
   int keep_diag;
   int router;                   // ta_router
   double price;                 // TA_ROUTER_PRICE's price
+  double cost[4];               // TA_ROUTER_PRICE's tier costs by tier code (defaults resolved)
   double retention;             // TA_ROUTER_ENTROPY's kappa
   double scale;                 // softmax scale (fp64 in the router)
   int* status;
@@ -53,11 +54,12 @@ struct PlanArgs {
 struct AttnArgs {
   int B, H, N, d, bq, bk, low;
   int nQb, nKb;
-  int64_t sb, sh, sn;           // element strides of O
+  int64_t sb, sh, sn;           // element strides of Q and O
   float scale_log2;             // softmax_scale * log2(e)
   int p_offset;                 // o of P' = 2^o exp(s - m)
   int debug_flags;
   int* status;
+  const __nv_bfloat16* Q;       // queries [B, H, N, d] (strides sb, sh, sn)
   const __nv_bfloat16* kbar_b;  // skip pseudo-keys [BH, nKb, d]
   const __nv_bfloat16* vbar_b;
   const int* row_counts;
@@ -82,5 +84,8 @@ struct AttnArgs {
 cudaError_t launch_prep(const PlanArgs& a, cudaStream_t s);
 cudaError_t launch_route(const PlanArgs& a, cudaStream_t s);
 cudaError_t launch_attn(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s);
+// The two-group kernel (d = 128, 128 x 128 tiles); cudaErrorNotSupported for
+// other shapes.
+cudaError_t launch_attn2(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s);
 
 }  // namespace ta

@@ -95,11 +95,12 @@ __global__ void __launch_bounds__(256) logits_kernel(const PlanArgs a) {
 // The price router's tier of one tile: the least predicted error + price *
 // cost among the tiers the low format provides, cheapest first, keeping the
 // cheaper tier on a tie.  Error = M * eps (eps: the tier's unit roundoff; for
-// skip, the tile's spread delta); cost = tensor-pipe time relative to an
-// NVFP4 tile.
-__device__ __forceinline__ int price_tier(double M, double delta, double price, int low) {
+// skip, the tile's spread delta); cost = the tier's per-tile time (ta_params
+// tier_cost, by default as measured on the fused kernel).
+__device__ __forceinline__ int price_tier(double M, double delta, double price, int low,
+                                          double c_skip, double c_low, double c_res, double c_full) {
   int best = TA_TIER_SKIP;
-  double obj = M * delta;
+  double obj = M * delta + price * c_skip;
   auto consider = [&](int tier, double eps, double cost) {
     const double o = M * eps + price * cost;
     if (o < obj) {
@@ -107,10 +108,10 @@ __device__ __forceinline__ int price_tier(double M, double delta, double price, 
       best = tier;
     }
   };
-  if (low == TA_LOW_FP8_E4M3) consider(TA_TIER_LOW, 0.0625, 2.0);
-  if (low == TA_LOW_NVFP4 || low == TA_LOW_NVFP4_RES) consider(TA_TIER_LOW, 0.25, 1.0);
-  if (low == TA_LOW_NVFP4_RES) consider(TA_TIER_RES, 0.0625, 3.0);
-  consider(TA_TIER_FULL, 0.00390625, 4.0);
+  if (low == TA_LOW_FP8_E4M3) consider(TA_TIER_LOW, 0.0625, c_low);
+  if (low == TA_LOW_NVFP4 || low == TA_LOW_NVFP4_RES) consider(TA_TIER_LOW, 0.25, c_low);
+  if (low == TA_LOW_NVFP4_RES) consider(TA_TIER_RES, 0.0625, c_res);
+  consider(TA_TIER_FULL, 0.00390625, c_full);
   return best;
 }
 
@@ -244,7 +245,8 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs 
       idx[k] = j;
       a.mass[g * nKb + j] = m;
       if (a.router == TA_ROUTER_PRICE)
-        tier[j] = (uint8_t)price_tier(m, a.spread[g * nKb + j], a.price, a.low);
+        tier[j] = (uint8_t)price_tier(m, a.spread[g * nKb + j], a.price, a.low, a.cost[TA_TIER_SKIP],
+                                      a.cost[TA_TIER_LOW], a.cost[TA_TIER_RES], a.cost[TA_TIER_FULL]);
     } else {
       key[k] = -1.0;
       idx[k] = 0x7fffffff - (sortn - j);

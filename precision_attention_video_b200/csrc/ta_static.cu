@@ -44,6 +44,8 @@ inline size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 }  // namespace
 
+void ta_resolve_tier_cost(const ta_params* p, double* cost);
+
 extern "C" ta_status tiered_attn_route_noalloc(const ta_params* p, const void* Q, const void* K,
                                                const void* V, uint8_t* tier_map,
                                                int32_t* row_counts, int32_t* row_lists,
@@ -104,6 +106,7 @@ extern "C" ta_status tiered_attn_route_noalloc(const ta_params* p, const void* Q
   a.keep_diag = p->keep_diag_full;
   a.router = p->router;
   a.price = p->price;
+  ta_resolve_tier_cost(p, a.cost);
   a.retention = p->retention;
   a.scale = p->softmax_scale > 0.0f ? (double)p->softmax_scale : 1.0 / std::sqrt((double)p->d);
   a.status = reinterpret_cast<int*>(base + off[0]);

@@ -59,7 +59,8 @@ def unpack_fp4(packed: np.ndarray) -> np.ndarray:
 def router_kwargs(cfg, low=None):
     """route_head keywords of the workload's router (mass thresholds or price)."""
     return {"router": getattr(cfg, "router", 0), "price": getattr(cfg, "price", 0.0),
-            "low": cfg.low if low is None else low, "kappa": getattr(cfg, "kappa", 1.0)}
+            "low": cfg.low if low is None else low, "kappa": getattr(cfg, "kappa", 1.0),
+            "tier_cost": getattr(cfg, "tier_cost", None)}
 
 
 def oracle_head(cfg, Q, K, V, b, h, qblocks=None, exact=False, tau=None, low=None,

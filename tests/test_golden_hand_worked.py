@@ -165,9 +165,11 @@ def test_price_and_entropy_router_rows_hand_worked(case):
         rows = np.arange(j * block, (j + 1) * block)
         K[rows, 0] = math.log(w[j]) + np.where(rows % 2 == 0, b[j], -b[j])
     np.testing.assert_allclose(R.block_spread(K, block)[:, 0], np.square(b), rtol=1e-12, atol=1e-15)
-    if case == "price":
+    if case.startswith("price"):
+        cost = None if sec["cost"] == "default" else _nums(sec["cost"])
         rt = R.route_head(Q, K, np.zeros((N, 1)), (0.5, 0.9), block, block, scale=1.0,
-                          router=R.ROUTER_PRICE, price=float(sec["price"]), low=LOW_NVFP4)
+                          router=R.ROUTER_PRICE, price=float(sec["price"]), low=LOW_NVFP4,
+                          tier_cost=cost)
         np.testing.assert_allclose(rt["delta"][0], b, rtol=1e-12, atol=1e-15)
     else:
         rt = R.route_head(Q, K, np.zeros((N, 1)), _nums(sec["tau"]), block, block, scale=1.0,

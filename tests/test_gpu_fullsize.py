@@ -67,7 +67,8 @@ def _check_head(cfg, Q, K, V, views, O, h, qblocks):
     return assert_out_close(to64(O[0, h].cpu()), Oref, f"{cfg.name} head {h}")
 
 
-@pytest.mark.parametrize("name", ["480p", "sweep70", "720p", "480p-price", "480p-entropy"])
+@pytest.mark.parametrize("name", ["480p", "sweep0", "sweep30", "sweep50", "sweep70", "sweep90", "720p",
+                                  "480p-price", "480p-entropy"])
 def test_fullsize_sampled_parity(cuda_ok, name):
     cfg, Q, K, V, views, O = _run_full(name)
     nqb = cfg.n_qb

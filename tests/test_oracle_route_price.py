@@ -115,15 +115,22 @@ def test_tiers_fall_monotonically_with_price():
     assert prev.max() == 0
 
 
-def test_no_move_pays_at_the_price():
+@pytest.mark.parametrize("tier_cost,n_tiers,prices", [
+    # nominal tensor-pipe rates: every tier has a use
+    ((0.0, 1.0, 3.0, 4.0), 3, (3e-3, 1e-2, 2e-2, 3e-2)),
+    # the defaults (measured kernel time): NVFP4 and the residual tier cost
+    # more than bf16, only skip and full pay
+    (None, 2, (3e-2, 0.1, 0.3, 1.0)),
+])
+def test_no_move_pays_at_the_price(tier_cost, n_tiers, prices):
     Q, K, V = _random(640, 32, seed=5)
     low = Qz.LOW_NVFP4_RES
-    table = R.price_tiers(low)
+    table = R.price_tiers(low, tier_cost)
     cost = [c for _, _, c in table]
     seen = set()
-    for price in (3e-3, 1e-2, 2e-2, 3e-2):
+    for price in prices:
         rt = R.route_head(Q, K, V, None, 64, 64, router=R.ROUTER_PRICE, price=price, low=low,
-                          keep_diag_full=False)
+                          keep_diag_full=False, tier_cost=tier_cost)
         M, delta, tiers = rt["M"], rt["delta"], rt["tiers"]
         for i in range(M.shape[0]):
             for j in range(M.shape[1]):
@@ -135,4 +142,4 @@ def test_no_move_pays_at_the_price():
                         assert err[k] - err[t] <= price * (cost[t] - cost[k]) * (1 + 1e-12)
                     elif cost[t] < cost[k]:  # cheaper: it would lose more error than the compute it saves
                         assert err[t] - err[k] > price * (cost[k] - cost[t]) * (1 - 1e-12)
-    assert len(seen) >= 3   # the prices above spread tiles over several tiers
+    assert len(seen) >= n_tiers   # the prices above spread tiles over several tiers
