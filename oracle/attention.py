@@ -31,6 +31,13 @@ block's tile list), in fp64, starting from m = -inf, l = 0, acc = 0:
     w_j = n_j 2^o exp(s_j - m');  l += sum w_j;  acc += bf16(w_j) bf16(vbar_j)
 * O = acc / l.
 
+Finer key granularity ("FG-Attn", searcharxiv author page, abstract: skip
+score computation at M x N sub-tiles, M >= 16 queries, N >= 1 keys): with
+narrow key blocks (block_k = 32) the kept blocks of one tier are taken
+``key_pack`` at a time in list order, their keys side by side, as one tile:
+one running-max update per tile, NVFP4 groups of P' starting at each block's
+first key (a block's real keys only), skipped blocks unchanged.
+
 Readings: the tier order (full, residual, low, skip) and the descending-mass
 order inside a tier put the running max near its final value before any P'
 is quantised; the denominator sums P' before
@@ -62,7 +69,7 @@ def nvfp4_along_keys(P: np.ndarray) -> np.ndarray:
     return nvfp4_dequant_groups(codes, sc).reshape(rows, npad)[:, :nk]
 
 
-def _qblock(i, Qh, Kh, Vh, rt, qt, low, Bq, Bk, o, scale, exact):
+def _qblock(i, Qh, Kh, Vh, rt, qt, low, Bq, Bk, o, scale, exact, pack):
     N = Qh.shape[0]
     r0, r1 = i * Bq, min(N, (i + 1) * Bq)
     q = Qh[r0:r1]
@@ -75,15 +82,20 @@ def _qblock(i, Qh, Kh, Vh, rt, qt, low, Bq, Bk, o, scale, exact):
     lst = rt["lists"][i]
     pos = 0
     for tier, cnt in ((TIER_FULL, counts[0]), (TIER_RES, counts[1]), (TIER_LOW, counts[2])):
-        for j in lst[pos:pos + cnt]:
-            k0, k1 = j * Bk, min(N, (j + 1) * Bk)
+        tier_blocks = lst[pos:pos + cnt]
+        for g0 in range(0, cnt, pack):
+            # one tile: `pack` consecutive list entries of the tier, their
+            # keys side by side (segments in list order)
+            segs = [(j * Bk, min(N, (j + 1) * Bk)) for j in tier_blocks[g0:g0 + pack]]
+            keys = np.concatenate([np.arange(k0, k1) for k0, k1 in segs])
+            cuts = np.cumsum([0] + [k1 - k0 for k0, k1 in segs])
             if tier == TIER_FULL:
-                s = (q @ Kh[k0:k1].T) * scale
+                s = (q @ Kh[keys].T) * scale
             elif tier == TIER_LOW:
-                s = (qt["dq"][r0:r1] @ qt["dk"][k0:k1].T) * scale
+                s = (qt["dq"][r0:r1] @ qt["dk"][keys].T) * scale
             else:
                 a1, a2 = qt["dq"][r0:r1], qt["rq"][r0:r1]
-                b1, b2 = qt["dk"][k0:k1], qt["rk"][k0:k1]
+                b1, b2 = qt["dk"][keys], qt["rk"][keys]
                 s = (a1 @ b1.T + a1 @ b2.T + a2 @ b1.T) * scale
             m_new = np.maximum(m, s.max(axis=1))
             alpha = np.exp(m - m_new)
@@ -91,19 +103,25 @@ def _qblock(i, Qh, Kh, Vh, rt, qt, low, Bq, Bk, o, scale, exact):
             acc *= alpha[:, None]
             P = two_o * np.exp(s - m_new[:, None])
             l += P.sum(axis=1)
+
+            def fp4(X):
+                # NVFP4 groups of 16 keys start at each key block's first key
+                return np.concatenate([nvfp4_along_keys(X[:, cuts[u]:cuts[u + 1]])
+                                       for u in range(len(segs))], axis=1)
+
             if tier == TIER_FULL:
-                acc += (P if exact else bf16_rne(P)) @ Vh[k0:k1]
+                acc += (P if exact else bf16_rne(P)) @ Vh[keys]
             elif tier == TIER_LOW and low == LOW_FP8:
-                acc += (P if exact else e4m3_round(P)) @ qt["dv"][k0:k1]
+                acc += (P if exact else e4m3_round(P)) @ qt["dv"][keys]
             elif tier == TIER_LOW:
-                acc += (P if exact else nvfp4_along_keys(P)) @ qt["dv"][k0:k1]
+                acc += (P if exact else fp4(P)) @ qt["dv"][keys]
             else:
-                v1, v2 = qt["dv"][k0:k1], qt["rv"][k0:k1]
+                v1, v2 = qt["dv"][keys], qt["rv"][keys]
                 if exact:
                     p1, p2 = P, np.zeros_like(P)
                 else:
-                    p1 = nvfp4_along_keys(P)
-                    p2 = nvfp4_along_keys(fp32_rne(P - p1))
+                    p1 = fp4(P)
+                    p2 = fp4(fp32_rne(P - p1))
                 acc += p1 @ v1 + p1 @ v2 + p2 @ v1
             m = m_new
         pos += cnt
@@ -121,8 +139,9 @@ def _qblock(i, Qh, Kh, Vh, rt, qt, low, Bq, Bk, o, scale, exact):
 
 
 def tiered_attention_head(Qh, Kh, Vh, rt, qt, low, block_q, block_k, p_offset_log2,
-                          scale=0.0, exact=False, qblocks=None, threads=1):
-    """O [N, d] (fp64) of one head; rows of q-blocks not in ``qblocks`` are NaN."""
+                          scale=0.0, exact=False, qblocks=None, threads=1, key_pack=1):
+    """O [N, d] (fp64) of one head; rows of q-blocks not in ``qblocks`` are NaN.
+    ``key_pack`` key blocks of one tier share a tile (one running-max update)."""
     N, d = Qh.shape
     if scale == 0.0:
         scale = 1.0 / math.sqrt(d)
@@ -130,7 +149,7 @@ def tiered_attention_head(Qh, Kh, Vh, rt, qt, low, block_q, block_k, p_offset_lo
     if qblocks is None:
         qblocks = range(nqb)
     O = np.full((N, d), np.nan)
-    args = (Qh, Kh, Vh, rt, qt, low, block_q, block_k, p_offset_log2, scale, exact)
+    args = (Qh, Kh, Vh, rt, qt, low, block_q, block_k, p_offset_log2, scale, exact, key_pack)
     if threads > 1:
         with ThreadPoolExecutor(max_workers=threads) as ex:
             results = list(ex.map(lambda i: _qblock(i, *args), qblocks))
@@ -143,7 +162,7 @@ def tiered_attention_head(Qh, Kh, Vh, rt, qt, low, block_q, block_k, p_offset_lo
 
 def tiered_attention(Q, K, V, tau, low, block_q, block_k, p_offset_log2, scale=0.0,
                      keep_diag_full=True, exact=False, heads=None, qblocks=None, threads=1,
-                     router=0, price=0.0, kappa=1.0):
+                     router=0, price=0.0, kappa=1.0, key_pack=1):
     """Route, quantise and attend over every (b, h) in ``heads`` (default all).
 
     Q, K, V: fp64 arrays [B, H, N, d] holding bf16 values.  Returns a dict
@@ -157,7 +176,7 @@ def tiered_attention(Q, K, V, tau, low, block_q, block_k, p_offset_log2, scale=0
                         router=router, price=price, low=low, kappa=kappa)
         qt = quantize_head(Q[b, h], K[b, h], V[b, h], low, block_q, block_k)
         O = tiered_attention_head(Q[b, h], K[b, h], V[b, h], rt, qt, low, block_q, block_k,
-                                  p_offset_log2, rt["scale"], exact, qblocks, threads)
+                                  p_offset_log2, rt["scale"], exact, qblocks, threads, key_pack)
         out[(b, h)] = {"route": rt, "quant": qt, "O": O}
     return out
 

@@ -197,3 +197,76 @@ def test_fine_grained_key_blocks_of_32():
     # (3) the diagonal of a 128-row query block covers four 32-key blocks
     assert R.diag_blocks(1, bq, bk, N) == [4, 5, 6, 7]
     assert all((rt["tiers"][1, 4:8] == R.TIER_FULL))
+
+
+def _expand_plan(rt, sub, nb_sub):
+    """The plan of 128-key blocks rewritten over key blocks `sub` times
+    narrower: block j becomes blocks sub*j .. sub*j + sub - 1, same tier,
+    same list position."""
+    counts = rt["counts"] * 0
+    lists = []
+    for i in range(len(rt["counts"])):
+        row, pos = [], 0
+        for t in range(4):
+            c = int(rt["counts"][i][t])
+            blocks = [sub * j + u for j in rt["lists"][i][pos:pos + c] for u in range(sub)
+                      if sub * j + u < nb_sub]
+            counts[i][t] = len(blocks)
+            row += blocks
+            pos += c
+        lists.append(row)
+    return {"counts": counts, "lists": np.array(lists, dtype=np.int32), "n_k": None}
+
+
+@pytest.mark.parametrize("low,tau", [(Qz.LOW_NVFP4, (0.5, 2.0)), (Qz.LOW_NVFP4_RES, (0.3, 0.6, 2.0))])
+def test_key_pack_of_narrow_blocks_equals_one_wide_block(low, tau):
+    # A tile that packs the four 32-key blocks of one 128-key block computes
+    # what the 128-key tile does: the same keys, one running-max update, P'
+    # groups of 16 keys from the same starts.  Rounded P', ragged 24-key tail.
+    rng = np.random.default_rng(21)
+    N, d, bq = 376, 32, 128
+    Q, K, V = (F.bf16_rne(rng.normal(size=(N, d)) * 2) for _ in range(3))
+    rt = R.route_head(Q, K, V, tau, bq, 128)
+    assert (rt["tiers"] != R.TIER_SKIP).all() and (rt["tiers"] != R.TIER_FULL).any()
+    qt = Qz.quantize_head(Q, K, V, low, bq, 128)
+    qt32 = Qz.quantize_head(Q, K, V, low, bq, 32)
+    for key in ("dq", "dk", "dv"):
+        np.testing.assert_array_equal(qt[key], qt32[key])
+    wide = tiered_attention_head(Q, K, V, rt, qt, low, bq, 128, 11, rt["scale"], False)
+    rt32 = _expand_plan(rt, 4, -(-N // 32))
+    narrow = tiered_attention_head(Q, K, V, rt32, qt32, low, bq, 32, 11, rt["scale"], False,
+                                   key_pack=4)
+    one_by_one = tiered_attention_head(Q, K, V, rt32, qt32, low, bq, 32, 11, rt["scale"], False)
+    assert _rel(narrow, wide) <= 1e-12
+    assert _rel(one_by_one, wide) > 1e-6      # the grouping is what makes them equal
+
+
+def test_key_pack_order_inside_a_tile_is_immaterial():
+    # Within one packed tile the order of its key blocks changes neither the
+    # running maximum nor any P' group (groups start at each block's first
+    # key), so reversing every pack changes only summation order -- also when
+    # the ragged 24-key block moves from the end of a pack to its front.
+    rng = np.random.default_rng(22)
+    N, d, bq, bk = 376, 32, 128, 32
+    Q, K, V = (F.bf16_rne(rng.normal(size=(N, d)) * 2) for _ in range(3))
+    low = Qz.LOW_NVFP4
+    rt = R.route_head(Q, K, V, (0.3, 2.0), bq, bk)
+    qt = Qz.quantize_head(Q, K, V, low, bq, bk)
+    rev = dict(rt)
+    lists = rt["lists"].copy()
+    moved = False
+    for i in range(len(lists)):
+        pos = 0
+        for t in range(3):
+            c = int(rt["counts"][i][t])
+            for g0 in range(pos, pos + c, 4):
+                g1 = min(pos + c, g0 + 4)
+                if g1 - g0 > 1 and lists[i][g1 - 1] == 11:
+                    moved = True
+                lists[i][g0:g1] = lists[i][g0:g1][::-1].copy()
+            pos += c
+    rev["lists"] = lists
+    assert moved
+    a = tiered_attention_head(Q, K, V, rt, qt, low, bq, bk, 11, rt["scale"], False, key_pack=4)
+    b = tiered_attention_head(Q, K, V, rev, qt, low, bq, bk, 11, rt["scale"], False, key_pack=4)
+    assert _rel(a, b) <= 1e-12
