@@ -33,58 +33,76 @@ namespace {
 // Pooled logits: logits[bh, i, j] = scale * sum_c qbar[bh, i, c] kbar[bh, j, c]
 // and, for the price router, the skip tier's error factor
 // spread[bh, i, j] = scale * sqrt(sum_c (qbar[bh, i, c]^2 + qvar[bh, i, c]) kvar[bh, j, c]).
-// 32 x 32 output tile per CTA, 2 x 2 per thread, d staged 32 at a time.
+// 64 x 64 output tile per CTA, 4 x 4 per thread (rows ty + 16 u, columns
+// tx + 16 v, so that a warp's 16 tx read 16 consecutive doubles: no bank
+// conflicts), d staged 16 at a time.
 // ---------------------------------------------------------------------------
+constexpr int kLT = 64, kLC = 16;
+
 __global__ void __launch_bounds__(256) logits_kernel(const PlanArgs a) {
-  __shared__ double qs[32][33];
-  __shared__ double ks[32][33];
-  __shared__ double vs[32][33];
-  __shared__ double qw[32][33];   // qbar^2 + qvar (price router)
+  __shared__ double qs[kLC][kLT];
+  __shared__ double ks[kLC][kLT];
+  __shared__ double qw[kLC][kLT];   // qbar^2 + qvar (price router)
+  __shared__ double vs[kLC][kLT];   // kvar (price router)
   const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
-  const int bh = blockIdx.z, i0 = blockIdx.x * 32, j0 = blockIdx.y * 32;
+  const int bh = blockIdx.z, i0 = blockIdx.x * kLT, j0 = blockIdx.y * kLT;
   const int D = a.d;
   const double* qb = a.qbar + (int64_t)bh * a.nQb * D;
   const double* kb = a.kbar + (int64_t)bh * a.nKb * D;
   const double* kvb = a.kvar ? a.kvar + (int64_t)bh * a.nKb * D : nullptr;
   const double* qvb = a.qvar ? a.qvar + (int64_t)bh * a.nQb * D : nullptr;
-  double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
-  double spr[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
-  for (int c0 = 0; c0 < D; c0 += 32) {
-    for (int e = tid; e < 32 * 32; e += 256) {
-      const int r = e / 32, c = e % 32;
-      qs[r][c] = (i0 + r < a.nQb) ? qb[(int64_t)(i0 + r) * D + c0 + c] : 0.0;
-      ks[r][c] = (j0 + r < a.nKb) ? kb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
+  double acc[4][4], spr[4][4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = spr[u][v] = 0.0;
+  for (int c0 = 0; c0 < D; c0 += kLC) {
+    // stage 64 rows x 16 coordinates of each operand: element e = r * 16 + c
+    for (int e = tid; e < kLT * kLC; e += 256) {
+      const int r = e / kLC, c = e % kLC;
+      const bool qi = i0 + r < a.nQb, kj = j0 + r < a.nKb;
+      const double q = qi ? qb[(int64_t)(i0 + r) * D + c0 + c] : 0.0;
+      qs[c][r] = q;
+      ks[c][r] = kj ? kb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
       if (kvb) {
-        vs[r][c] = (j0 + r < a.nKb) ? kvb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
-        qw[r][c] = (i0 + r < a.nQb) ? qs[r][c] * qs[r][c] + qvb[(int64_t)(i0 + r) * D + c0 + c] : 0.0;
+        vs[c][r] = kj ? kvb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
+        qw[c][r] = qi ? q * q + qvb[(int64_t)(i0 + r) * D + c0 + c] : 0.0;
       }
     }
     __syncthreads();
-#pragma unroll 8
-    for (int c = 0; c < 32; ++c) {
-      const double q0 = qs[ty * 2][c], q1 = qs[ty * 2 + 1][c];
-      const double k0 = ks[tx * 2][c], k1 = ks[tx * 2 + 1][c];
-      acc[0][0] += q0 * k0;
-      acc[0][1] += q0 * k1;
-      acc[1][0] += q1 * k0;
-      acc[1][1] += q1 * k1;
+#pragma unroll 4
+    for (int c = 0; c < kLC; ++c) {
+      double q[4], k[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) q[u] = qs[c][ty + 16 * u];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) k[v] = ks[c][tx + 16 * v];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fma(q[u], k[v], acc[u][v]);
     }
     if (kvb) {
-#pragma unroll 8
-      for (int c = 0; c < 32; ++c) {
-        const double w0 = qw[ty * 2][c], w1 = qw[ty * 2 + 1][c];
-        const double v0 = vs[tx * 2][c], v1 = vs[tx * 2 + 1][c];
-        spr[0][0] += w0 * v0;
-        spr[0][1] += w0 * v1;
-        spr[1][0] += w1 * v0;
-        spr[1][1] += w1 * v1;
+#pragma unroll 4
+      for (int c = 0; c < kLC; ++c) {
+        double w[4], k[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) w[u] = qw[c][ty + 16 * u];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) k[v] = vs[c][tx + 16 * v];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) spr[u][v] = fma(w[u], k[v], spr[u][v]);
       }
     }
     __syncthreads();
   }
-  for (int u = 0; u < 2; ++u)
-    for (int v = 0; v < 2; ++v) {
-      const int i = i0 + ty * 2 + u, j = j0 + tx * 2 + v;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int i = i0 + ty + 16 * u, j = j0 + tx + 16 * v;
       if (i < a.nQb && j < a.nKb) {
         a.logits[((int64_t)bh * a.nQb + i) * a.nKb + j] = acc[u][v] * a.scale;
         if (kvb) a.spread[((int64_t)bh * a.nQb + i) * a.nKb + j] = a.scale * sqrt(spr[u][v]);
@@ -320,10 +338,226 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(const PlanArgs 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Per-row routing for long rows (more than 256 key blocks), one CTA per
+// (bh, query block): the same steps as route_kernel, with the row held in
+// shared memory and the (-M, j) sort, the exclusive prefix of the sorted
+// masses and the list compaction done by the whole CTA.  A warp with 32
+// elements a lane (route_kernel<32>) needs 159 registers and runs one CTA
+// per SM; here many rows are in flight on each SM.
+// ---------------------------------------------------------------------------
+constexpr int kRowThreads = 256;
+
+// Block-wide exclusive prefix sum of one value per thread; `total` gets the sum.
+__device__ __forceinline__ double block_excl_scan(double v, double* wsum, double& total) {
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  double incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  double base = 0.0, tot = 0.0;
+  for (int w = 0; w < kRowThreads / 32; ++w) {
+    const double x = wsum[w];
+    if (w < warp) base += x;
+    tot += x;
+  }
+  __syncthreads();
+  total = tot;
+  return base + incl - v;
+}
+__device__ __forceinline__ int block_excl_scan_int(int v, int* wsum, int& total) {
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int base = 0, tot = 0;
+  for (int w = 0; w < kRowThreads / 32; ++w) {
+    const int x = wsum[w];
+    if (w < warp) base += x;
+    tot += x;
+  }
+  __syncthreads();
+  total = tot;
+  return base + incl - v;
+}
+__device__ __forceinline__ double block_reduce(double v, double* wsum, bool is_max) {
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double y = __shfl_xor_sync(0xffffffffu, v, o);
+    v = is_max ? fmax(v, y) : v + y;
+  }
+  if (lane == 0) wsum[warp] = v;
+  __syncthreads();
+  double r = is_max ? -INFINITY : 0.0;
+  for (int w = 0; w < kRowThreads / 32; ++w) r = is_max ? fmax(r, wsum[w]) : r + wsum[w];
+  __syncthreads();
+  return r;
+}
+
+// EPT: elements a thread owns (sortn = kRowThreads * EPT, a power of two).
+template <int EPT>
+__global__ void __launch_bounds__(kRowThreads) route_row_kernel(const PlanArgs a) {
+  constexpr int sortn = kRowThreads * EPT;
+  __shared__ double key[sortn];
+  __shared__ int idx[sortn];
+  __shared__ uint8_t tier[sortn];
+  __shared__ double wsum_d[kRowThreads / 32];
+  __shared__ int wsum_i[kRowThreads / 32];
+  const int tid = threadIdx.x;
+  const int64_t g = blockIdx.x;   // global row (bh, i)
+  const int i = (int)(g % a.nQb);
+  const int nKb = a.nKb;
+  const double* lrow = a.logits + g * nKb;
+
+  // pooled block softmax weighted by key counts; thread tid owns elements
+  // tid * EPT .. (contiguous), which also makes the prefix scan below a
+  // scan over threads
+  double mx = -INFINITY;
+  for (int e = 0; e < EPT; ++e) {
+    const int j = tid * EPT + e;
+    const double v = j < nKb ? lrow[j] : -INFINITY;
+    key[j] = v;
+    mx = fmax(mx, v);
+  }
+  mx = block_reduce(mx, wsum_d, true);
+  double part = 0.0;
+  for (int e = 0; e < EPT; ++e) {
+    const int j = tid * EPT + e;
+    if (j < nKb) {
+      const int nj = min(a.bk, a.N - j * a.bk);
+      const double w = (double)nj * exp(key[j] - mx);
+      key[j] = w;
+      part += w;
+    }
+  }
+  const double total = block_reduce(part, wsum_d, false);
+  int keep = nKb;
+  if (a.router == TA_ROUTER_ENTROPY) {
+    double hp = 0.0;
+    for (int e = 0; e < EPT; ++e) {
+      const int j = tid * EPT + e;
+      if (j < nKb) {
+        const double m = key[j] / total;
+        if (m > 0.0) hp -= m * log(m);
+      }
+    }
+    const double want = a.retention * exp(block_reduce(hp, wsum_d, false));
+    keep = (int)fmin((double)nKb, fmax(1.0, ceil(want)));
+  }
+  for (int e = 0; e < EPT; ++e) {
+    const int j = tid * EPT + e;
+    if (j < nKb) {
+      const double m = key[j] / total;
+      key[j] = m;
+      idx[j] = j;
+      a.mass[g * nKb + j] = m;
+      if (a.router == TA_ROUTER_PRICE)
+        tier[j] = (uint8_t)price_tier(m, a.spread[g * nKb + j], a.price, a.low, a.cost[TA_TIER_SKIP],
+                                      a.cost[TA_TIER_LOW], a.cost[TA_TIER_RES], a.cost[TA_TIER_FULL]);
+    } else {
+      key[j] = -1.0;
+      idx[j] = 0x7fffffff - (sortn - j);
+    }
+  }
+  __syncthreads();
+
+  // bitonic sort into (-M, j) order: position r holds (key[r], idx[r])
+  for (int size = 2; size <= sortn; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int pp = tid; pp < sortn / 2; pp += kRowThreads) {
+        const int lo = 2 * pp - (pp & (stride - 1));   // lower position of the pair
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;               // this block sorts (-M, j) ascending
+        const double kl = key[lo], kh = key[hi];
+        const int il = idx[lo], ih = idx[hi];
+        const bool hi_first = before(kh, ih, kl, il);
+        if (up == hi_first) {
+          key[lo] = kh;
+          key[hi] = kl;
+          idx[lo] = ih;
+          idx[hi] = il;
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // tiers by rank: exclusive prefix C of the sorted masses
+  int codes[3];
+  if (a.n_tau == 1) {
+    codes[0] = TA_TIER_FULL;
+  } else if (a.n_tau == 2) {
+    codes[0] = TA_TIER_FULL;
+    codes[1] = TA_TIER_LOW;
+  } else {
+    codes[0] = TA_TIER_FULL;
+    codes[1] = TA_TIER_RES;
+    codes[2] = TA_TIER_LOW;
+  }
+  if (a.router != TA_ROUTER_PRICE) {
+    const int kept_low = codes[a.n_tau - 1];
+    double mine = 0.0;
+    for (int e = 0; e < EPT; ++e) mine += fmax(key[tid * EPT + e], 0.0);
+    double tot;
+    double C = block_excl_scan(mine, wsum_d, tot);
+    for (int e = 0; e < EPT; ++e) {
+      const int r = tid * EPT + e;
+      const int j = idx[r];
+      const double mk = fmax(key[r], 0.0);
+      if (j < nKb) {
+        int t = TA_TIER_SKIP;
+        for (int q = a.n_tau - 1; q >= 0; --q)
+          if (C < a.tau[q]) t = codes[q];
+        if (a.router == TA_ROUTER_ENTROPY) t = (r >= keep) ? TA_TIER_SKIP : (t == TA_TIER_SKIP ? kept_low : t);
+        tier[j] = (uint8_t)t;
+      }
+      C += mk;
+    }
+  }
+  __syncthreads();
+  if (a.keep_diag && tid == 0) {
+    const int r0 = i * a.bq, r1 = min(a.N, (i + 1) * a.bq);
+    for (int j = r0 / a.bk; j <= (r1 - 1) / a.bk; ++j) tier[j] = TA_TIER_FULL;
+  }
+  __syncthreads();
+
+  // tier map row, counts and the compacted list (tiers full, res, low, skip;
+  // within a tier in rank order)
+  for (int j = tid; j < nKb; j += kRowThreads) a.tier_map[g * nKb + j] = tier[j];
+  const int order[4] = {TA_TIER_FULL, TA_TIER_RES, TA_TIER_LOW, TA_TIER_SKIP};
+  int base = 0;
+  for (int q = 0; q < 4; ++q) {
+    const int t = order[q];
+    int mine = 0;
+    for (int e = 0; e < EPT; ++e) {
+      const int j = idx[tid * EPT + e];
+      mine += (j < nKb && tier[j] == t) ? 1 : 0;
+    }
+    int cnt;
+    int pos = block_excl_scan_int(mine, wsum_i, cnt);
+    for (int e = 0; e < EPT; ++e) {
+      const int j = idx[tid * EPT + e];
+      if (j < nKb && tier[j] == t) a.row_lists[g * nKb + base + pos++] = j;
+    }
+    if (tid == 0) a.row_counts[g * 4 + q] = cnt;
+    base += cnt;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_route(const PlanArgs& a, cudaStream_t s) {
-  dim3 g1((a.nQb + 31) / 32, (a.nKb + 31) / 32, a.B * a.H);
+  dim3 g1((a.nQb + kLT - 1) / kLT, (a.nKb + kLT - 1) / kLT, a.B * a.H);
   logits_kernel<<<g1, 256, 0, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -331,13 +565,14 @@ cudaError_t launch_route(const PlanArgs& a, cudaStream_t s) {
   while (sortn < a.nKb) sortn <<= 1;
   const int64_t rows = (int64_t)a.B * a.H * a.nQb;
   dim3 g2((unsigned)((rows + kRouteWarps - 1) / kRouteWarps));
+  // rows of up to 256 key blocks: one warp a row; longer rows: one CTA a row
   switch (sortn) {
     case 32: route_kernel<1><<<g2, kRouteWarps * 32, 0, s>>>(a); break;
     case 64: route_kernel<2><<<g2, kRouteWarps * 32, 0, s>>>(a); break;
     case 128: route_kernel<4><<<g2, kRouteWarps * 32, 0, s>>>(a); break;
     case 256: route_kernel<8><<<g2, kRouteWarps * 32, 0, s>>>(a); break;
-    case 512: route_kernel<16><<<g2, kRouteWarps * 32, 0, s>>>(a); break;
-    case 1024: route_kernel<32><<<g2, kRouteWarps * 32, 0, s>>>(a); break;
+    case 512: route_row_kernel<2><<<(unsigned)rows, kRowThreads, 0, s>>>(a); break;
+    case 1024: route_row_kernel<4><<<(unsigned)rows, kRowThreads, 0, s>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

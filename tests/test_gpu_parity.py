@@ -384,3 +384,22 @@ def test_sequences_shorter_than_one_tile(cuda_ok, name, N):
         n_diff, _ = compare_tiers(views["tier_map"][h].numpy(), rt)
         assert n_diff == 0
         assert_out_close(to64(O[0, h]), Oref, f"{name} N={N} head {h}")
+
+
+@pytest.mark.parametrize("name,over", [
+    # rows of 512 key blocks (480p with 64-key blocks): the one-CTA-a-row router
+    ("480p", {"H": 1, "block_k": 64}),
+    ("480p", {"H": 1, "block_k": 64, "router": 1, "price": 0.004, "tier_cost": (0.0, 1.0, 3.0, 4.0)}),
+    ("480p", {"H": 1, "block_k": 64, "router": 2, "kappa": 0.7}),
+    # rows of 929 key blocks (720p, four tiers)
+    ("720p", {"H": 1}),
+    ("720p", {"H": 1, "router": 2, "kappa": 1.0}),
+])
+def test_long_row_router_parity(cuda_ok, name, over):
+    # the router for rows of more than 256 key blocks (one CTA a row): tier
+    # maps, counts and lists against the oracle, on whole heads
+    cfg, Q, K, V = inputs(name, **over)
+    _, views, _, st = run_gpu(cfg, Q, K, V, forward=False)
+    assert st == 0
+    assert len(np.unique(views["tier_map"].numpy())) >= 2
+    _plan_parity(cfg, Q, K, V, views, [(0, 0)])
