@@ -234,6 +234,48 @@ def sweep(args):
         del ws
 
 
+def tier_costs(args):
+    """Forward cost of each tier on the 480p shape (``--heads`` heads, 8 by
+    default): thresholds chosen so that every tile but the forced diagonal
+    falls in one tier, one JSON line per case with the time per kept tile
+    and SM (the price router's default tier costs are these, relative to
+    the bf16 tile)."""
+    import precision_attention_video_b200 as pav
+
+    dev = torch.device("cuda", 0)
+    base = get_config("480p").with_(H=args.heads or 8)
+    Q, K, V = make_qkv(base)
+    Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+    O = torch.empty_like(Qd)
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    cases = [("full", 2, (2.0, 2.0)), ("fp8", 1, (0.0, 2.0)), ("nvfp4", 2, (0.0, 2.0)),
+             ("res", 3, (0.0, 2.0, 2.0)), ("skip", 2, (0.0, 0.0))]
+    for name, low, tau in cases:
+        cfg = base.with_(low=low, tau=tau)
+        p = pav.params_for(cfg)
+        ws = pav.alloc_workspace(p, dev)
+        pav.plan(p, Qd, Kd, Vd, ws)
+        for _ in range(args.warmup):
+            pav.forward(p, Qd, Kd, Vd, ws, O)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            pav.forward(p, Qd, Kd, Vd, ws, O)
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        t = pav.plan_views(p, ws)["tier_map"].cpu()
+        n = {k: int((t == c).sum()) for k, c in (("full", 3), ("res", 2), ("low", 1), ("skip", 0))}
+        ms = statistics.median(ts)
+        kept = n["full"] + n["res"] + n["low"]
+        print(json.dumps({"tier_case": name, "status": pav.get_status(ws), "ms_forward": ms, "tiles": n,
+                          "us_per_kept_tile_per_sm": ms * 1e3 * n_sm / kept,
+                          "us_per_cta_per_sm": ms * 1e3 * n_sm / (cfg.n_qb * cfg.H)}), flush=True)
+        del ws
+
+
 def plan_reuse(args):
     """Plan reuse across timesteps: on a slowly changing sequence of K inputs
     (latent_gen.make_qkv_steps, correlation rho between steps), one plan
@@ -408,7 +450,8 @@ def cpu_baseline(cfg, budget_s: float = 20.0, threads: int = 0):
         t = time.time()
         rt = Rt.route_head(Qh, Kh, Vh, cfg.tau, cfg.block_q, cfg.block_k,
                            router=getattr(cfg, "router", 0), price=getattr(cfg, "price", 0.0),
-                           low=cfg.low, kappa=getattr(cfg, "kappa", 1.0))
+                           low=cfg.low, kappa=getattr(cfg, "kappa", 1.0),
+                           tier_cost=getattr(cfg, "tier_cost", None))
         qt = Qz.quantize_head(Qh, Kh, Vh, cfg.low, cfg.block_q, cfg.block_k)
         spent += time.time() - t
         done = 0
@@ -417,7 +460,7 @@ def cpu_baseline(cfg, budget_s: float = 20.0, threads: int = 0):
             t = time.time()
             oracle.tiered_attention_head(Qh, Kh, Vh, rt, qt, cfg.low, cfg.block_q, cfg.block_k,
                                          cfg.p_offset_log2, rt["scale"], False, blocks,
-                                         threads=cores)
+                                         threads=cores, key_pack=cfg.key_pack)
             spent += time.time() - t
             rows += sum(min(cfg.block_q, cfg.N - i * cfg.block_q) for i in blocks)
             done += len(blocks)
@@ -462,8 +505,14 @@ def main():
                     help="time plan reuse instead: one plan per K timesteps of a correlated sequence")
     ap.add_argument("--rho", type=float, default=0.99,
                     help="correlation between consecutive timesteps for --reuse")
+    ap.add_argument("--tier-costs", action="store_true",
+                    help="time each tier alone on the 480p shape instead (one JSON line per tier)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+
+    if args.tier_costs:
+        tier_costs(args)
+        return
 
     if args.sweep:
         sweep(args)

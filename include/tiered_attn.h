@@ -82,7 +82,16 @@ typedef struct {
   int32_t B, H, N, d;        /* batch, heads, tokens (N >= 1; the last query and
                                 key blocks may be partial, down to one token),
                                 head dim (d in {64,128})                       */
-  int32_t block_q, block_k;  /* tile rows / keys, each in {64,128}            */
+  int32_t block_q, block_k;  /* query rows in {64,128}; keys per block in
+                                {32,64,128}.  32-key blocks ("FG-Attn",
+                                searcharxiv author page, abstract: skipping at
+                                M x N sub-tiles) need d = 128, block_q = 128
+                                and low NONE, NVFP4 or NVFP4 + residual
+                                (else TA_ERR_UNSUPPORTED): the router tiers
+                                32-key blocks and the attention kernel packs
+                                the kept blocks of one tier four at a time, in
+                                list order, into 128-key tiles (one running-
+                                max update per tile)                           */
   int32_t low;               /* ta_low_format                                 */
   int32_t n_thresholds;      /* 1 (full only), 2 (full, low), 3 (full, res, low) */
   double  tau[3];            /* ascending cumulative-mass thresholds          */

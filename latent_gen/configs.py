@@ -64,6 +64,11 @@ class Workload:
     def n_kb(self) -> int:
         return -(-self.N // self.block_k)
 
+    @property
+    def key_pack(self) -> int:
+        """Key blocks per attention tile: 32-key blocks go four to a 128-key tile."""
+        return 4 if self.block_k == 32 else 1
+
     def dense_flops(self) -> float:
         """Dense-equivalent attention FLOPs: 4*B*H*N^2*d (QK^T and PV)."""
         return 4.0 * self.B * self.H * float(self.N) ** 2 * self.d
@@ -123,6 +128,12 @@ def _build() -> Dict[str, Workload]:
     c["480p-entropy"] = Workload("480p-entropy", 1, 40, 128, (21, 30, 52), 128, 128, 4.0,
                                  LOW_NVFP4, (0.6, 0.9), p_offset_log2=11, router=2,
                                  kappa=_kappa())
+    # The 480p layer routed at 32-key granularity ("FG-Attn", searcharxiv
+    # author page, abstract: skipping at M x N sub-tiles, M >= 16, N >= 1;
+    # here M = 128 queries, N = 32 keys); the attention kernel packs four kept
+    # 32-key blocks of one tier into each 128-key tile.
+    c["480p-fg"] = Workload("480p-fg", 1, 40, 128, (21, 30, 52), 128, 32, 4.0, LOW_NVFP4,
+                            (0.6, 0.9), p_offset_log2=11)
     # Sparsity sweep on the 480p shape with an FP8 low tier; the 0% point runs
     # every tile in bf16 (thresholds above every cumulative mass).
     sweep = _sweep_tau()

@@ -50,7 +50,12 @@ ta_status validate(const ta_params* p) {
   if (!p) return TA_ERR_INVALID_ARG;
   if (p->B < 1 || p->H < 1 || p->N < 1) return TA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return TA_ERR_UNSUPPORTED;
-  if ((p->block_q != 64 && p->block_q != 128) || (p->block_k != 64 && p->block_k != 128))
+  if ((p->block_q != 64 && p->block_q != 128) ||
+      (p->block_k != 32 && p->block_k != 64 && p->block_k != 128))
+    return TA_ERR_UNSUPPORTED;
+  // 32-key blocks run packed four to a 128-key tile, in the d = 128 kernel with
+  // 128-query blocks, for the bf16 and NVFP4 tiers
+  if (p->block_k == 32 && (p->d != 128 || p->block_q != 128 || p->low == TA_LOW_FP8_E4M3))
     return TA_ERR_UNSUPPORTED;
   if (p->low < TA_LOW_NONE || p->low > TA_LOW_NVFP4_RES) return TA_ERR_INVALID_ARG;
   const int want_tau = p->low == TA_LOW_NONE ? 1 : (p->low == TA_LOW_NVFP4_RES ? 3 : 2);
@@ -287,12 +292,21 @@ bool make_map_u8(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE,
-            box_inner == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+            box_inner == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                             : (box_inner == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE),
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 bool make_map_fp4(CUtensorMap* m, const void* base, int64_t BH, int64_t rows, int64_t inner,
                   int box_rows) {
   return make_map_u8(m, base, BH, rows, inner, box_rows, 64);
+}
+
+// Transposed NVFP4 V codes [BH, d, Np / 2]: a box is all d rows by the codes of
+// one key block.  128-key blocks: 64 bytes, 64-byte swizzle.  32-key blocks:
+// 16 bytes, unswizzled, so that the four blocks of a packed tile land as the
+// four 16-byte K columns of core matrices of one K-major operand.
+bool make_map_vt(CUtensorMap* m, const void* base, int64_t BH, int64_t d, int64_t inner, int block_k) {
+  return make_map_u8(m, base, BH, d, inner, (int)d, block_k / 2);
 }
 
 // bf16 tensor [B, H, N, d] (element strides sb, sh, sn), box = 64 x rows, 128B swizzle.
@@ -424,7 +438,8 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
   if ((st = check_ws(p, ws, ws_bytes)) != TA_OK) return st;
   // native NVFP4 (and residual) tiles are built for d = 128 with 128 x 128 tiles
   const bool fp4 = p->low == TA_LOW_NVFP4 || p->low == TA_LOW_NVFP4_RES;
-  if (fp4 && (p->d != 128 || p->block_q != 128 || p->block_k != 128)) return TA_ERR_UNSUPPORTED;
+  if (fp4 && (p->d != 128 || p->block_q != 128 || (p->block_k != 128 && p->block_k != 32)))
+    return TA_ERR_UNSUPPORTED;
   const Shape s = shape_of(p);
   const Layout L = layout_of(p);
   ta::AttnArgs a;
@@ -473,11 +488,11 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
     const int64_t BH = (int64_t)p->B * p->H;
     ok = ok && make_map_fp4(&maps[3], at<void>(ws, L.q_codes), BH, p->N, p->d / 2, p->block_q) &&
          make_map_fp4(&maps[4], at<void>(ws, L.k_codes), BH, p->N, p->d / 2, p->block_k) &&
-         make_map_fp4(&maps[5], at<void>(ws, L.v_codes), BH, p->d, s.Np / 2, p->d);
+         make_map_vt(&maps[5], at<void>(ws, L.v_codes), BH, p->d, s.Np / 2, p->block_k);
     if (p->low == TA_LOW_NVFP4_RES) {
       ok = ok && make_map_fp4(&maps[6], at<void>(ws, L.rq_codes), BH, p->N, p->d / 2, p->block_q) &&
            make_map_fp4(&maps[7], at<void>(ws, L.rk_codes), BH, p->N, p->d / 2, p->block_k) &&
-           make_map_fp4(&maps[8], at<void>(ws, L.rv_codes), BH, p->d, s.Np / 2, p->d);
+           make_map_vt(&maps[8], at<void>(ws, L.rv_codes), BH, p->d, s.Np / 2, p->block_k);
     } else {
       maps[6] = maps[3];
       maps[7] = maps[4];

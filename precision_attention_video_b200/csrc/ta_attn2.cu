@@ -81,6 +81,7 @@ struct Lay {
   static constexpr int oPinV = 16384;            // low P inside its V stage
   static_assert(kQlow == 0 || oQL % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(kTotal <= 227 * 1024, "shared memory");
+  static_assert(NK <= 3 && NV <= 3, "the mbarrier slots below hold at most three stages per ring");
 };
 
 // TMEM columns.
@@ -134,6 +135,68 @@ __device__ __forceinline__ bool bar_and2(int id, int count, bool pred) {
   return out != 0;
 }
 
+// Tile t of a row whose kept key blocks are KB keys wide, PK = 128 / KB of
+// them (consecutive in the list, one tier) to a 128-key tile: its kind, the
+// list position of its first block and how many blocks it holds (for a skip
+// chunk: how many skipped blocks, up to 128).  Skipped blocks follow the kept
+// tiles in chunks of 128.
+template <int PK>
+__device__ __forceinline__ void tile_of_packed(const RowPlan& rp, int t, int& kind, int& first, int& cnt) {
+  const int nf = (rp.n_full + PK - 1) / PK, nr = (rp.n_res + PK - 1) / PK;
+  const int nl = (rp.n_low + PK - 1) / PK;
+  if (t < nf) {
+    kind = KIND_FULL;
+    first = t * PK;
+    cnt = min(PK, rp.n_full - first);
+  } else if (t < nf + nr) {
+    const int u = (t - nf) * PK;
+    kind = KIND_RES;
+    first = rp.n_full + u;
+    cnt = min(PK, rp.n_res - u);
+  } else if (t < nf + nr + nl) {
+    const int u = (t - nf - nr) * PK;
+    kind = KIND_LOW;
+    first = rp.n_full + rp.n_res + u;
+    cnt = min(PK, rp.n_low - u);
+  } else {
+    const int kept = rp.n_full + rp.n_res + rp.n_low;
+    kind = KIND_SKIP;
+    first = kept + (t - nf - nr - nl) * 128;
+    cnt = min(128, rp.n_skip - (first - kept));
+  }
+}
+
+// Key blocks of a packed tile: slot i holds list entry first + i; slots past
+// cnt repeat the last real block (their columns are masked, their values
+// only need to be finite).
+template <int PK>
+__device__ __forceinline__ void pack_blocks(const RowPlan& rp, int first, int cnt, int (&jsl)[PK]) {
+#pragma unroll
+  for (int i = 0; i < PK; ++i) jsl[i] = rp.list[first + min(i, cnt - 1)];
+}
+
+// NVFP4 block scales of the 128 key rows of a packed tile (row rr = slot
+// rr / KB, key (rr % KB) of that slot's block) into the two [32][16 B] blocks
+// at dst: row 32*m1 + m0 of K chunk c at dst + c*512 + m0*16 + m1*4.  Keys
+// past N get zero scales.  `src` points at the head's [N][8] scales.
+template <int KB, int PK>
+__device__ __forceinline__ void gather_key_sf(unsigned char* dst, const uint8_t* src, const int (&jsl)[PK],
+                                              int N, int lane) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = lane * 4 + i, slot = rr / KB;
+    int j = jsl[0];
+#pragma unroll
+    for (int u = 1; u < PK; ++u) j = (slot == u) ? jsl[u] : j;
+    const int key = j * KB + rr % KB;
+    uint2 v = make_uint2(0u, 0u);
+    if (key < N) v = *reinterpret_cast<const uint2*>(src + (int64_t)key * 8);
+    const int off = (rr & 31) * 16 + (rr >> 5) * 4;
+    *reinterpret_cast<uint32_t*>(dst + off) = v.x;
+    *reinterpret_cast<uint32_t*>(dst + 512 + off) = v.y;
+  }
+}
+
 // Formats of P' in a tile's softmax tail.
 enum { T_BF16 = 0, T_SKIP = 1, T_FP4 = 2, T_RES = 3, T_F8 = 4 };
 
@@ -151,9 +214,10 @@ constexpr int kEmuPairs() {
 struct Tail {
   float c2t, mc;            // P' = 2^(s * c2t - mc)
   float alpha;              // exp(m_old - m_new) of this row
-  int t, nv;                // tile index, valid columns
+  int t;                    // tile index
   int last_col;             // skip chunks: column of the last key block, or -1
   float w_last;             // its key count
+  float w_blk;              // the key count of every other block
   uint64_t* bars;
   AbortCtx ctx;
   unsigned char* sm;
@@ -190,11 +254,11 @@ __device__ __forceinline__ bool tail(float (&x)[128], const float (&gm)[8], cons
     }
   }
   if constexpr (K == T_SKIP) {
-    // pooled keys weigh n_j: 128 for every block but the sequence's ragged
+    // pooled keys weigh n_j: KB for every block but the sequence's ragged
     // last one, which sits in column q.last_col (or nowhere: -1); columns
     // past nv are exp(-inf) = 0 already
 #pragma unroll
-    for (int c = 0; c < 128; ++c) x[c] *= (c == q.last_col) ? q.w_last : 128.0f;
+    for (int c = 0; c < 128; ++c) x[c] *= (c == q.last_col) ? q.w_last : q.w_blk;
   }
   {
     uint64_t sa = pack2(0.0f, 0.0f), sb = pack2(0.0f, 0.0f);
@@ -295,7 +359,7 @@ __device__ __forceinline__ bool tail(float (&x)[128], const float (&gm)[8], cons
   return true;
 }
 
-template <int LM>
+template <int LM, int KB>
 __global__ void __launch_bounds__(kThreads2, 1)
     attn2_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tmQ,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -306,6 +370,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
   using TM = Tm<LM>;
   constexpr bool FP4 = L::FP4, RES = L::RES, F8 = L::F8;
   constexpr int NK = L::NK, NV = L::NV;
+  constexpr int PK = kBK / KB;   // key blocks per tile
+  static_assert(PK == 1 || (PK == 4 && !F8), "32-key blocks: bf16 and NVFP4 tiers");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw;
   if (smem_u32(sm) & 1023u) {
@@ -328,7 +394,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
   rp.n_low = a.row_counts[row_id * 4 + 2];
   rp.n_skip = a.row_counts[row_id * 4 + 3];
   rp.list = a.row_lists + row_id * a.nKb;
-  rp.T = rp.n_full + rp.n_res + rp.n_low + (rp.n_skip + kBK - 1) / kBK;
+  rp.T = (rp.n_full + PK - 1) / PK + (rp.n_res + PK - 1) / PK + (rp.n_low + PK - 1) / PK +
+         (rp.n_skip + kBK - 1) / kBK;
   const int kept = rp.n_full + rp.n_res + rp.n_low;
   const bool has_low = (FP4 || F8) && (rp.n_low > 0 || rp.n_res > 0);
   const int nq = rp.n_res > 0 ? 2 : (has_low ? 1 : 0);   // query low copies to load
@@ -414,12 +481,77 @@ __global__ void __launch_bounds__(kThreads2, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) { aborted = true; break; }
       }
-      int kind, first;
-      tile_of<kBK>(rp, t, kind, first);
+      int kind, first, cnt = 0;
+      if constexpr (PK == 1)
+        tile_of<kBK>(rp, t, kind, first);
+      else
+        tile_of_packed<PK>(rp, t, kind, first, cnt);
       unsigned char* st = sm + (isK ? L::oK : L::oV) + s * L::kStage;
       unsigned char* side = sm + (isK ? L::oKS + s * L::kKSide : L::oVS + s * L::kVSide);
       const bool drop = isK && (t == 0) && (a.debug_flags & TA_DEBUG_DROP_FIRST_K);
-      if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
+      if (kind != KIND_SKIP && PK > 1) {
+        // packed tile: PK key blocks of KB keys side by side
+        int jsl[PK];
+        pack_blocks<PK>(rp, first, cnt, jsl);
+        if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
+          const int ncopy = (RES && kind == KIND_RES) ? 2 : 1;
+          for (int c = 0; c < ncopy; ++c) {
+            if (isK) {
+              gather_key_sf<KB, PK>(side + c * L::kSfBlk, (c ? a.rk_sf : a.k_sf) + (int64_t)bh * a.N * 8, jsl,
+                                    a.N, lane);
+            } else {
+              // V scales: groups of 16 keys of each d row of V^T; group k of K
+              // chunk kc covers keys 64 kc + 16 k .. of the tile, in block
+              // (4 kc + k) / (KB / 16)
+              const uint8_t* vsf = c ? a.rv_sf : a.v_sf;
+              const int ng = a.Np / 16;
+#pragma unroll
+              for (int kc = 0; kc < 2; ++kc) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  constexpr int kGroups = KB / 16;   // scale groups per key block
+                  const int gi = jsl[(kc * 4 + k) / kGroups] * kGroups + (kc * 4 + k) % kGroups;
+                  uint32_t w = 0u;
+                  if (gi < ng)
+                    w = *reinterpret_cast<const uint32_t*>(vsf + ((int64_t)bh * ng + gi) * kD + lane * 4);
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    const int m = lane * 4 + i;
+                    side[c * L::kSfBlk + kc * 512 + (m & 31) * 16 + (m >> 5) * 4 + k] = (unsigned char)(w >> (8 * i));
+                  }
+                }
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && !drop) {
+            mbar_arrive_expect_tx(&full[s], ncopy * 128 * 64);
+            for (int c = 0; c < ncopy; ++c) {
+#pragma unroll
+              for (int i = 0; i < PK; ++i) {
+                // K: KB rows of 64 bytes; V^T: 128 rows of KB / 2 bytes
+                if (isK)
+                  tma_load_3d(st + c * L::kCodes + i * (KB * 64), c ? &tmRK : &tmDK, &full[s], 0, jsl[i] * KB, bh);
+                else
+                  tma_load_3d(st + c * L::kCodes + i * (KB * 64), c ? &tmRV : &tmDV, &full[s], jsl[i] * (KB / 2),
+                              0, bh);
+              }
+            }
+            issued[s]++;
+          }
+        } else {
+          if (lane == 0 && !drop) {
+            mbar_arrive_expect_tx(&full[s], kBK * kD * 2);
+#pragma unroll
+            for (int i = 0; i < PK; ++i)
+              for (int x = 0; x < 2; ++x)
+                tma_load_4d(st + x * (kBK * 128) + i * (KB * 128), isK ? &tmK : &tmV, &full[s], x * 64,
+                            jsl[i] * KB, h, b);
+            issued[s]++;
+          }
+        }
+      } else if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
         const int j = rp.list[first];
         const int ncopy = (RES && kind == KIND_RES) ? 2 : 1;
         for (int c = 0; c < ncopy; ++c) {
@@ -486,7 +618,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
         // pooled rows of the chunk's skipped blocks as a pseudo tile: the
         // list entries once (lane l holds columns l, l+32, ...), then every
         // 16-byte piece as an asynchronous copy (zero past the chunk's end)
-        const int cnt = min(kBK, rp.n_skip - (first - kept));
+        if constexpr (PK == 1) cnt = min(kBK, rp.n_skip - (first - kept));
         int jl[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -548,8 +680,11 @@ __global__ void __launch_bounds__(kThreads2, 1)
         const int s = t % NK;
         if (!wait_all(&bars[B_KF + s], (t / NK) & 1, 2)) return false;
         tc_fence_after();
-        int kind, first;
-        tile_of<kBK>(rp, t, kind, first);
+        int kind, first, cnt;
+        if constexpr (PK == 1)
+          tile_of<kBK>(rp, t, kind, first);
+        else
+          tile_of_packed<PK>(rp, t, kind, first, cnt);
         const uint32_t sk = smem_u32(sm + L::oK + s * L::kStage);
         const uint32_t d = tS0 + 128 * (t & 1);
         if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
@@ -595,8 +730,11 @@ __global__ void __launch_bounds__(kThreads2, 1)
         if (!wait_all(&bars[B_PR + g], (t >> 1) & 1, 4)) return false;
         if (!wait_all(&bars[B_VF + s], (t / NV) & 1, 5)) return false;
         tc_fence_after();
-        int kind, first;
-        tile_of<kBK>(rp, t, kind, first);
+        int kind, first, cnt;
+        if constexpr (PK == 1)
+          tile_of<kBK>(rp, t, kind, first);
+        else
+          tile_of_packed<PK>(rp, t, kind, first, cnt);
         const uint32_t sv = smem_u32(sm + L::oV + s * L::kStage);
         const uint32_t acc0 = t > 0 ? 1u : 0u;
         if (FP4 && (kind == KIND_LOW || kind == KIND_RES)) {
@@ -610,16 +748,25 @@ __global__ void __launch_bounds__(kThreads2, 1)
             tc_cp_sf_w(tmem + TM::sfbV(c), smem_desc_rows16(vsf));
             tc_cp_sf_w(tmem + TM::sfbV(c) + 4, smem_desc_rows16(vsf + 512));
           }
+          // V^T copy c, keys 64 kk ..: 64-byte-swizzled rows of one 128-key
+          // block, or (32-key blocks) the unswizzled 16-byte columns of two
+          // blocks, 2048 bytes apart
+          auto vdesc = [&](int c, int kk) -> uint64_t {
+            if constexpr (PK == 1)
+              return smem_desc_sw64(sv + c * L::kCodes + kk * 32);
+            else
+              return smem_desc_kmajor_noswz(sv + c * L::kCodes + kk * 4096, 2048, 128);
+          };
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
-            mma_nvfp4_ss_w(tO, smem_desc_sw64(pb + kk * 32), smem_desc_sw64(sv + kk * 32),
+            mma_nvfp4_ss_w(tO, smem_desc_sw64(pb + kk * 32), vdesc(0, kk),
                          idesc_nvfp4(128, kD), tmem + TM::sfaP(0) + kk * 4,
                          tmem + TM::sfbV(0) + kk * 4, (acc0 || kk > 0) ? 1u : 0u);
             if (RES && kind == KIND_RES) {
-              mma_nvfp4_ss_w(tO, smem_desc_sw64(pb + kk * 32), smem_desc_sw64(sv + L::kCodes + kk * 32),
+              mma_nvfp4_ss_w(tO, smem_desc_sw64(pb + kk * 32), vdesc(1, kk),
                            idesc_nvfp4(128, kD), tmem + TM::sfaP(0) + kk * 4,
                            tmem + TM::sfbV(1) + kk * 4, 1u);
-              mma_nvfp4_ss_w(tO, smem_desc_sw64(pb + L::kCodes + kk * 32), smem_desc_sw64(sv + kk * 32),
+              mma_nvfp4_ss_w(tO, smem_desc_sw64(pb + L::kCodes + kk * 32), vdesc(0, kk),
                            idesc_nvfp4(128, kD), tmem + TM::sfaP(1) + kk * 4,
                            tmem + TM::sfbV(0) + kk * 4, 1u);
             }
@@ -696,12 +843,12 @@ __global__ void __launch_bounds__(kThreads2, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_QR]);
     }
-    // the ragged last key block (n < 128 keys) and its position in the row's
-    // list: the only skipped block whose pooled key does not weigh 128
-    const int n_last = a.N - (a.nKb - 1) * kBK;
+    // the ragged last key block (n < KB keys) and its position in the row's
+    // list: the only skipped block whose pooled key does not weigh KB
+    const int n_last = a.N - (a.nKb - 1) * KB;
     const float w_last = (float)n_last;
     int pos_last = -1000000;
-    if (n_last < kBK) {
+    if (n_last < KB) {
       for (int i0 = 0; i0 < a.nKb; i0 += 32) {
         const int i = i0 + lane;
         const unsigned bal = __ballot_sync(0xffffffffu, i < a.nKb && rp.list[i] == a.nKb - 1);
@@ -714,25 +861,64 @@ __global__ void __launch_bounds__(kThreads2, 1)
       ok = ok && mbar_wait(&bars[B_SR + g], (t >> 1) & 1, ctx, 6);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      int kind, first;
-      tile_of<kBK>(rp, t, kind, first);
-      const int j = (kind == KIND_SKIP) ? 0 : rp.list[first];
-      const int nv = (kind == KIND_SKIP) ? min(kBK, rp.n_skip - (first - kept)) : min(kBK, a.N - j * kBK);
-      const float sqk = (F8 && kind == KIND_LOW) ? s_q8 * a.k_s8[(int64_t)bh * a.nKb + j] : 1.0f;
+      int kind, first, cnt;
+      float sqk = 1.0f;
       float x[128];
-      tc_fence_after();
-      {
-        uint32_t raw[128];
+      if constexpr (PK == 1) {
+        tile_of<kBK>(rp, t, kind, first);
+        const int j = (kind == KIND_SKIP) ? 0 : rp.list[first];
+        const int nv = (kind == KIND_SKIP) ? min(kBK, rp.n_skip - (first - kept)) : min(kBK, a.N - j * kBK);
+        if (F8 && kind == KIND_LOW) sqk = s_q8 * a.k_s8[(int64_t)bh * a.nKb + j];
+        tc_fence_after();
+        {
+          uint32_t raw[128];
 #pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) tmem_ld32_nw(tS + c0, raw + c0);
-        tmem_wait_ld();
+          for (int c0 = 0; c0 < 128; c0 += 32) tmem_ld32_nw(tS + c0, raw + c0);
+          tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(raw[c]);
-      }
-      if (nv < 128) {
+          for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(raw[c]);
+        }
+        // columns past the skip chunk's end or past N in the ragged last block
+        if (nv < 128) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= nv) x[c] = -INFINITY;
+          for (int c = 0; c < 128; ++c)
+            if (c >= nv) x[c] = -INFINITY;
+        }
+      } else {
+        tile_of_packed<PK>(rp, t, kind, first, cnt);
+        int jsl[PK];
+        if (kind != KIND_SKIP) pack_blocks<PK>(rp, first, cnt, jsl);
+        tc_fence_after();
+        {
+          uint32_t raw[128];
+#pragma unroll
+          for (int c0 = 0; c0 < 128; c0 += 32) tmem_ld32_nw(tS + c0, raw + c0);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(raw[c]);
+        }
+        // columns without a real key: past the skip chunk's end, past N in
+        // the ragged last block, and in slots past the tile's blocks
+        if (kind == KIND_SKIP) {
+          if (cnt < 128) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (c >= cnt) x[c] = -INFINITY;
+          }
+        } else {
+          int vs[PK];
+          bool ragged = false;
+#pragma unroll
+          for (int i = 0; i < PK; ++i) {
+            vs[i] = (i < cnt) ? min(KB, a.N - jsl[i] * KB) : 0;
+            ragged |= vs[i] < KB;
+          }
+          if (ragged) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (c % KB >= vs[c / KB]) x[c] = -INFINITY;
+          }
+        }
       }
       // maxima of the 8 groups of 16 columns (the NVFP4 scale groups), then of the row
       float gm[8];
@@ -762,9 +948,9 @@ __global__ void __launch_bounds__(kThreads2, 1)
       q.mc = m_new * c2 - o_off;
       q.alpha = fast_exp2((m_in - m_new) * c2);
       q.t = t;
-      q.nv = nv;
       q.last_col = (kind == KIND_SKIP) ? pos_last - first : -1;
       q.w_last = w_last;
+      q.w_blk = (float)KB;
       q.bars = bars;
       q.ctx = ctx;
       q.sm = sm;
@@ -841,10 +1027,10 @@ __global__ void __launch_bounds__(kThreads2, 1)
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
-template <int LM>
+template <int LM, int KB>
 cudaError_t launch2(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
   using L = Lay<LM>;
-  auto k = attn2_kernel<LM>;
+  auto k = attn2_kernel<LM, KB>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nQb, a.B * a.H);
@@ -855,14 +1041,22 @@ cudaError_t launch2(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) 
 
 }  // namespace
 
-// d = 128 with 128 x 128 tiles: every low format this kernel has a tail for.
-// Returns cudaErrorNotSupported for shapes it does not cover.
+// d = 128 with 128-query blocks and 128-key tiles: every low format this
+// kernel has a tail for; 32-key blocks (four to a tile) for the bf16 and
+// NVFP4 tiers.  Returns cudaErrorNotSupported for shapes it does not cover.
 cudaError_t launch_attn2(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t s) {
-  if (a.d != 128 || a.bk != 128) return cudaErrorNotSupported;
-  if (a.low == TA_LOW_NONE) return launch2<LM_IMAGE>(a, maps, s);
-  if (a.low == TA_LOW_NVFP4) return launch2<LM_NVFP4>(a, maps, s);
-  if (a.low == TA_LOW_NVFP4_RES) return launch2<LM_NVFP4_RES>(a, maps, s);
-  if (a.low == TA_LOW_FP8_E4M3 && a.bq == 128) return launch2<LM_FP8>(a, maps, s);
+  if (a.d != 128 || a.bq != 128) return cudaErrorNotSupported;
+  if (a.bk == 32) {
+    if (a.low == TA_LOW_NONE) return launch2<LM_IMAGE, 32>(a, maps, s);
+    if (a.low == TA_LOW_NVFP4) return launch2<LM_NVFP4, 32>(a, maps, s);
+    if (a.low == TA_LOW_NVFP4_RES) return launch2<LM_NVFP4_RES, 32>(a, maps, s);
+    return cudaErrorInvalidValue;   // no other kernel takes 32-key blocks   // no other kernel takes 32-key blocks
+  }
+  if (a.bk != 128) return cudaErrorNotSupported;
+  if (a.low == TA_LOW_NONE) return launch2<LM_IMAGE, 128>(a, maps, s);
+  if (a.low == TA_LOW_NVFP4) return launch2<LM_NVFP4, 128>(a, maps, s);
+  if (a.low == TA_LOW_NVFP4_RES) return launch2<LM_NVFP4_RES, 128>(a, maps, s);
+  if (a.low == TA_LOW_FP8_E4M3) return launch2<LM_FP8, 128>(a, maps, s);
   return cudaErrorNotSupported;
 }
 

@@ -369,6 +369,17 @@ __device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr) {
   d |= (uint64_t)4 << 61;
   return d;
 }
+// Descriptor of an unswizzled K-major operand: core matrices of 8 rows x 16
+// bytes (128 contiguous bytes), `lbo` bytes apart along K and `sbo` bytes
+// apart along M / N (layout code 0).
+__device__ __forceinline__ uint64_t smem_desc_kmajor_noswz(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
 // Descriptor of an unswizzled, contiguous [rows][16 bytes] block (8-row core
 // matrices of 128 bytes, back to back).
 __device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t saddr) {

@@ -57,10 +57,13 @@ __device__ __forceinline__ float fp8_pow2_scale(float amax) {
 // `tab[c]` = (value, correctly rounded 1 / value) of ue4m3 code c.
 __device__ __forceinline__ uint32_t nvfp4_group(const float (&x)[16], uint32_t (&packed)[2],
                                                 const float2* tab) {
-  float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  // amax of |x| with three-input maxima: 8 instructions for 16 values
+  float am[3];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) am[i & 3] = fmaxf(am[i & 3], fabsf(x[i]));
-  const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
+  for (int u = 0; u < 3; ++u)
+    am[u] = fmax3(fabsf(x[5 * u]), fabsf(x[5 * u + 1]), fmax3(fabsf(x[5 * u + 2]), fabsf(x[5 * u + 3]),
+                                                               fabsf(x[5 * u + 4])));
+  const float amax = fmax3(am[0], fmax3(am[1], am[2], fabsf(x[15])), 0.0f);
   const uint32_t scc = cvt_e4m3x2(div6(amax), 0.0f) & 0xFFu;
   const float inv = tab[scc].y;
   const uint64_t inv2 = pack2(inv, inv);
@@ -107,8 +110,9 @@ struct PrepSmem {
   static constexpr size_t kSums = (size_t)SEG * D * 12, kVst = (size_t)2 * G * VP * 8;
   static constexpr size_t oScale = oPsum + (kSums > kVst ? kSums : kVst);
   static constexpr size_t kBytes = oScale + 8 * sizeof(float);
-  static_assert(kThreads % CP == 0 && R % SEG == 0 && 64 % RS == 0,
-                "a row segment must lie inside one block");
+  static_assert(kThreads % CP == 0 && R % SEG == 0 && 32 % RS == 0,
+                "a row segment must lie inside one block (blocks of 32, 64 or 128 rows)");
+  static_assert(SEG >= R / 32, "the column maxima of every block fit the reduction area");
 };
 
 template <int D, int R>
@@ -158,40 +162,58 @@ __global__ void __launch_bounds__(kThreads, 4) prep_kernel(const PlanArgs a) {
     const uint32_t* col = tile32 + seg * L::RS * L::CP + cp;
     double s0 = 0.0, s1 = 0.0;
     float m0 = 0.0f, m1 = 0.0f;
+    if (a.low == TA_LOW_FP8_E4M3) {
+      // column maxima: only the FP8 tile scale needs them
 #pragma unroll 8
-    for (int r = 0; r < L::RS; ++r) {
-      const uint32_t w = col[r * L::CP];
-      const float lo = bf_lo(w), hi = bf_hi(w);
-      s0 += (double)lo;
-      s1 += (double)hi;
-      m0 = fmaxf(m0, fabsf(lo));
-      m1 = fmaxf(m1, fabsf(hi));
+      for (int r = 0; r < L::RS; ++r) {
+        const uint32_t w = col[r * L::CP];
+        const float lo = bf_lo(w), hi = bf_hi(w);
+        s0 += (double)lo;
+        s1 += (double)hi;
+        m0 = fmaxf(m0, fabsf(lo));
+        m1 = fmaxf(m1, fabsf(hi));
+      }
+    } else {
+#pragma unroll 8
+      for (int r = 0; r < L::RS; ++r) {
+        const uint32_t w = col[r * L::CP];
+        s0 += (double)bf_lo(w);
+        s1 += (double)bf_hi(w);
+      }
     }
     *reinterpret_cast<double2*>(psum + seg * D + 2 * cp) = make_double2(s0, s1);
     *reinterpret_cast<float2*>(red + seg * D + 2 * cp) = make_float2(m0, m1);
   }
   __syncthreads();
-  // nb * D <= 256 = kThreads: one (block, column) per thread
-  const bool mine = tid < nb * D;
-  double s = 0.0;
-  float amax_c = 0.0f;
-  if (mine) {
-    const int jb = tid / D, c = tid % D;
-    const int spb = L::SEG / nb;   // segments per block
-    for (int k = 0; k < spb; ++k) {
-      s += psum[(jb * spb + k) * D + c];
-      amax_c = fmaxf(amax_c, red[(jb * spb + k) * D + c]);
+  // nb * D (block, column) pairs, at most kPer per thread
+  constexpr int kPer = (R / 32) * D / kThreads > 0 ? (R / 32) * D / kThreads : 1;
+  double s[kPer];
+  float amax_c[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int w = tid + u * kThreads;
+    s[u] = 0.0;
+    amax_c[u] = 0.0f;
+    if (w < nb * D) {
+      const int jb = w / D, c = w % D;
+      const int spb = L::SEG / nb;   // segments per block
+      for (int k = 0; k < spb; ++k) {
+        s[u] += psum[(jb * spb + k) * D + c];
+        amax_c[u] = fmaxf(amax_c[u], red[(jb * spb + k) * D + c]);
+      }
     }
   }
   __syncthreads();
-  if (mine) {
-    const int w = tid;
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int w = tid + u * kThreads;
+    if (w >= nb * D) continue;
     const int jb = w / D, c = w % D;
     const int rs = jb * blk, re = min(rs + blk, nrows);
-    red[w] = amax_c;
+    red[w] = amax_c[u];
     if (re > rs) {
       const int gb = r0 / blk + jb;
-      const double mean = s / (double)(re - rs);
+      const double mean = s[u] / (double)(re - rs);
       if (which == 0) {
         a.qbar[((int64_t)bh * a.nQb + gb) * D + c] = mean;
         if (a.qvar) {

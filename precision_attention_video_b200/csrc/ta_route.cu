@@ -33,81 +33,76 @@ namespace {
 // Pooled logits: logits[bh, i, j] = scale * sum_c qbar[bh, i, c] kbar[bh, j, c]
 // and, for the price router, the skip tier's error factor
 // spread[bh, i, j] = scale * sqrt(sum_c (qbar[bh, i, c]^2 + qvar[bh, i, c]) kvar[bh, j, c]).
-// 64 x 64 output tile per CTA, 4 x 4 per thread (rows ty + 16 u, columns
+// 128 x 128 output tile per CTA, 8 x 8 per thread (rows ty + 16 u, columns
 // tx + 16 v, so that a warp's 16 tx read 16 consecutive doubles: no bank
-// conflicts), d staged 16 at a time.
+// conflicts), d staged kLC coordinates at a time; 16 shared loads feed 64
+// fp64 FMAs.  The spread is a second pass over d with the same registers.
 // ---------------------------------------------------------------------------
-constexpr int kLT = 64, kLC = 16;
+constexpr int kLT = 128, kLC = 8;
+
+template <bool SPREAD>
+__device__ __forceinline__ void logits_pass(const PlanArgs& a, int bh, int i0, int j0, double (&qs)[kLC][kLT],
+                                            double (&ks)[kLC][kLT], double (&acc)[8][8]) {
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  const int D = a.d;
+  const double* qb = a.qbar + (int64_t)bh * a.nQb * D;
+  const double* kb = (SPREAD ? a.kvar : a.kbar) + (int64_t)bh * a.nKb * D;
+  const double* qvb = SPREAD ? a.qvar + (int64_t)bh * a.nQb * D : nullptr;
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+#pragma unroll
+    for (int v = 0; v < 8; ++v) acc[u][v] = 0.0;
+  for (int c0 = 0; c0 < D; c0 += kLC) {
+    // stage 128 rows x kLC coordinates of each operand: element e = r * kLC + c
+    for (int e = tid; e < kLT * kLC; e += 256) {
+      const int r = e / kLC, c = e % kLC;
+      const bool qi = i0 + r < a.nQb, kj = j0 + r < a.nKb;
+      double q = qi ? qb[(int64_t)(i0 + r) * D + c0 + c] : 0.0;
+      if (SPREAD && qi) q = q * q + qvb[(int64_t)(i0 + r) * D + c0 + c];
+      qs[c][r] = q;
+      ks[c][r] = kj ? kb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 2
+    for (int c = 0; c < kLC; ++c) {
+      double q[8], k[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) q[u] = qs[c][ty + 16 * u];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) k[v] = ks[c][tx + 16 * v];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int v = 0; v < 8; ++v) acc[u][v] = fma(q[u], k[v], acc[u][v]);
+    }
+    __syncthreads();
+  }
+}
 
 __global__ void __launch_bounds__(256) logits_kernel(const PlanArgs a) {
   __shared__ double qs[kLC][kLT];
   __shared__ double ks[kLC][kLT];
-  __shared__ double qw[kLC][kLT];   // qbar^2 + qvar (price router)
-  __shared__ double vs[kLC][kLT];   // kvar (price router)
   const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
   const int bh = blockIdx.z, i0 = blockIdx.x * kLT, j0 = blockIdx.y * kLT;
-  const int D = a.d;
-  const double* qb = a.qbar + (int64_t)bh * a.nQb * D;
-  const double* kb = a.kbar + (int64_t)bh * a.nKb * D;
-  const double* kvb = a.kvar ? a.kvar + (int64_t)bh * a.nKb * D : nullptr;
-  const double* qvb = a.qvar ? a.qvar + (int64_t)bh * a.nQb * D : nullptr;
-  double acc[4][4], spr[4][4];
+  double acc[8][8];
+  logits_pass<false>(a, bh, i0, j0, qs, ks, acc);
 #pragma unroll
-  for (int u = 0; u < 4; ++u)
+  for (int u = 0; u < 8; ++u)
 #pragma unroll
-    for (int v = 0; v < 4; ++v) acc[u][v] = spr[u][v] = 0.0;
-  for (int c0 = 0; c0 < D; c0 += kLC) {
-    // stage 64 rows x 16 coordinates of each operand: element e = r * 16 + c
-    for (int e = tid; e < kLT * kLC; e += 256) {
-      const int r = e / kLC, c = e % kLC;
-      const bool qi = i0 + r < a.nQb, kj = j0 + r < a.nKb;
-      const double q = qi ? qb[(int64_t)(i0 + r) * D + c0 + c] : 0.0;
-      qs[c][r] = q;
-      ks[c][r] = kj ? kb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
-      if (kvb) {
-        vs[c][r] = kj ? kvb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
-        qw[c][r] = qi ? q * q + qvb[(int64_t)(i0 + r) * D + c0 + c] : 0.0;
-      }
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int c = 0; c < kLC; ++c) {
-      double q[4], k[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) q[u] = qs[c][ty + 16 * u];
-#pragma unroll
-      for (int v = 0; v < 4; ++v) k[v] = ks[c][tx + 16 * v];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] = fma(q[u], k[v], acc[u][v]);
-    }
-    if (kvb) {
-#pragma unroll 4
-      for (int c = 0; c < kLC; ++c) {
-        double w[4], k[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) w[u] = qw[c][ty + 16 * u];
-#pragma unroll
-        for (int v = 0; v < 4; ++v) k[v] = vs[c][tx + 16 * v];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int v = 0; v < 4; ++v) spr[u][v] = fma(w[u], k[v], spr[u][v]);
-      }
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
+    for (int v = 0; v < 8; ++v) {
       const int i = i0 + ty + 16 * u, j = j0 + tx + 16 * v;
-      if (i < a.nQb && j < a.nKb) {
-        a.logits[((int64_t)bh * a.nQb + i) * a.nKb + j] = acc[u][v] * a.scale;
-        if (kvb) a.spread[((int64_t)bh * a.nQb + i) * a.nKb + j] = a.scale * sqrt(spr[u][v]);
-      }
+      if (i < a.nQb && j < a.nKb) a.logits[((int64_t)bh * a.nQb + i) * a.nKb + j] = acc[u][v] * a.scale;
     }
+  if (a.kvar) {
+    logits_pass<true>(a, bh, i0, j0, qs, ks, acc);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const int i = i0 + ty + 16 * u, j = j0 + tx + 16 * v;
+        if (i < a.nQb && j < a.nKb) a.spread[((int64_t)bh * a.nQb + i) * a.nKb + j] = a.scale * sqrt(acc[u][v]);
+      }
+  }
 }
 
 // The price router's tier of one tile: the least predicted error + price *
@@ -404,12 +399,89 @@ __device__ __forceinline__ double block_reduce(double v, double* wsum, bool is_m
   return r;
 }
 
+// One compare-exchange of the (-M, j) bitonic network: (ka, ia) sits at the
+// lower position, (kb, ib) at the higher; `up` sorts the pair ascending.
+__device__ __forceinline__ void cmp_swap(double& ka, int& ia, double& kb, int& ib, bool up) {
+  if (up == before(kb, ib, ka, ia)) {
+    const double k = ka;
+    const int i = ia;
+    ka = kb;
+    ia = ib;
+    kb = k;
+    ib = i;
+  }
+}
+
+// Bitonic sort of kRowThreads * EPT elements into (-M, j) order; thread tid
+// holds positions tid * EPT .. tid * EPT + EPT - 1 in (kr, ir).  Strides
+// below EPT run inside a thread, strides below 32 * EPT between the lanes of
+// a warp (shuffles), longer ones through shared memory (`xk`, `xi`: one
+// element per thread and slot, slot-major so that a warp's accesses fall on
+// distinct banks).
+template <int EPT>
+__device__ __forceinline__ void sort_row(double (&kr)[EPT], int (&ir)[EPT], double* xk, int* xi) {
+  constexpr int sortn = kRowThreads * EPT;
+  const int tid = threadIdx.x;
+  for (int size = 2; size <= sortn; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride < EPT) {
+#pragma unroll
+        for (int s = EPT / 2; s >= 1; s >>= 1) {
+          if (s != stride) continue;
+#pragma unroll
+          for (int e = 0; e < EPT; ++e)
+            if ((e & s) == 0) cmp_swap(kr[e], ir[e], kr[e + s], ir[e + s], ((tid * EPT + e) & size) == 0);
+        }
+        continue;
+      }
+      // the partner of position p = tid * EPT + e is p ^ stride = (tid ^ m) * EPT + e
+      const int m = stride / EPT;
+      const bool lower = (tid & m) == 0;
+      const bool up = ((tid * EPT) & size) == 0;   // size > stride >= EPT: one direction a thread
+      double kp[EPT];
+      int ip[EPT];
+      if (stride < 32 * EPT) {
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+          kp[e] = __shfl_xor_sync(0xffffffffu, kr[e], m);
+          ip[e] = __shfl_xor_sync(0xffffffffu, ir[e], m);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+          xk[e * kRowThreads + tid] = kr[e];
+          xi[e * kRowThreads + tid] = ir[e];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+          kp[e] = xk[e * kRowThreads + (tid ^ m)];
+          ip[e] = xi[e * kRowThreads + (tid ^ m)];
+        }
+        __syncthreads();
+      }
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) {
+        // both threads of a pair take the same decision and keep their side
+        const bool hi_first = lower ? before(kp[e], ip[e], kr[e], ir[e]) : before(kr[e], ir[e], kp[e], ip[e]);
+        if (up == hi_first) {
+          kr[e] = kp[e];
+          ir[e] = ip[e];
+        }
+      }
+    }
+  }
+}
+
 // EPT: elements a thread owns (sortn = kRowThreads * EPT, a power of two).
+// Thread tid owns key blocks tid * EPT .. (contiguous) before the sort and
+// ranks tid * EPT .. after it, which makes the prefix over the sorted masses
+// a scan over threads.
 template <int EPT>
 __global__ void __launch_bounds__(kRowThreads) route_row_kernel(const PlanArgs a) {
   constexpr int sortn = kRowThreads * EPT;
-  __shared__ double key[sortn];
-  __shared__ int idx[sortn];
+  __shared__ double xk[sortn];
+  __shared__ int xi[sortn];
   __shared__ uint8_t tier[sortn];
   __shared__ double wsum_d[kRowThreads / 32];
   __shared__ int wsum_i[kRowThreads / 32];
@@ -419,78 +491,60 @@ __global__ void __launch_bounds__(kRowThreads) route_row_kernel(const PlanArgs a
   const int nKb = a.nKb;
   const double* lrow = a.logits + g * nKb;
 
-  // pooled block softmax weighted by key counts; thread tid owns elements
-  // tid * EPT .. (contiguous), which also makes the prefix scan below a
-  // scan over threads
+  // pooled block softmax weighted by key counts
+  double kr[EPT];
+  int ir[EPT];
   double mx = -INFINITY;
+#pragma unroll
   for (int e = 0; e < EPT; ++e) {
     const int j = tid * EPT + e;
-    const double v = j < nKb ? lrow[j] : -INFINITY;
-    key[j] = v;
-    mx = fmax(mx, v);
+    kr[e] = j < nKb ? lrow[j] : -INFINITY;
+    mx = fmax(mx, kr[e]);
   }
   mx = block_reduce(mx, wsum_d, true);
   double part = 0.0;
+#pragma unroll
   for (int e = 0; e < EPT; ++e) {
     const int j = tid * EPT + e;
     if (j < nKb) {
       const int nj = min(a.bk, a.N - j * a.bk);
-      const double w = (double)nj * exp(key[j] - mx);
-      key[j] = w;
-      part += w;
+      kr[e] = (double)nj * exp(kr[e] - mx);
+      part += kr[e];
     }
   }
   const double total = block_reduce(part, wsum_d, false);
   int keep = nKb;
   if (a.router == TA_ROUTER_ENTROPY) {
     double hp = 0.0;
+#pragma unroll
     for (int e = 0; e < EPT; ++e) {
       const int j = tid * EPT + e;
       if (j < nKb) {
-        const double m = key[j] / total;
+        const double m = kr[e] / total;
         if (m > 0.0) hp -= m * log(m);
       }
     }
     const double want = a.retention * exp(block_reduce(hp, wsum_d, false));
     keep = (int)fmin((double)nKb, fmax(1.0, ceil(want)));
   }
+#pragma unroll
   for (int e = 0; e < EPT; ++e) {
     const int j = tid * EPT + e;
     if (j < nKb) {
-      const double m = key[j] / total;
-      key[j] = m;
-      idx[j] = j;
+      const double m = kr[e] / total;
+      kr[e] = m;
+      ir[e] = j;
       a.mass[g * nKb + j] = m;
       if (a.router == TA_ROUTER_PRICE)
         tier[j] = (uint8_t)price_tier(m, a.spread[g * nKb + j], a.price, a.low, a.cost[TA_TIER_SKIP],
                                       a.cost[TA_TIER_LOW], a.cost[TA_TIER_RES], a.cost[TA_TIER_FULL]);
     } else {
-      key[j] = -1.0;
-      idx[j] = 0x7fffffff - (sortn - j);
+      kr[e] = -1.0;
+      ir[e] = 0x7fffffff - (sortn - j);
     }
   }
-  __syncthreads();
 
-  // bitonic sort into (-M, j) order: position r holds (key[r], idx[r])
-  for (int size = 2; size <= sortn; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int pp = tid; pp < sortn / 2; pp += kRowThreads) {
-        const int lo = 2 * pp - (pp & (stride - 1));   // lower position of the pair
-        const int hi = lo + stride;
-        const bool up = (lo & size) == 0;               // this block sorts (-M, j) ascending
-        const double kl = key[lo], kh = key[hi];
-        const int il = idx[lo], ih = idx[hi];
-        const bool hi_first = before(kh, ih, kl, il);
-        if (up == hi_first) {
-          key[lo] = kh;
-          key[hi] = kl;
-          idx[lo] = ih;
-          idx[hi] = il;
-        }
-      }
-      __syncthreads();
-    }
-  }
+  sort_row<EPT>(kr, ir, xk, xi);   // rank tid * EPT + e now holds (kr[e], ir[e])
 
   // tiers by rank: exclusive prefix C of the sorted masses
   int codes[3];
@@ -507,13 +561,15 @@ __global__ void __launch_bounds__(kRowThreads) route_row_kernel(const PlanArgs a
   if (a.router != TA_ROUTER_PRICE) {
     const int kept_low = codes[a.n_tau - 1];
     double mine = 0.0;
-    for (int e = 0; e < EPT; ++e) mine += fmax(key[tid * EPT + e], 0.0);
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) mine += fmax(kr[e], 0.0);
     double tot;
     double C = block_excl_scan(mine, wsum_d, tot);
+#pragma unroll
     for (int e = 0; e < EPT; ++e) {
       const int r = tid * EPT + e;
-      const int j = idx[r];
-      const double mk = fmax(key[r], 0.0);
+      const int j = ir[e];
+      const double mk = fmax(kr[e], 0.0);
       if (j < nKb) {
         int t = TA_TIER_SKIP;
         for (int q = a.n_tau - 1; q >= 0; --q)
@@ -534,21 +590,21 @@ __global__ void __launch_bounds__(kRowThreads) route_row_kernel(const PlanArgs a
   // tier map row, counts and the compacted list (tiers full, res, low, skip;
   // within a tier in rank order)
   for (int j = tid; j < nKb; j += kRowThreads) a.tier_map[g * nKb + j] = tier[j];
+  uint8_t tr[EPT];
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) tr[e] = ir[e] < nKb ? tier[ir[e]] : 0xFF;
   const int order[4] = {TA_TIER_FULL, TA_TIER_RES, TA_TIER_LOW, TA_TIER_SKIP};
   int base = 0;
   for (int q = 0; q < 4; ++q) {
     const int t = order[q];
     int mine = 0;
-    for (int e = 0; e < EPT; ++e) {
-      const int j = idx[tid * EPT + e];
-      mine += (j < nKb && tier[j] == t) ? 1 : 0;
-    }
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) mine += (tr[e] == t) ? 1 : 0;
     int cnt;
     int pos = block_excl_scan_int(mine, wsum_i, cnt);
-    for (int e = 0; e < EPT; ++e) {
-      const int j = idx[tid * EPT + e];
-      if (j < nKb && tier[j] == t) a.row_lists[g * nKb + base + pos++] = j;
-    }
+#pragma unroll
+    for (int e = 0; e < EPT; ++e)
+      if (tr[e] == t) a.row_lists[g * nKb + base + pos++] = ir[e];
     if (tid == 0) a.row_counts[g * 4 + q] = cnt;
     base += cnt;
   }

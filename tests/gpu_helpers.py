@@ -74,7 +74,8 @@ def oracle_head(cfg, Q, K, V, b, h, qblocks=None, exact=False, tau=None, low=Non
     O = None
     if qblocks != []:
         O = oracle.tiered_attention_head(Qh, Kh, Vh, rt, qt, low, cfg.block_q, cfg.block_k,
-                                         cfg.p_offset_log2, rt["scale"], exact, qblocks)
+                                         cfg.p_offset_log2, rt["scale"], exact, qblocks,
+                                         key_pack=cfg.key_pack)
     return rt, qt, O
 
 

@@ -63,12 +63,13 @@ def _check_head(cfg, Q, K, V, views, O, h, qblocks):
                      qt[f"{pre}v_codes"], qt[f"{pre}v_sc"])
     sample = [i for i in qblocks if i not in rows]
     Oref = tiered_attention_head(Qh, Kh, Vh, rt, qt, cfg.low, cfg.block_q, cfg.block_k,
-                                 cfg.p_offset_log2, rt["scale"], False, sample, threads=4)
+                                 cfg.p_offset_log2, rt["scale"], False, sample, threads=4,
+                                 key_pack=cfg.key_pack)
     return assert_out_close(to64(O[0, h].cpu()), Oref, f"{cfg.name} head {h}")
 
 
 @pytest.mark.parametrize("name", ["480p", "sweep0", "sweep30", "sweep50", "sweep70", "sweep90", "720p",
-                                  "480p-price", "480p-entropy"])
+                                  "480p-price", "480p-entropy", "480p-fg"])
 def test_fullsize_sampled_parity(cuda_ok, name):
     cfg, Q, K, V, views, O = _run_full(name)
     nqb = cfg.n_qb
