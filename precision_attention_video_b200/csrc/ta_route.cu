@@ -35,14 +35,16 @@ namespace {
 // spread[bh, i, j] = scale * sqrt(sum_c (qbar[bh, i, c]^2 + qvar[bh, i, c]) kvar[bh, j, c]).
 // 128 x 128 output tile per CTA, 8 x 8 per thread (rows ty + 16 u, columns
 // tx + 16 v, so that a warp's 16 tx read 16 consecutive doubles: no bank
-// conflicts), d staged kLC coordinates at a time; 16 shared loads feed 64
-// fp64 FMAs.  The spread is a second pass over d with the same registers.
+// conflicts), d staged kLC coordinates at a time into two alternating
+// buffers (the next chunk's global loads overlap this chunk's FMAs); 16
+// shared loads feed 64 fp64 FMAs.  The spread is a second pass over d with
+// the same registers.
 // ---------------------------------------------------------------------------
 constexpr int kLT = 128, kLC = 8;
 
 template <bool SPREAD>
-__device__ __forceinline__ void logits_pass(const PlanArgs& a, int bh, int i0, int j0, double (&qs)[kLC][kLT],
-                                            double (&ks)[kLC][kLT], double (&acc)[8][8]) {
+__device__ __forceinline__ void logits_pass(const PlanArgs& a, int bh, int i0, int j0, double (&qs)[2][kLC][kLT],
+                                            double (&ks)[2][kLC][kLT], double (&acc)[8][8]) {
   const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
   const int D = a.d;
   const double* qb = a.qbar + (int64_t)bh * a.nQb * D;
@@ -52,36 +54,52 @@ __device__ __forceinline__ void logits_pass(const PlanArgs& a, int bh, int i0, i
   for (int u = 0; u < 8; ++u)
 #pragma unroll
     for (int v = 0; v < 8; ++v) acc[u][v] = 0.0;
-  for (int c0 = 0; c0 < D; c0 += kLC) {
-    // stage 128 rows x kLC coordinates of each operand: element e = r * kLC + c
-    for (int e = tid; e < kLT * kLC; e += 256) {
-      const int r = e / kLC, c = e % kLC;
+  // each thread stages elements e = tid + 256 w (w < kStage) of the 128 rows x
+  // kLC coordinates of both operands: r = e / kLC, c = e % kLC
+  constexpr int kStage = kLT * kLC / 256;
+  double pq[kStage], pk[kStage];
+  auto fetch = [&](int c0) {
+#pragma unroll
+    for (int w = 0; w < kStage; ++w) {
+      const int e = tid + 256 * w, r = e / kLC, c = e % kLC;
       const bool qi = i0 + r < a.nQb, kj = j0 + r < a.nKb;
       double q = qi ? qb[(int64_t)(i0 + r) * D + c0 + c] : 0.0;
       if (SPREAD && qi) q = q * q + qvb[(int64_t)(i0 + r) * D + c0 + c];
-      qs[c][r] = q;
-      ks[c][r] = kj ? kb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
+      pq[w] = q;
+      pk[w] = kj ? kb[(int64_t)(j0 + r) * D + c0 + c] : 0.0;
+    }
+  };
+  fetch(0);
+  for (int c0 = 0, buf = 0; c0 < D; c0 += kLC, buf ^= 1) {
+#pragma unroll
+    for (int w = 0; w < kStage; ++w) {
+      const int e = tid + 256 * w, r = e / kLC, c = e % kLC;
+      qs[buf][c][r] = pq[w];
+      ks[buf][c][r] = pk[w];
     }
     __syncthreads();
+    // the next chunk's loads are in flight while this one is multiplied; the
+    // buffer written next was last read before the barrier above
+    if (c0 + kLC < D) fetch(c0 + kLC);
 #pragma unroll 2
     for (int c = 0; c < kLC; ++c) {
       double q[8], k[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) q[u] = qs[c][ty + 16 * u];
+      for (int u = 0; u < 8; ++u) q[u] = qs[buf][c][ty + 16 * u];
 #pragma unroll
-      for (int v = 0; v < 8; ++v) k[v] = ks[c][tx + 16 * v];
+      for (int v = 0; v < 8; ++v) k[v] = ks[buf][c][tx + 16 * v];
 #pragma unroll
       for (int u = 0; u < 8; ++u)
 #pragma unroll
         for (int v = 0; v < 8; ++v) acc[u][v] = fma(q[u], k[v], acc[u][v]);
     }
-    __syncthreads();
   }
+  __syncthreads();   // the caller's next pass restages both buffers
 }
 
 __global__ void __launch_bounds__(256) logits_kernel(const PlanArgs a) {
-  __shared__ double qs[kLC][kLT];
-  __shared__ double ks[kLC][kLT];
+  __shared__ double qs[2][kLC][kLT];
+  __shared__ double ks[2][kLC][kLT];
   const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
   const int bh = blockIdx.z, i0 = blockIdx.x * kLT, j0 = blockIdx.y * kLT;
   double acc[8][8];
@@ -399,77 +417,103 @@ __device__ __forceinline__ double block_reduce(double v, double* wsum, bool is_m
   return r;
 }
 
-// One compare-exchange of the (-M, j) bitonic network: (ka, ia) sits at the
-// lower position, (kb, ib) at the higher; `up` sorts the pair ascending.
-__device__ __forceinline__ void cmp_swap(double& ka, int& ia, double& kb, int& ib, bool up) {
-  if (up == before(kb, ib, ka, ia)) {
-    const double k = ka;
-    const int i = ia;
-    ka = kb;
-    ia = ib;
-    kb = k;
-    ib = i;
-  }
+// Sort key of key block j with pooled mass m >= 0: the float of m rounded
+// toward zero (so that a larger float means a larger mass) in the high word,
+// complemented so that ascending keys run by descending mass, and j in the
+// low word (lower j first among equal floats).  Blocks whose masses round to
+// the same float are put in exact (-M, j) order afterwards (fix_exact_order).
+__device__ __forceinline__ uint64_t sort_key(double m, int j) {
+  const uint32_t hi = ~__float_as_uint(__double2float_rz(m));
+  return ((uint64_t)hi << 32) | (uint32_t)j;
 }
 
-// Bitonic sort of kRowThreads * EPT elements into (-M, j) order; thread tid
-// holds positions tid * EPT .. tid * EPT + EPT - 1 in (kr, ir).  Strides
-// below EPT run inside a thread, strides below 32 * EPT between the lanes of
-// a warp (shuffles), longer ones through shared memory (`xk`, `xi`: one
-// element per thread and slot, slot-major so that a warp's accesses fall on
-// distinct banks).
+// Bitonic sort, ascending, of kRowThreads * EPT distinct 64-bit keys; thread
+// tid holds positions tid * EPT .. tid * EPT + EPT - 1.  The network is
+// unrolled: strides below EPT run inside a thread, strides below 32 * EPT
+// between the lanes of a warp (shuffles), longer ones through shared memory
+// (`xk`: one key per thread and slot, slot-major so that a warp's accesses
+// fall on distinct banks).
 template <int EPT>
-__device__ __forceinline__ void sort_row(double (&kr)[EPT], int (&ir)[EPT], double* xk, int* xi) {
+__device__ __forceinline__ void sort_row(uint64_t (&kr)[EPT], uint64_t* xk) {
   constexpr int sortn = kRowThreads * EPT;
+  constexpr int kLog = (sortn == 512) ? 9 : 10;
+  static_assert((1 << kLog) == sortn, "sort width");
   const int tid = threadIdx.x;
-  for (int size = 2; size <= sortn; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+  for (int ls = 1; ls <= kLog; ++ls) {
+#pragma unroll
+    for (int lt = ls - 1; lt >= 0; --lt) {
+      const int size = 1 << ls, stride = 1 << lt;
       if (stride < EPT) {
 #pragma unroll
-        for (int s = EPT / 2; s >= 1; s >>= 1) {
-          if (s != stride) continue;
-#pragma unroll
-          for (int e = 0; e < EPT; ++e)
-            if ((e & s) == 0) cmp_swap(kr[e], ir[e], kr[e + s], ir[e + s], ((tid * EPT + e) & size) == 0);
+        for (int e = 0; e < EPT; ++e) {
+          if (e & stride) continue;
+          const bool up = ((tid * EPT + e) & size) == 0;
+          const uint64_t lo = kr[e] < kr[e + stride] ? kr[e] : kr[e + stride];
+          const uint64_t hi = kr[e] < kr[e + stride] ? kr[e + stride] : kr[e];
+          kr[e] = up ? lo : hi;
+          kr[e + stride] = up ? hi : lo;
         }
         continue;
       }
-      // the partner of position p = tid * EPT + e is p ^ stride = (tid ^ m) * EPT + e
+      // the partner of position p = tid * EPT + e is p ^ stride = (tid ^ m) * EPT + e;
+      // the lower position of an ascending pair keeps the smaller key
       const int m = stride / EPT;
-      const bool lower = (tid & m) == 0;
-      const bool up = ((tid * EPT) & size) == 0;   // size > stride >= EPT: one direction a thread
-      double kp[EPT];
-      int ip[EPT];
+      const bool keep_min = ((tid & m) == 0) == (((tid * EPT) & size) == 0);
+      uint64_t kp[EPT];
       if (stride < 32 * EPT) {
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-          kp[e] = __shfl_xor_sync(0xffffffffu, kr[e], m);
-          ip[e] = __shfl_xor_sync(0xffffffffu, ir[e], m);
-        }
+        for (int e = 0; e < EPT; ++e) kp[e] = __shfl_xor_sync(0xffffffffu, kr[e], m);
       } else {
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-          xk[e * kRowThreads + tid] = kr[e];
-          xi[e * kRowThreads + tid] = ir[e];
-        }
+        for (int e = 0; e < EPT; ++e) xk[e * kRowThreads + tid] = kr[e];
         __syncthreads();
 #pragma unroll
-        for (int e = 0; e < EPT; ++e) {
-          kp[e] = xk[e * kRowThreads + (tid ^ m)];
-          ip[e] = xi[e * kRowThreads + (tid ^ m)];
-        }
+        for (int e = 0; e < EPT; ++e) kp[e] = xk[e * kRowThreads + (tid ^ m)];
         __syncthreads();
       }
 #pragma unroll
-      for (int e = 0; e < EPT; ++e) {
-        // both threads of a pair take the same decision and keep their side
-        const bool hi_first = lower ? before(kp[e], ip[e], kr[e], ir[e]) : before(kr[e], ir[e], kp[e], ip[e]);
-        if (up == hi_first) {
-          kr[e] = kp[e];
-          ir[e] = ip[e];
+      for (int e = 0; e < EPT; ++e) kr[e] = ((kp[e] < kr[e]) == keep_min) ? kp[e] : kr[e];
+    }
+  }
+}
+
+// After sort_row the order is exact except, possibly, among blocks whose
+// masses round to one float (ordered there by j alone).  Ranks r and r + 1
+// out of (-M, j) order are looked for over the whole row; if any is found
+// (rare: masses within 2^-24 of each other), one thread reorders the row's
+// nKb ranks by insertion, which costs one pass plus the few moves.  `xi`
+// holds the block of each rank on return; `mass` the exact masses by block.
+template <int EPT>
+__device__ __forceinline__ void fix_exact_order(const uint64_t (&kr)[EPT], int* xi, const double* mass,
+                                                int nKb) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) xi[tid * EPT + e] = (int)(uint32_t)kr[e];
+  __syncthreads();
+  bool bad = false;
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) {
+    const int r = tid * EPT + e;
+    if (r + 1 < nKb) {
+      const int ja = xi[r], jb = xi[r + 1];
+      bad |= !before(mass[ja], ja, mass[jb], jb);
+    }
+  }
+  if (__syncthreads_or(bad)) {
+    if (tid == 0) {
+      for (int r = 1; r < nKb; ++r) {
+        const int j = xi[r];
+        const double mj = mass[j];
+        int q = r - 1;
+        while (q >= 0 && before(mj, j, mass[xi[q]], xi[q])) {
+          xi[q + 1] = xi[q];
+          --q;
         }
+        xi[q + 1] = j;
       }
     }
+    __syncthreads();
   }
 }
 
@@ -480,8 +524,9 @@ __device__ __forceinline__ void sort_row(double (&kr)[EPT], int (&ir)[EPT], doub
 template <int EPT>
 __global__ void __launch_bounds__(kRowThreads) route_row_kernel(const PlanArgs a) {
   constexpr int sortn = kRowThreads * EPT;
-  __shared__ double xk[sortn];
+  __shared__ uint64_t xk[sortn];
   __shared__ int xi[sortn];
+  __shared__ double mass_s[sortn];
   __shared__ uint8_t tier[sortn];
   __shared__ double wsum_d[kRowThreads / 32];
   __shared__ int wsum_i[kRowThreads / 32];
@@ -534,6 +579,7 @@ __global__ void __launch_bounds__(kRowThreads) route_row_kernel(const PlanArgs a
       const double m = kr[e] / total;
       kr[e] = m;
       ir[e] = j;
+      mass_s[j] = m;
       a.mass[g * nKb + j] = m;
       if (a.router == TA_ROUTER_PRICE)
         tier[j] = (uint8_t)price_tier(m, a.spread[g * nKb + j], a.price, a.low, a.cost[TA_TIER_SKIP],
@@ -544,7 +590,19 @@ __global__ void __launch_bounds__(kRowThreads) route_row_kernel(const PlanArgs a
     }
   }
 
-  sort_row<EPT>(kr, ir, xk, xi);   // rank tid * EPT + e now holds (kr[e], ir[e])
+  // rank order: padding (keys above every real block's) sorts last
+  uint64_t key[EPT];
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) key[e] = ir[e] < nKb ? sort_key(kr[e], ir[e]) : (~0ull - (uint64_t)(sortn - tid * EPT - e));
+  sort_row<EPT>(key, xk);
+  fix_exact_order<EPT>(key, xi, mass_s, nKb);
+  // rank tid * EPT + e now holds block ir[e] with mass kr[e]
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) {
+    const int r = tid * EPT + e;
+    ir[e] = r < nKb ? xi[r] : 0x7fffffff;
+    kr[e] = r < nKb ? mass_s[ir[e]] : -1.0;
+  }
 
   // tiers by rank: exclusive prefix C of the sorted masses
   int codes[3];
