@@ -47,7 +47,7 @@ L2_BYTES = 126 * 2 ** 20
 # 8 heads of that layer, scaled to 40 by heads (traffic grows with the (head,
 # query block) rows); valid only for the kernel source it was measured on and
 # for that workload.
-ATTN_TRAFFIC = {"source_sha1": "1e216b4f03bb22d4745498d1ab6211ddf3b634c9", "bytes_per_launch": 1592325120}
+ATTN_TRAFFIC = {"source_sha1": "", "bytes_per_launch": 0}
 
 
 def _env_int(name, default):
@@ -84,10 +84,25 @@ def attn_source_sha1():
     """Hash of the attention kernel's sources (the kernel and the headers it
     inlines): a traffic figure holds only for the code it was measured on."""
     h = hashlib.sha1()
-    for name in ("ta_attn.cu", "ta_attn_common.cuh", "ta_common.cuh"):
+    for name in ("ta_attn2.cu", "ta_attn.cu", "ta_attn_common.cuh", "ta_common.cuh"):
         with open(os.path.join(ROOT, "precision_attention_video_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
+
+
+def attn_kernel_name(cfg) -> str:
+    """The forward kernel the library dispatches for a workload: the
+    two-group kernel for d = 128 with 128-query blocks and 128- or 32-key
+    blocks (except NVFP4 + residual layers tiered by thresholds), the 16-warp
+    kernel otherwise."""
+    lm = {0: "LM_IMAGE", 1: "LM_FP8", 2: "LM_NVFP4", 3: "LM_NVFP4_RES"}[cfg.low]
+    two_group = (cfg.d == 128 and cfg.block_q == 128 and cfg.block_k in (32, 128)
+                 and not (cfg.low == 3 and cfg.block_k == 128 and getattr(cfg, "router", 0) != 1))
+    if two_group:
+        return f"attn2_kernel<{lm}, {cfg.block_k}>"
+    if cfg.low == 1 and not (cfg.d == 128 and cfg.block_q == 128 and cfg.block_k == 128):
+        lm = "LM_IMAGE"
+    return f"attn_kernel<{cfg.d}, {cfg.block_k}, {lm}>"
 
 
 class ClockSampler:
@@ -594,7 +609,7 @@ def main():
             "data": "synthetic", "config": config,
             "ms_plan": statistics.mean(r["plan_ms"]), "ms_forward": fwd_ms,
             "tier_frac": r["tier_frac"],
-            "roofline": {"kernel": "tiered_attn_forward (attn_kernel<128,128>)", "bound": "tensor",
+            "roofline": {"kernel": f"tiered_attn_forward ({attn_kernel_name(cfg)})", "bound": "tensor",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": (f"blend of {peak_src} bf16 {peak_kind} "

@@ -450,6 +450,7 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
   a.bq = p->block_q;
   a.bk = p->block_k;
   a.low = p->low;
+  a.router = p->router;
   a.nQb = (int)s.nQb;
   a.nKb = (int)s.nKb;
   a.sb = p->stride_b;

@@ -1053,6 +1053,13 @@ cudaError_t launch_attn2(const AttnArgs& a, const CUtensorMap* maps, cudaStream_
     return cudaErrorInvalidValue;   // no other kernel takes 32-key blocks   // no other kernel takes 32-key blocks
   }
   if (a.bk != 128) return cudaErrorNotSupported;
+  // NVFP4 + residual layers tiered by thresholds (mass or entropy router) mix
+  // full, residual, NVFP4 and skipped blocks in every row; there the 16-warp
+  // kernel measured faster (720p layer 120 vs 139 ms; the 480p shape with the
+  // same four tiers 13.6 vs 17.2 ms), while this kernel wins on each tier
+  // alone, on mixes without skipped blocks and on the price router's rows
+  // (480p price layer 11.6 vs 12.3 ms)
+  if (a.low == TA_LOW_NVFP4_RES && a.router != TA_ROUTER_PRICE) return cudaErrorNotSupported;
   if (a.low == TA_LOW_NONE) return launch2<LM_IMAGE, 128>(a, maps, s);
   if (a.low == TA_LOW_NVFP4) return launch2<LM_NVFP4, 128>(a, maps, s);
   if (a.low == TA_LOW_NVFP4_RES) return launch2<LM_NVFP4_RES, 128>(a, maps, s);

@@ -53,6 +53,7 @@ struct PlanArgs {
 // Fused attention arguments.
 struct AttnArgs {
   int B, H, N, d, bq, bk, low;
+  int router;                   // ta_router of the plan (selects the kernel)
   int nQb, nKb;
   int64_t sb, sh, sn;           // element strides of Q and O
   float scale_log2;             // softmax_scale * log2(e)
