@@ -43,11 +43,11 @@ UNIT = "TFLOPS"
 L2_BYTES = 126 * 2 ** 20
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one forward
-# launch of the 480p-video-like layer, from the ncu capture of this kernel on
-# 8 heads of that layer, scaled to 40 by heads (traffic grows with the (head,
-# query block) rows); valid only for the kernel source it was measured on and
-# for that workload.
-ATTN_TRAFFIC = {"source_sha1": "", "bytes_per_launch": 0}
+# launch of the 480p-video-like layer, from the ncu capture of the two-group
+# kernel (attn2_kernel<LM_NVFP4, 128>) on 8 heads of that layer, scaled to 40
+# by heads (traffic grows with the (head, query block) rows); valid only for
+# the kernel sources it was measured on and for that workload.
+ATTN_TRAFFIC = {"source_sha1": "bbc9a9fcd43ca187737ecadeef396da59666b9f3", "bytes_per_launch": 1604586240}
 
 
 def _env_int(name, default):
@@ -84,7 +84,7 @@ def attn_source_sha1():
     """Hash of the attention kernel's sources (the kernel and the headers it
     inlines): a traffic figure holds only for the code it was measured on."""
     h = hashlib.sha1()
-    for name in ("ta_attn2.cu", "ta_attn.cu", "ta_attn_common.cuh", "ta_common.cuh"):
+    for name in ("ta_attn2.cu", "ta_attn_common.cuh", "ta_common.cuh", "ta_kernels.cuh"):
         with open(os.path.join(ROOT, "precision_attention_video_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -100,8 +100,6 @@ def attn_kernel_name(cfg) -> str:
                  and not (cfg.low == 3 and cfg.block_k == 128 and getattr(cfg, "router", 0) != 1))
     if two_group:
         return f"attn2_kernel<{lm}, {cfg.block_k}>"
-    if cfg.low == 1 and not (cfg.d == 128 and cfg.block_q == 128 and cfg.block_k == 128):
-        lm = "LM_IMAGE"
     return f"attn_kernel<{cfg.d}, {cfg.block_k}, {lm}>"
 
 
@@ -586,12 +584,10 @@ def main():
     peaks, peak_src = load_peaks()
     p_bf16, peak_kind = bf16_peak(peaks, r["clocks"])
     # Full tiles and skip chunks run on the bf16 pipe; NVFP4 tiles (low and
-    # residual) on the FP4 pipe and native FP8 tiles (d = 128, 128 x 128) on
-    # the FP8 pipe, whose peaks are taken as 4x and 2x the measured bf16 one
-    # (the nominal ratios); FP8 tiles of other shapes run on bf16 images.
-    native_f8 = cfg.d == 128 and cfg.block_q == 128 and cfg.block_k == 128
+    # residual) on the FP4 pipe and FP8 tiles on the FP8 pipe, whose peaks are
+    # taken as 4x and 2x the measured bf16 one (the nominal ratios).
     p_fp4 = 4.0 * p_bf16
-    p_low = {1: (2.0 if native_f8 else 1.0) * p_bf16, 2: p_fp4, 3: p_fp4}.get(cfg.low, p_bf16)
+    p_low = {1: 2.0 * p_bf16, 2: p_fp4, 3: p_fp4}.get(cfg.low, p_bf16)
     executed = r["full_flops"] + r["res_flops"] + r["low_flops"] + r["skip_flops"]
     t_min = ((r["full_flops"] + r["skip_flops"]) / (p_bf16 * 1e12) + r["res_flops"] / (p_fp4 * 1e12)
              + r["low_flops"] / (p_low * 1e12))

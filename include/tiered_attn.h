@@ -160,10 +160,8 @@ typedef struct {
   /* residual NVFP4 copies (TA_LOW_NVFP4_RES), same layouts as above */
   uint8_t* rq_codes; uint8_t* rk_codes; uint8_t* rv_codes;
   uint8_t* rq_scales; uint8_t* rk_scales; uint8_t* rv_scales;
-  /* bf16 [BH, N, d] dequantised values of the FP8 copies (exact in bf16);
-   * present only for an FP8 low tier with d = 64 or 64-row tiles, whose
-   * tiles run on these images (128 x 128 FP8 tiles and every NVFP4 tile run
-   * on the codes and scales directly) */
+  /* always NULL: every FP8 and NVFP4 tile runs on the codes and scales, and
+   * no bf16 image of a low copy is kept (the fields keep the struct's layout) */
   uint16_t* dq; uint16_t* dk; uint16_t* dv;
   /* always NULL: no bf16 image of the residual copies is kept */
   uint16_t* drq; uint16_t* drk; uint16_t* drv;
@@ -184,9 +182,8 @@ size_t tiered_attn_workspace_bytes(const ta_params* p);
 
 /* Router + quantiser ("Triage" abstract: the router predicts from block
  * statistics; NVFP4 skim / refine copies).  Reads Q, K, V once: block means of
- * Q, K, V (fp64), the low-precision copies of Q, K, V (and, for an FP8 low
- * tier the kernel runs on images, their dequantised bf16 values); then the
- * pooled logits, the
+ * Q, K, V (fp64), the low-precision copies of Q, K, V; then the pooled
+ * logits, the
  * n_j-weighted pooled block softmax M, the tiers, and the per-row tile lists.
  * Tiers:
  *  - TA_ROUTER_MASS: by exclusive cumulative mass in (-M, j) order (most

@@ -86,10 +86,6 @@ ta_status validate(const ta_params* p) {
   return TA_OK;
 }
 
-// FP8 low tiles run on the FP8 tensor pipe for d = 128 with 128 x 128 tiles.
-bool native_fp8(const ta_params* p) {
-  return p->low == TA_LOW_FP8_E4M3 && p->d == 128 && p->block_q == 128 && p->block_k == 128;
-}
 
 // Workspace layout: byte offsets of every array (kAbsent when not produced).
 struct Layout {
@@ -149,13 +145,7 @@ Layout layout_of(const ta_params* p) {
       }
     }
   }
-  // bf16 images of the low copies: only FP8 tiles of d = 64 or 64-row tiles
-  // read them; NVFP4 (+ residual) and 128 x 128 FP8 tiles run natively on the codes
-  if (p->low == TA_LOW_FP8_E4M3 && !native_fp8(p)) {
-    L.dq = take(tok * 2);
-    L.dk = take(tok * 2);
-    L.dv = take(tok * 2);
-  }
+  // (no bf16 images of the low copies: FP8 and NVFP4 tiles run on the codes)
   L.total = off;
   return L;
 }
@@ -479,7 +469,6 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
   a.rv_sf = at<uint8_t>(ws, L.rv_scales);
 
   CUtensorMap maps[9];
-  const int64_t cb = (int64_t)p->H * p->N * p->d, ch = (int64_t)p->N * p->d, cn = p->d;
   bool ok = make_map(&maps[0], Q, p->B, p->H, p->N, p->d, p->stride_b, p->stride_h, p->stride_n, p->block_q) &&
             make_map(&maps[1], K, p->B, p->H, p->N, p->d, p->stride_b, p->stride_h, p->stride_n, p->block_k) &&
             make_map(&maps[2], V, p->B, p->H, p->N, p->d, p->stride_b, p->stride_h, p->stride_n, p->block_k);
@@ -499,18 +488,12 @@ ta_status tiered_attn_forward(const ta_params* p, const void* Q, const void* K, 
       maps[7] = maps[4];
       maps[8] = maps[5];
     }
-  } else if (native_fp8(p)) {
+  } else if (p->low == TA_LOW_FP8_E4M3) {
+    // FP8 codes, rows of d bytes (128- or 64-byte swizzle)
     const int64_t BH = (int64_t)p->B * p->H;
-    ok = ok && make_map_u8(&maps[3], at<void>(ws, L.q_codes), BH, p->N, p->d, p->block_q, 128) &&
-         make_map_u8(&maps[4], at<void>(ws, L.k_codes), BH, p->N, p->d, p->block_k, 128) &&
-         make_map_u8(&maps[5], at<void>(ws, L.v_codes), BH, p->N, p->d, p->block_k, 128);
-  } else if (L.dq != kAbsent) {
-    const void* dq = at<void>(ws, L.dq);
-    const void* dk = at<void>(ws, L.dk);
-    const void* dv = at<void>(ws, L.dv);
-    ok = ok && make_map(&maps[3], dq, p->B, p->H, p->N, p->d, cb, ch, cn, p->block_q) &&
-         make_map(&maps[4], dk, p->B, p->H, p->N, p->d, cb, ch, cn, p->block_k) &&
-         make_map(&maps[5], dv, p->B, p->H, p->N, p->d, cb, ch, cn, p->block_k);
+    ok = ok && make_map_u8(&maps[3], at<void>(ws, L.q_codes), BH, p->N, p->d, p->block_q, p->d) &&
+         make_map_u8(&maps[4], at<void>(ws, L.k_codes), BH, p->N, p->d, p->block_k, p->d) &&
+         make_map_u8(&maps[5], at<void>(ws, L.v_codes), BH, p->N, p->d, p->block_k, p->d);
   } else {
     maps[3] = maps[0];
     maps[4] = maps[1];

@@ -18,12 +18,12 @@
 //   warp 4S+2   S issuer: S = Q K^T into a double-buffered TMEM accumulator,
 //               as soon as the softmax has read the buffer's previous S;
 //   warp 4S+3   PV issuer: O += P V into a TMEM accumulator.  One thread each
-//               issues tcgen05.mma: kind::f16 for full and skip tiles and for
-//               FP8 tiles of the small shapes (bf16 images of the codes);
+//               issues tcgen05.mma: kind::f16 for full and skip tiles;
 //               kind::mxf4nvf4.block16 for NVFP4 tiles (ue4m3 scales copied
 //               to TMEM with tcgen05.cp; three MMAs per product on residual
 //               tiles); kind::f8f6f4 for FP8 S and kind::mxf8f6f4 for FP8 PV
-//               (V's power-of-two tile scale as a UE8M0 block scale).  Two
+//               (V's power-of-two tile scale as a UE8M0 block scale; d = 64
+//               or 64-key tiles use 64-byte-swizzled FP8 rows).  Two
 //               threads, because one thread issues an N <= 128 MMA only every
 //               ~100 cycles.  Completion is signalled with tcgen05.commit on
 //               mbarriers;
@@ -91,7 +91,8 @@ struct Smem {
   static constexpr int kQ = 128 * D * 2;      // one query tile, 128 rows
   static constexpr int kKV = BK * D * 2;      // one K or V tile
   static constexpr int kPfp4 = 128 * 64 + 1024;  // one NVFP4 tile: codes + scales
-  static constexpr int kF8 = 128 * 128;                // one FP8 tile (128 rows x 128 B)
+  static constexpr int kF8 = 128 * 128;                // an FP8 Q or P buffer (128 rows x up to 128 B)
+  static constexpr int kF8KV = BK * D;                 // an FP8 K or V tile; V's scales follow it
   static constexpr int kQlow = FP4 ? NC * kPfp4 : (F8 ? kF8 : kQ);  // low query copies
   // P: bf16 P lives in TMEM; NVFP4 / FP8 P in two shared-memory buffers
   static constexpr int kP = FP4 ? 2 * NC * kPfp4 : (F8 ? 2 * kF8 + 1024 : 0);
@@ -121,7 +122,7 @@ enum {
 };
 
 // Formats of P' in the softmax's tile tail.
-enum { PK_BF16 = 0, PK_SKIP = 1, PK_FP4 = 2, PK_RES = 3, PK_F8 = 4, PK_IMG_F8 = 5 };
+enum { PK_BF16 = 0, PK_SKIP = 1, PK_FP4 = 2, PK_RES = 3, PK_F8 = 4 };
 
 // What the tail of one tile's softmax needs (one thread: one query row, one
 // column part of HB keys).
@@ -205,13 +206,6 @@ __device__ __forceinline__ bool softmax_tail(const SoftmaxTail q, float& psum) {
 #pragma unroll
     for (int c = 0; c < HB; c += 4)
       p[c / 4] = cvt_e4m3x2(x[c], x[c + 1]) | (cvt_e4m3x2(x[c + 2], x[c + 3]) << 16);
-  } else if constexpr (PK == PK_IMG_F8) {
-    // e4m3 rounding of P', carried exactly in bf16
-#pragma unroll
-    for (int c = 0; c < HB; c += 2) {
-      const float2 f = e4m3x2_to_float2(cvt_e4m3x2(x[c], x[c + 1]));
-      p[c / 2] = pack_bf16(f.x, f.y);
-    }
   } else {
 #pragma unroll
     for (int c = 0; c < HB; c += 2) p[c / 2] = pack_bf16(x[c], x[c + 1]);
@@ -261,13 +255,15 @@ __device__ __forceinline__ bool softmax_tail(const SoftmaxTail q, float& psum) {
       *reinterpret_cast<uint16_t*>(pbuf + L::kPfp4 + soff) = (uint16_t)p[12];
     }
   } else if constexpr (PK == PK_F8) {
-    // FP8 P part: 32 codes into the 128-byte-swizzled tile of buffer s
+    // FP8 P part: HB codes into the tile of buffer s, rows of BK bytes,
+    // 128-byte swizzle (BK = 128) or 64-byte swizzle (BK = 64)
     unsigned char* pbuf = q.sm + L::oP + s * L::kF8;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int ch = q.part * 2 + h;
-      *reinterpret_cast<uint4*>(pbuf + q.r * 128 + ((ch ^ (q.r & 7)) * 16)) =
-          make_uint4(p[h * 4 + 0], p[h * 4 + 1], p[h * 4 + 2], p[h * 4 + 3]);
+    for (int h = 0; h < HB / 16; ++h) {
+      const int ch = q.part * (HB / 16) + h;
+      const uint32_t off = (BK == 128) ? q.r * 128 + ((ch ^ (q.r & 7)) * 16)
+                                       : q.r * 64 + ((ch ^ ((q.r >> 1) & 3)) * 16);
+      *reinterpret_cast<uint4*>(pbuf + off) = make_uint4(p[h * 4 + 0], p[h * 4 + 1], p[h * 4 + 2], p[h * 4 + 3]);
     }
   } else {
     // bf16 P' of this part into the TMEM P columns
@@ -295,8 +291,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
   constexpr int kSplit = RL::kSplit, kSoftmaxWarps = RL::kSoftmaxWarps;
   constexpr int kProducerKWarp = RL::kProducerKWarp, kProducerVWarp = RL::kProducerVWarp;
   constexpr int kMmaWarp = RL::kMmaWarp, kPvWarp = RL::kPvWarp;
-  static_assert(!(FP4 || F8) || (D == 128 && BK == 128),
-                "native NVFP4 / FP8 tiles need d = 128, 128-key tiles");
+  static_assert(!FP4 || (D == 128 && BK == 128), "native NVFP4 tiles need d = 128, 128-key tiles");
   constexpr uint32_t kTmemCols = TS::kCols;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = smem_raw;
@@ -411,7 +406,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         tma_prefetch_desc(&tmK);
         const uint32_t qbytes = (uint32_t)a.bq * D * 2;
         const uint32_t lbytes = FP4 ? (uint32_t)(nq * a.bq * 64)
-                                : (has_low ? (F8 ? (uint32_t)a.bq * 128 : qbytes) : 0u);
+                                : (has_low ? (F8 ? (uint32_t)a.bq * D : qbytes) : 0u);
         mbar_arrive_expect_tx(&bars[BAR_Q], qbytes + lbytes);
         for (int x = 0; x < D / 64; ++x)
           tma_load_4d(sm + L::oQ + x * (128 * 128), &tmQ, &bars[BAR_Q], x * 64, q0, h, b);
@@ -493,17 +488,17 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         if (!isK) {
           // UE8M0 scale factor of this V tile: the exponent of its power-of-two scale
           const uint32_t e = (__float_as_uint(a.v_s8[(int64_t)bh * a.nKb + j]) >> 23) & 0xFFu;
-          reinterpret_cast<uint32_t*>(st + L::kF8)[lane * 4 + 0] = e * 0x01010101u;
-          reinterpret_cast<uint32_t*>(st + L::kF8)[lane * 4 + 1] = e * 0x01010101u;
-          reinterpret_cast<uint32_t*>(st + L::kF8)[lane * 4 + 2] = e * 0x01010101u;
-          reinterpret_cast<uint32_t*>(st + L::kF8)[lane * 4 + 3] = e * 0x01010101u;
+          reinterpret_cast<uint32_t*>(st + L::kF8KV)[lane * 4 + 0] = e * 0x01010101u;
+          reinterpret_cast<uint32_t*>(st + L::kF8KV)[lane * 4 + 1] = e * 0x01010101u;
+          reinterpret_cast<uint32_t*>(st + L::kF8KV)[lane * 4 + 2] = e * 0x01010101u;
+          reinterpret_cast<uint32_t*>(st + L::kF8KV)[lane * 4 + 3] = e * 0x01010101u;
           fence_proxy_async_smem();
         }
         __syncwarp();
         if (lane == 0) {
           const bool drop = isK && (t == 0) && (a.debug_flags & TA_DEBUG_DROP_FIRST_K);
           if (!drop) {
-            mbar_arrive_expect_tx(&full[s], BK * 128);
+            mbar_arrive_expect_tx(&full[s], BK * D);
             tma_load_3d(st, isK ? &tmDK : &tmDV, &full[s], 0, j * BK, bh);
             issued[s]++;
           }
@@ -606,11 +601,17 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
             }
           }
         } else if (F8 && kind == KIND_LOW) {
-          // FP8 codes: 4 MMAs of K = 32 over the 128-byte rows (scales applied in softmax)
+          // FP8 codes: D / 32 MMAs of K = 32 over the D-byte rows, 128- or
+          // 64-byte swizzled (scales applied in the softmax)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f8_ss(d, smem_desc_sw128(aq + kk * 32, 16, 1024),
-                      smem_desc_sw128(sk + kk * 32, 16, 1024), idesc_f8(128, BK), kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 32; ++kk) {
+            if constexpr (D == 128)
+              mma_f8_ss(d, smem_desc_sw128(aq + kk * 32, 16, 1024),
+                        smem_desc_sw128(sk + kk * 32, 16, 1024), idesc_f8(128, BK), kk > 0 ? 1u : 0u);
+            else
+              mma_f8_ss(d, smem_desc_sw64(aq + kk * 32), smem_desc_sw64(sk + kk * 32), idesc_f8(128, BK),
+                        kk > 0 ? 1u : 0u);
+          }
         } else {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -672,12 +673,17 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
           // FP8 P codes (scale 2^0) x FP8 V codes (MN-major) with V's power-of-two
           // tile scale as the UE8M0 block scale
           const uint32_t pb = sP + s * L::kF8;
-          tc_cp_sf(tmem + TS::sfbV8(), smem_desc_rows16(sv + L::kF8));
+          tc_cp_sf(tmem + TS::sfbV8(), smem_desc_rows16(sv + L::kF8KV));
+          // BK / 32 MMAs of K = 32 keys: P rows of BK bytes (K-major), V rows
+          // of D bytes (MN-major), each 128- or 64-byte swizzled
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_mxf8_ss(tO, smem_desc_sw128(pb + kk * 32, 16, 1024),
-                        smem_desc_sw128(sv + kk * 32 * 128, 16, 1024), idesc_mxf8_bmn(128, D),
-                        tmem + TS::sfaP8(), tmem + TS::sfbV8(), (t > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BK / 32; ++kk) {
+            const uint64_t ad = (BK == 128) ? smem_desc_sw128(pb + kk * 32, 16, 1024) : smem_desc_sw64(pb + kk * 32);
+            const uint64_t bd = (D == 128) ? smem_desc_sw128(sv + kk * 32 * 128, 16, 1024)
+                                           : smem_desc_sw64(sv + kk * 32 * 64);
+            mma_mxf8_ss(tO, ad, bd, idesc_mxf8_bmn(128, D), tmem + TS::sfaP8(), tmem + TS::sfbV8(),
+                        (t > 0 || kk > 0) ? 1u : 0u);
+          }
         } else {
           // A = bf16 P' in the TMEM P columns
 #pragma unroll
@@ -796,7 +802,7 @@ __global__ void __launch_bounds__(Roles<D, BK>::kThreads, 1)
         } else if constexpr (F8) {
           ok3 = softmax_tail<PK_F8, D, BK, LM>(q, psum);
         } else {
-          ok3 = softmax_tail<PK_IMG_F8, D, BK, LM>(q, psum);
+          ok3 = false;   // no low tier in this instance: not reached
         }
       }
       // a failed wait leaves the loop at the next row barrier, with the other
@@ -872,12 +878,18 @@ cudaError_t launch_attn(const AttnArgs& a, const CUtensorMap* maps, cudaStream_t
   // d = 128 with 128 x 128 tiles runs on the two-group kernel (ta_attn2.cu)
   const cudaError_t e2 = launch_attn2(a, maps, s);
   if (e2 != cudaErrorNotSupported) return e2;
+  // FP8 low tiles run natively on the FP8 tensor pipe at every shape
+  if (a.low == TA_LOW_FP8_E4M3) {
+    if (a.d == 64 && a.bk == 64) return launch_d<64, 64, LM_FP8>(a, maps, s);
+    if (a.d == 64 && a.bk == 128) return launch_d<64, 128, LM_FP8>(a, maps, s);
+    if (a.d == 128 && a.bk == 64) return launch_d<128, 64, LM_FP8>(a, maps, s);
+    return launch_d<128, 128, LM_FP8>(a, maps, s);
+  }
   if (a.d == 64 && a.bk == 64) return launch_d<64, 64, LM_IMAGE>(a, maps, s);
   if (a.d == 64 && a.bk == 128) return launch_d<64, 128, LM_IMAGE>(a, maps, s);
   if (a.d == 128 && a.bk == 64) return launch_d<128, 64, LM_IMAGE>(a, maps, s);
   if (a.low == TA_LOW_NVFP4) return launch_d<128, 128, LM_NVFP4>(a, maps, s);
   if (a.low == TA_LOW_NVFP4_RES) return launch_d<128, 128, LM_NVFP4_RES>(a, maps, s);
-  if (a.low == TA_LOW_FP8_E4M3 && a.bq == 128) return launch_d<128, 128, LM_FP8>(a, maps, s);
   return launch_d<128, 128, LM_IMAGE>(a, maps, s);
 }
 

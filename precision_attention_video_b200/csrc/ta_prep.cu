@@ -15,10 +15,7 @@
 //   * NVFP4: per 16 elements along d (Q, K rows) or along tokens (V columns,
 //     groups aligned to token 0) a ue4m3 scale sc = e4m3_rn(amax / 6), codes
 //     e2m1_rn_satfinite(x * rcp_rn(sc)); residual copies quantise
-//     fp32(x - dequant(x)) the same way;
-//   * for an FP8 low tier that the attention kernel runs on bf16 images (d =
-//     64 or 64-row tiles), the dequantised values in bf16 (exact: at most 4
-//     significant bits), row-major like the input.
+//     fp32(x - dequant(x)) the same way.
 // One CTA per (chunk of R = max(bq, bk) tokens, head, operand Q / K / V); the
 // chunk is staged in shared memory with 16-byte coalesced loads and written
 // back coalesced.

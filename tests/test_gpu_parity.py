@@ -50,7 +50,7 @@ def _plan_parity(cfg, Q, K, V, views, heads):
             for t in "qkv":
                 np.testing.assert_array_equal(views[f"{t}_codes"][bh].numpy(), qt[f"{t}_codes"])
                 np.testing.assert_array_equal(views[f"{t}_scales"][bh].numpy().astype(np.float64), qt[f"{t}_scale"])
-                if f"d{t}" in views:   # images exist only where a tile path reads them
+                if f"d{t}" in views:   # no bf16 images are kept (the views are absent)
                     np.testing.assert_array_equal(to64(views[f"d{t}"][bh]), qt[f"d{t}"][:cfg.N])
         elif cfg.low in (Qz.LOW_NVFP4, Qz.LOW_NVFP4_RES):
             pres = ["", "r"] if cfg.low == Qz.LOW_NVFP4_RES else [""]
@@ -62,7 +62,7 @@ def _plan_parity(cfg, Q, K, V, views, heads):
                 check_vt(views[f"{pre}v_codes"][bh].numpy(), views[f"{pre}v_scales"][bh].numpy(),
                          qt[f"{pre}v_codes"], qt[f"{pre}v_sc"])
             for t in "qkv":
-                if f"d{t}" in views:   # bf16 images exist only where a tile path reads them
+                if f"d{t}" in views:   # no bf16 images are kept (the views are absent)
                     np.testing.assert_array_equal(to64(views[f"d{t}"][bh]), qt[f"d{t}"][:cfg.N])
             if cfg.low == Qz.LOW_NVFP4_RES:
                 for t, key in (("q", "rq"), ("k", "rk"), ("v", "rv")):
@@ -197,8 +197,8 @@ def _forward_parity(cfg, Q, K, V, what, need_tiers=()):
 
 
 def test_forward_parity_d128_query_blocks_of_64(cuda_ok):
-    # d = 128 with 64-row query blocks and 128-key tiles: the FP8 tiles run on
-    # bf16 images, and the TMEM lanes of rows 64..127 carry no query rows
+    # d = 128 with 64-row query blocks and 128-key tiles: native FP8 tiles in
+    # the 16-warp kernel, whose TMEM lanes of rows 64..127 carry no query rows
     cfg, Q, K, V = inputs("sweep70", grid=(3, 10, 21), H=2, block_q=64)
     _forward_parity(cfg, Q, K, V, "d128 bq64", need_tiers=(1, 3))
 
@@ -237,7 +237,7 @@ NOMINAL_FP8 = (0.0, 2.0, 3.0, 4.0)
     ("480p-price", (3, 10, 21), 0.028, NOMINAL_NVFP4, 3),  # bf16, NVFP4 + residual, NVFP4, skip
     ("480p", (3, 10, 21), 0.04, NOMINAL_NVFP4, 3),         # NVFP4 low tier
     ("sweep70", (3, 10, 21), 0.06, NOMINAL_FP8, 3),        # native FP8 low tier
-    ("small", None, 0.002, NOMINAL_FP8, 3),                # FP8 low tier on bf16 images
+    ("small", None, 0.002, NOMINAL_FP8, 3),                # FP8 low tier, d = 64, 64-key tiles
     ("480p-price", (3, 10, 21), 0.05, (0.0, 0.0, 0.0, 0.0), 2),   # the default (measured) costs
 ])
 def test_price_router_parity(cuda_ok, name, grid, price, cost, n_tiers):
@@ -303,7 +303,7 @@ def test_plan_reuse_parity(cuda_ok):
     ("480p", (3, 10, 21), 0.5),          # NVFP4 low tier
     ("720p", (3, 9, 20), 1.0),           # four tiers
     ("sweep70", (3, 10, 21), 0.5),       # native FP8 low tier
-    ("small", None, 0.5),                # FP8 low tier on bf16 images
+    ("small", None, 0.5),                # FP8 low tier, d = 64, 64-key tiles
 ])
 def test_entropy_router_parity(cuda_ok, name, grid, kappa):
     over = {"H": 2, "router": 2, "kappa": kappa}
