@@ -847,12 +847,30 @@ __global__ void __launch_bounds__(kThreads2, 1)
     // list: the only skipped block whose pooled key does not weigh KB
     const int n_last = a.N - (a.nKb - 1) * KB;
     const float w_last = (float)n_last;
+    // (only a skipped ragged block needs it, so only the skip segment of the
+    // list is searched, 128 entries per round of loads; rows of 32-key blocks
+    // keep the plain scan over the whole list, which measured faster there)
     int pos_last = -1000000;
-    if (n_last < KB) {
+    if (PK > 1 && n_last < KB) {
       for (int i0 = 0; i0 < a.nKb; i0 += 32) {
         const int i = i0 + lane;
         const unsigned bal = __ballot_sync(0xffffffffu, i < a.nKb && rp.list[i] == a.nKb - 1);
         if (bal) pos_last = i0 + __ffs(bal) - 1;
+      }
+    } else if (n_last < KB && rp.n_skip > 0) {
+      const int s0 = rp.n_full + rp.n_res + rp.n_low, s1 = s0 + rp.n_skip;
+      for (int i0 = s0; i0 < s1; i0 += 128) {
+        int v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + 32 * u + lane;
+          v[u] = i < s1 ? rp.list[i] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const unsigned bal = __ballot_sync(0xffffffffu, v[u] == a.nKb - 1);
+          if (bal) pos_last = i0 + 32 * u + __ffs(bal) - 1;
+        }
       }
     }
     float m_own = -INFINITY, l_own = 0.0f;   // this group's last max and its row sum
