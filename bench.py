@@ -47,7 +47,7 @@ L2_BYTES = 126 * 2 ** 20
 # kernel (attn2_kernel<LM_NVFP4, 128>) on 8 heads of that layer, scaled to 40
 # by heads (traffic grows with the (head, query block) rows); valid only for
 # the kernel sources it was measured on and for that workload.
-ATTN_TRAFFIC = {"source_sha1": "bbc9a9fcd43ca187737ecadeef396da59666b9f3", "bytes_per_launch": 1604586240}
+ATTN_TRAFFIC = {"source_sha1": "d223a0f993cc30019cade72bd2975369e1d42ed8", "bytes_per_launch": 1596980480}
 
 
 def _env_int(name, default):
