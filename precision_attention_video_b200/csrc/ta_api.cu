@@ -241,12 +241,6 @@ void fill_plan_args(const ta_params* p, const void* Q, const void* K, const void
   a.rq_scales = at<uint8_t>(ws, L.rq_scales);
   a.rk_scales = at<uint8_t>(ws, L.rk_scales);
   a.rv_scales = at<uint8_t>(ws, L.rv_scales);
-  a.dq = at<__nv_bfloat16>(ws, L.dq);
-  a.dk = at<__nv_bfloat16>(ws, L.dk);
-  a.dv = at<__nv_bfloat16>(ws, L.dv);
-  a.drq = at<__nv_bfloat16>(ws, L.drq);
-  a.drk = at<__nv_bfloat16>(ws, L.drk);
-  a.drv = at<__nv_bfloat16>(ws, L.drv);
 }
 
 // ---- TMA descriptors through the driver entry point (no libcuda link) ----

@@ -47,7 +47,6 @@ struct PlanArgs {
   void *q_scales, *k_scales, *v_scales;
   uint8_t *rq_codes, *rk_codes, *rv_codes;
   uint8_t *rq_scales, *rk_scales, *rv_scales;
-  __nv_bfloat16 *dq, *dk, *dv, *drq, *drk, *drv;
 };
 
 // Fused attention arguments.

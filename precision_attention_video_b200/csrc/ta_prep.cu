@@ -245,7 +245,6 @@ __global__ void __launch_bounds__(kThreads, 4) prep_kernel(const PlanArgs a) {
   if (a.low == TA_LOW_NONE) return;
 
   uint8_t* codes = which == 0 ? a.q_codes : which == 1 ? a.k_codes : a.v_codes;
-  __nv_bfloat16* deq_out = which == 0 ? a.dq : which == 1 ? a.dk : a.dv;
 
   if (a.low == TA_LOW_FP8_E4M3) {
     // ---- FP8: one power-of-two scale per tile of `blk` rows ----
@@ -268,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 4) prep_kernel(const PlanArgs a) {
       if (r >= nrows) continue;
       const float sc = tile_scale[r / blk];
       const float inv = 1.0f / sc;  // exact: sc is a power of two
-      __nv_bfloat16* px = tile + r * D + g * 16;
+      const __nv_bfloat16* px = tile + r * D + g * 16;
       uint32_t w[4];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -278,15 +277,12 @@ __global__ void __launch_bounds__(kThreads, 4) prep_kernel(const PlanArgs a) {
           w[i >> 1] |= c2 << 16;
         else
           w[i >> 1] = c2;
-        const float2 f = e4m3x2_to_float2(c2);
-        px[2 * i] = __float2bfloat16_rn(f.x * sc);
-        px[2 * i + 1] = __float2bfloat16_rn(f.y * sc);
       }
       *reinterpret_cast<uint4*>(codes + (bhN + r0 + r) * D + g * 16) =
           make_uint4(w[0], w[1], w[2], w[3]);
     }
   } else {
-    // ---- NVFP4 (+ residual); no bf16 images of these copies are kept ----
+    // ---- NVFP4 (+ residual) ----
     const bool res = (a.low == TA_LOW_NVFP4_RES);
     uint8_t* rcodes = which == 0 ? a.rq_codes : which == 1 ? a.rk_codes : a.rv_codes;
     uint8_t* scales = reinterpret_cast<uint8_t*>(which == 0 ? a.q_scales
@@ -368,15 +364,6 @@ __global__ void __launch_bounds__(kThreads, 4) prep_kernel(const PlanArgs a) {
       }
     }
   }
-  __syncthreads();
-  // ---- dequantised copy, coalesced (only where a tile path reads it) ----
-  if (deq_out != nullptr)
-    for (int idx = tid; idx < R * (D / 8); idx += kThreads) {
-      const int r = idx / (D / 8), c8 = idx % (D / 8);
-      if (r < nrows)
-        *reinterpret_cast<uint4*>(deq_out + (bhN + r0 + r) * D + c8 * 8) =
-            *reinterpret_cast<const uint4*>(tile + r * D + c8 * 8);
-    }
 }
 
 template <int D, int R>

@@ -74,3 +74,37 @@ def test_key_blocks_of_32_skip_only(cuda_ok):
     for h in range(cfg.H):
         _, _, Oref = oracle_head(cfg, Q, K, V, 0, h, tau=(0.0, 0.0))
         assert_out_close(to64(O[0, h]), Oref, f"skip-only head {h}")
+
+
+@pytest.mark.parametrize("N", [1, 17, 40, 100])
+def test_key_blocks_of_32_short_sequences(cuda_ok, N):
+    # sequences shorter than one 128-query block: one to four 32-key blocks,
+    # the last one ragged (N = 1, 17, 40, 100), every block of the row inside
+    # one packed tile with the forced diagonal
+    base, Q, K, V = inputs("480p-fg", grid=(3, 10, 21), H=2)
+    cfg = base.with_(grid=(1, 1, N))
+    Qs, Ks, Vs = (x[:, :, :N].contiguous() for x in (Q, K, V))
+    _, views, O, st = run_gpu(cfg, Qs, Ks, Vs)
+    assert st == 0
+    _plan_parity(cfg, Qs, Ks, Vs, views, [(0, h) for h in range(cfg.H)])
+    for h in range(cfg.H):
+        rt, _, Oref = oracle_head(cfg, Qs, Ks, Vs, 0, h)
+        n_diff, _ = compare_tiers(views["tier_map"][h].numpy(), rt)
+        assert n_diff == 0
+        assert_out_close(to64(O[0, h]), Oref, f"fg N={N} head {h}")
+
+
+def test_key_blocks_of_32_batch_of_two(cuda_ok):
+    # B = 2 with 32-key blocks: every (b, h) routed, packed and attended
+    # independently, strides over b (N = 320: ten 32-key blocks)
+    cfg, Q, K, V = inputs("480p-fg", grid=(2, 10, 16), H=2, B=2)
+    _, views, O, st = run_gpu(cfg, Q, K, V)
+    assert st == 0
+    _plan_parity(cfg, Q, K, V, views, [(b, h) for b in range(2) for h in range(2)])
+    for b in range(2):
+        for h in range(2):
+            rt, qt, Oref = oracle_head(cfg, Q, K, V, b, h)
+            _, rows = compare_tiers(views["tier_map"][b * cfg.H + h].numpy(), rt)
+            for i in rows:
+                Oref[i * cfg.block_q:(i + 1) * cfg.block_q] = np.nan
+            assert_out_close(to64(O[b, h]), Oref, f"fg batch {b} head {h}")
