@@ -47,7 +47,7 @@ L2_BYTES = 126 * 2 ** 20
 # kernel (attn2_kernel<LM_NVFP4, 128>) on 8 heads of that layer, scaled to 40
 # by heads (traffic grows with the (head, query block) rows); valid only for
 # the kernel sources it was measured on and for that workload.
-ATTN_TRAFFIC = {"source_sha1": "d223a0f993cc30019cade72bd2975369e1d42ed8", "bytes_per_launch": 1596980480}
+ATTN_TRAFFIC = {"source_sha1": "c6ce1c5746f83ed3fa1b162b3b4376714885727e", "bytes_per_launch": 1596980480}
 
 
 def _env_int(name, default):
@@ -84,9 +84,15 @@ def attn_source_sha1():
     """Hash of the attention kernel's sources (the kernel and the headers it
     inlines): a traffic figure holds only for the code it was measured on."""
     h = hashlib.sha1()
-    for name in ("ta_attn2.cu", "ta_attn_common.cuh", "ta_common.cuh", "ta_kernels.cuh"):
-        with open(os.path.join(ROOT, "precision_attention_video_b200", "csrc", name), "rb") as f:
+    csrc = os.path.join(ROOT, "precision_attention_video_b200", "csrc")
+    for name in ("ta_attn2.cu", "ta_attn_common.cuh", "ta_common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
+    # of the shared argument header, only the struct the kernel takes
+    with open(os.path.join(csrc, "ta_kernels.cuh")) as f:
+        hdr = f.read()
+    start = hdr.index("struct AttnArgs {")
+    h.update(hdr[start:hdr.index("};", start)].encode())
     return h.hexdigest()
 
 
