@@ -78,3 +78,29 @@ def test_bf16_peak_follows_the_sampled_clock():
     assert bench.bf16_peak(peaks, slow)[0] == 1365.0
     none = {"sm_mhz": None, "sm_max_mhz": None, "reasons": []}
     assert "sustained" in bench.bf16_peak(peaks, none)[1]
+
+
+def test_kernel_named_in_the_roofline_follows_the_dispatch():
+    # the two-group kernel for d = 128 with 128-query blocks and 128- or
+    # 32-key blocks, except residual layers tiered by thresholds; the 16-warp
+    # kernel for the other shapes (FP8 natively at every shape)
+    from latent_gen import get_config
+    want = {"480p": "attn2_kernel<LM_NVFP4, 128>", "480p-fg": "attn2_kernel<LM_NVFP4, 32>",
+            "480p-price": "attn2_kernel<LM_NVFP4_RES, 128>", "sweep70": "attn2_kernel<LM_FP8, 128>",
+            "720p": "attn_kernel<128, 128, LM_NVFP4_RES>", "small": "attn_kernel<64, 64, LM_FP8>",
+            "tiny": "attn_kernel<64, 64, LM_FP8>"}
+    bench = _bench()
+    for name, kernel in want.items():
+        assert bench.attn_kernel_name(get_config(name)) == kernel, name
+    assert bench.attn_kernel_name(get_config("sweep70").with_(block_q=64)) == "attn_kernel<128, 128, LM_FP8>"
+
+
+def test_traffic_figure_is_tied_to_the_kernel_sources():
+    # the recorded DRAM traffic belongs to the sources it was captured on
+    # (the bench line reports it only while the hash matches); the hash is
+    # stable across calls and covers the kernel file, its headers and its
+    # argument struct
+    bench = _bench()
+    h = bench.attn_source_sha1()
+    assert len(h) == 40 and h == bench.attn_source_sha1()
+    assert bench.ATTN_TRAFFIC["bytes_per_launch"] > 0 and len(bench.ATTN_TRAFFIC["source_sha1"]) == 40

@@ -27,6 +27,8 @@ CASES = [
     ("small", {"H": 3, "router": 1, "price": 0.002}),        # price router, FP8 tiers
     ("480p", {"H": 2, "grid": (3, 10, 21), "router": 2, "kappa": 0.5}),  # entropy router
     ("720p", {"H": 2, "grid": (3, 9, 20), "router": 2, "kappa": 1.0}),   # entropy, four tiers
+    ("480p-fg", {"H": 2, "grid": (3, 10, 21)}),              # 32-key blocks, ragged
+    ("480p-fg", {"H": 1, "grid": (4, 32, 72)}),              # 288 32-key blocks a row (CTA-a-row router)
 ]
 
 
