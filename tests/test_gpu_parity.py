@@ -403,3 +403,37 @@ def test_long_row_router_parity(cuda_ok, name, over):
     assert st == 0
     assert len(np.unique(views["tier_map"].numpy())) >= 2
     _plan_parity(cfg, Q, K, V, views, [(0, 0)])
+
+
+def test_long_row_router_orders_masses_that_share_a_float(cuda_ok):
+    # The router of rows longer than 256 key blocks sorts on the float of
+    # each block's mass (then j) and repairs the order among masses that
+    # round to the same float.  Here 40 key blocks differ only in one
+    # coordinate of one key, which the queries weigh by 2^-12: their masses
+    # differ by about 3e-9 relative (one float), and increase with j, so the
+    # float sort alone would list them in the wrong order.
+    nkb, d = 300, 128
+    N = nkb * 128
+    cfg = inputs("480p", grid=(3, 10, 21), H=1)[0].with_(grid=(1, 1, N), H=1)
+    rng = np.random.default_rng(5)
+    base = np.round(rng.normal(size=d) * 0.5 * 128) / 128
+    base[0] = 1.0
+    K = np.tile(base, (N, 1)) + np.round(rng.normal(size=(N, d)) * 0.01 * 256) / 256
+    K[:, 0] = 1.0
+    g0 = 100
+    for u in range(40):                        # the near-tied group: blocks g0 .. g0 + 39
+        blk = slice((g0 + u) * 128, (g0 + u + 1) * 128)
+        K[blk] = K[g0 * 128:(g0 + 1) * 128]      # a copy of block g0 ...
+        K[(g0 + u) * 128, 0] = 1.0 + u * 2.0 ** -6   # ... but for one coordinate of one key
+    Qm = np.round(rng.normal(size=(N, d)) * 256) / 256
+    Qm[:, 0] = 2.0 ** -12
+    V = rng.normal(size=(N, d))
+    to_bf16 = lambda a: torch.from_numpy(a).to(torch.bfloat16).reshape(1, 1, N, d)
+    Q, Kt, Vt = to_bf16(Qm), to_bf16(K), to_bf16(V)
+    _, views, _, st = run_gpu(cfg, Q, Kt, Vt, forward=False)
+    assert st == 0
+    # the group's masses: distinct doubles, one float at most a few
+    mass = views["mass"][0].numpy()
+    grp = mass[0, g0:g0 + 40]
+    assert len(np.unique(grp)) > 30 and len(np.unique(grp.astype(np.float32))) <= 4
+    _plan_parity(cfg, Q, Kt, Vt, views, [(0, 0)])
