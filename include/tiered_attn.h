@@ -81,7 +81,10 @@ enum { TA_TIER_SKIP = 0, TA_TIER_LOW = 1, TA_TIER_RES = 2, TA_TIER_FULL = 3 };
 typedef struct {
   int32_t B, H, N, d;        /* batch, heads, tokens (N >= 1; the last query and
                                 key blocks may be partial, down to one token),
-                                head dim (d in {64,128})                       */
+                                head dim (d in {64,128}).  Limits, else
+                                TA_ERR_UNSUPPORTED: B * H <= 65535 and
+                                ceil(N / block_k) <= 1024 key blocks (the
+                                width of the router's per-row sort)            */
   int32_t block_q, block_k;  /* query rows in {64,128}; keys per block in
                                 {32,64,128}.  32-key blocks ("FG-Attn",
                                 searcharxiv author page, abstract: skipping at

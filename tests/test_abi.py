@@ -79,6 +79,34 @@ def test_workspace_bytes_and_validation(pav):
     assert pav.workspace_bytes(_params(pav, router=2, retention=0.5)) == n
 
 
+def test_shape_limits_at_their_edges(pav):
+    ws = pav.workspace_bytes
+    fg = dict(d=128, block_q=128, block_k=32, low=2, tau=(0.6, 0.9))   # NVFP4
+    # 32-key blocks: d = 128, 128-query blocks, bf16 / NVFP4 / NVFP4 + residual
+    assert ws(_params(pav, **fg)) > 0
+    assert ws(_params(pav, **dict(fg, low=0, tau=(0.9,)))) > 0
+    assert ws(_params(pav, **dict(fg, low=3, tau=(0.5, 0.6, 0.8)))) > 0
+    assert ws(_params(pav, **dict(fg, low=1))) == 0        # FP8
+    assert ws(_params(pav, **dict(fg, d=64))) == 0
+    assert ws(_params(pav, **dict(fg, block_q=64))) == 0
+    # the router sorts at most 1024 key blocks a row: N up to 1024 blocks,
+    # the last one ragged or whole, and not one token more
+    for bk in (32, 64, 128):
+        kw = dict(fg, block_k=bk)
+        assert ws(_params(pav, **dict(kw, N=1024 * bk))) > 0, bk
+        assert ws(_params(pav, **dict(kw, N=1023 * bk + 1))) > 0, bk
+        assert ws(_params(pav, **dict(kw, N=1024 * bk + 1))) == 0, bk
+    # one CTA row per (batch, head): B * H <= 65535
+    assert ws(_params(pav, B=1, H=65535, N=64)) > 0
+    assert ws(_params(pav, B=3, H=21845, N=64)) > 0
+    assert ws(_params(pav, B=2, H=32768, N=64)) == 0
+    # P' offsets 2^0 .. 2^15
+    assert ws(_params(pav, p_offset_log2=0)) > 0
+    assert ws(_params(pav, p_offset_log2=15)) > 0
+    assert ws(_params(pav, p_offset_log2=16)) == 0
+    assert ws(_params(pav, p_offset_log2=-1)) == 0
+
+
 def test_calls_reject_bad_arguments_before_launch(pav):
     lib = pav.binding.lib() if hasattr(pav, "binding") else None
     from precision_attention_video_b200 import binding as B
