@@ -152,8 +152,10 @@ __global__ void __launch_bounds__(kThreads, 4) prep_kernel(const PlanArgs a) {
   // in fp64 while a block's values span at most 38 binades (53 - 8 - 7 bits),
   // and then the order of the additions does not matter.  Each thread takes
   // two adjacent columns over one segment of RS rows (zero rows add nothing) ----
+  // block sizes are powers of two (32, 64 or 128 rows): shifts, not divisions
   const int blk = (which == 0) ? a.bq : a.bk;
-  const int nb = R / blk;
+  const int lb = __ffs(blk) - 1;            // log2(blk)
+  const int nb = R >> lb;
   {
     const int cp = tid % L::CP, seg = tid / L::CP;
     const uint32_t* col = tile32 + seg * L::RS * L::CP + cp;
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 4) prep_kernel(const PlanArgs a) {
     amax_c[u] = 0.0f;
     if (w < nb * D) {
       const int jb = w / D, c = w % D;
-      const int spb = L::SEG / nb;   // segments per block
+      const int spb = L::SEG >> (__ffs(nb) - 1);   // segments per block
       for (int k = 0; k < spb; ++k) {
         s[u] += psum[(jb * spb + k) * D + c];
         amax_c[u] = fmaxf(amax_c[u], red[(jb * spb + k) * D + c]);
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 4) prep_kernel(const PlanArgs a) {
     const int rs = jb * blk, re = min(rs + blk, nrows);
     red[w] = amax_c[u];
     if (re > rs) {
-      const int gb = r0 / blk + jb;
+      const int gb = (r0 >> lb) + jb;
       const double mean = s[u] / (double)(re - rs);
       if (which == 0) {
         a.qbar[((int64_t)bh * a.nQb + gb) * D + c] = mean;
@@ -253,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 4) prep_kernel(const PlanArgs a) {
       for (int c = 0; c < D; ++c) amax = fmaxf(amax, red[tid * D + c]);
       const float sc = fp8_pow2_scale(amax);
       tile_scale[tid] = sc;
-      const int gb = r0 / blk + tid;
+      const int gb = (r0 >> lb) + tid;
       if (tid * blk < nrows) {
         float* scp = reinterpret_cast<float*>(which == 0 ? a.q_scales
                                               : which == 1 ? a.k_scales
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 4) prep_kernel(const PlanArgs a) {
     for (int idx = tid; idx < R * (D / 16); idx += kThreads) {
       const int r = idx / (D / 16), g = idx % (D / 16);
       if (r >= nrows) continue;
-      const float sc = tile_scale[r / blk];
+      const float sc = tile_scale[r >> lb];
       const float inv = 1.0f / sc;  // exact: sc is a power of two
       const __nv_bfloat16* px = tile + r * D + g * 16;
       uint32_t w[4];
@@ -356,11 +358,20 @@ __global__ void __launch_bounds__(kThreads, 4) prep_kernel(const PlanArgs a) {
       __syncthreads();
       const int gv = min(L::G, (a.Np - r0) / 16);   // groups below the pitch
       const int copies = res ? 2 : 1;
-      for (int idx = tid; idx < copies * D * gv; idx += kThreads) {
-        const int copy = idx / (D * gv), rem = idx % (D * gv);
-        const int c = rem / gv, g = rem % gv;
+      // 8 bytes (group g of column c) of one copy's codes
+      auto put = [&](int copy, int c, int g) {
         uint8_t* dst = (copy ? rcodes : codes) + ((int64_t)bh * D + c) * (a.Np / 2) + r0 / 2 + g * 8;
         *reinterpret_cast<uint2*>(dst) = vst[(copy * L::G + g) * L::VP + c];
+      };
+      if (gv == L::G) {
+        // every chunk but the sequence's last: compile-time index arithmetic
+        for (int idx = tid; idx < copies * D * L::G; idx += kThreads)
+          put(idx / (D * L::G), (idx / L::G) % D, idx % L::G);
+      } else {
+        for (int idx = tid; idx < copies * D * gv; idx += kThreads) {
+          const int copy = idx / (D * gv), rem = idx % (D * gv);
+          put(copy, rem / gv, rem % gv);
+        }
       }
     }
   }
