@@ -111,6 +111,52 @@ def _check(call: str, code: int) -> None:
         raise TieredAttnError(call, code)
 
 
+def _span(p: ta_params) -> int:
+    """Elements from the first element of a [B, H, N, d] operand with p's
+    strides to one past the last one the library reads or writes."""
+    return (p.B - 1) * p.stride_b + (p.H - 1) * p.stride_h + (p.N - 1) * p.stride_n + p.d
+
+
+def _elems_after(t: torch.Tensor) -> int:
+    """Elements of t's storage from t's first element on."""
+    return t.untyped_storage().nbytes() // t.element_size() - t.storage_offset()
+
+
+def _operand(name: str, t, *, cuda: bool = True, dtype=None, need: int = 0) -> int:
+    """t's data pointer, after the checks that the C ABI cannot make on a bare
+    pointer: a CUDA tensor on the current device (the library launches there)
+    or, with cuda=False, a host tensor; of `dtype`; with at least `need`
+    elements of storage from its first element on."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if cuda:
+        if not t.is_cuda:
+            raise ValueError(f"{name}: expected a CUDA tensor, got one on {t.device}")
+        cur = torch.cuda.current_device()
+        if t.device.index != cur:
+            raise ValueError(f"{name}: on {t.device}, but the library launches on the current "
+                             f"device cuda:{cur}")
+    elif t.device.type != "cpu":
+        raise ValueError(f"{name}: expected a host tensor, got one on {t.device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if need and _elems_after(t) < need:
+        raise ValueError(f"{name}: {_elems_after(t)} elements of storage from its first element, "
+                         f"the layout of the parameters needs {need}")
+    return t.data_ptr()
+
+
+def _qkv(p: ta_params, Q, K, V, cuda: bool = True, names=("Q", "K", "V")):
+    """Pointers of three bf16 [B, H, N, d] operands laid out by p's strides."""
+    n = _span(p)
+    return tuple(_operand(nm, t, cuda=cuda, dtype=torch.bfloat16, need=n)
+                 for nm, t in zip(names, (Q, K, V)))
+
+
+def _ws(ws) -> int:
+    return _operand("ws", ws, dtype=torch.uint8)
+
+
 def make_params(B: int, H: int, N: int, d: int, block_q: int, block_k: int, low: int,
                 tau: Sequence[float], p_offset_log2: int, keep_diag_full: int = 1,
                 softmax_scale: float = 0.0, debug_flags: int = 0,
@@ -164,50 +210,62 @@ def alloc_workspace(p: ta_params, device="cuda") -> torch.Tensor:
 
 def plan(p: ta_params, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, ws: torch.Tensor,
          stream=None) -> None:
+    q, k, v = _qkv(p, Q, K, V)
     _check("tiered_attn_plan", lib().tiered_attn_plan(
-        ctypes.byref(p), Q.data_ptr(), K.data_ptr(), V.data_ptr(), ws.data_ptr(),
-        ws.numel(), _stream(stream)))
+        ctypes.byref(p), q, k, v, _ws(ws), ws.numel(), _stream(stream)))
 
 
 def prep(p, Q, K, V, ws, stream=None) -> None:
+    q, k, v = _qkv(p, Q, K, V)
     _check("tiered_attn_prep", lib().tiered_attn_prep(
-        ctypes.byref(p), Q.data_ptr(), K.data_ptr(), V.data_ptr(), ws.data_ptr(),
-        ws.numel(), _stream(stream)))
+        ctypes.byref(p), q, k, v, _ws(ws), ws.numel(), _stream(stream)))
 
 
 def route(p, ws, stream=None) -> None:
     _check("tiered_attn_route", lib().tiered_attn_route(
-        ctypes.byref(p), ws.data_ptr(), ws.numel(), _stream(stream)))
+        ctypes.byref(p), _ws(ws), ws.numel(), _stream(stream)))
 
 
 def route_noalloc(p: ta_params, Q, K, V, tier_map, row_counts, row_lists, stream=None) -> None:
     """Tier map, row counts and row lists without any workspace: the router's
-    intermediates live in the library's fixed device array (see the header)."""
+    intermediates live in the library's fixed device array (see the header).
+    Operands must be CUDA tensors on the current device, Q, K, V bf16; their
+    sizes are the caller's to get right, as in the C ABI (the library checks
+    the problem against its scratch before reading any of them)."""
+    q, k, v = (_operand(nm, t, dtype=torch.bfloat16) for nm, t in (("Q", Q), ("K", K), ("V", V)))
     _check("tiered_attn_route_noalloc", lib().tiered_attn_route_noalloc(
-        ctypes.byref(p), Q.data_ptr(), K.data_ptr(), V.data_ptr(), tier_map.data_ptr(),
-        row_counts.data_ptr(), row_lists.data_ptr(), _stream(stream)))
+        ctypes.byref(p), q, k, v, _operand("tier_map", tier_map),
+        _operand("row_counts", row_counts), _operand("row_lists", row_lists), _stream(stream)))
 
 
 def forward(p: ta_params, Q, K, V, ws, O, stream=None) -> None:
+    q, k, v = _qkv(p, Q, K, V)
+    o = _operand("O", O, dtype=torch.bfloat16, need=_span(p))
     _check("tiered_attn_forward", lib().tiered_attn_forward(
-        ctypes.byref(p), Q.data_ptr(), K.data_ptr(), V.data_ptr(), ws.data_ptr(), ws.numel(),
-        O.data_ptr(), _stream(stream)))
+        ctypes.byref(p), q, k, v, _ws(ws), ws.numel(), o, _stream(stream)))
 
 
 def layer_from_host(p, Qh, Kh, Vh, Oh, Qd, Kd, Vd, Od, ws, stream=None) -> None:
+    """One layer from host buffers: Qh, Kh, Vh, Oh host bf16 tensors (pinned
+    for overlapped copies), Qd, Kd, Vd, Od device bf16 tensors of the same
+    layout, all laid out by p's strides."""
+    qh, kh, vh = _qkv(p, Qh, Kh, Vh, cuda=False, names=("Qh", "Kh", "Vh"))
+    oh = _operand("Oh", Oh, cuda=False, dtype=torch.bfloat16, need=_span(p))
+    qd, kd, vd = _qkv(p, Qd, Kd, Vd, names=("Qd", "Kd", "Vd"))
+    od = _operand("Od", Od, dtype=torch.bfloat16, need=_span(p))
     _check("tiered_attn_layer_from_host", lib().tiered_attn_layer_from_host(
-        ctypes.byref(p), Qh.data_ptr(), Kh.data_ptr(), Vh.data_ptr(), Oh.data_ptr(),
-        Qd.data_ptr(), Kd.data_ptr(), Vd.data_ptr(), Od.data_ptr(), ws.data_ptr(), ws.numel(),
-        _stream(stream)))
+        ctypes.byref(p), qh, kh, vh, oh, qd, kd, vd, od, _ws(ws), ws.numel(), _stream(stream)))
 
 
 def get_status(ws: torch.Tensor, stream=None) -> int:
-    return int(lib().tiered_attn_get_status(ws.data_ptr(), _stream(stream)))
+    return int(lib().tiered_attn_get_status(_ws(ws), _stream(stream)))
 
 
 def plan_views(p: ta_params, ws: torch.Tensor) -> Dict[str, torch.Tensor]:
     """Typed tensor views of a planned workspace (no copies)."""
     v = ta_plan_views()
+    if ws.dtype != torch.uint8:
+        raise TypeError(f"ws: expected torch.uint8, got {ws.dtype}")
     _check("tiered_attn_plan_views", lib().tiered_attn_plan_views(
         ctypes.byref(p), ws.data_ptr(), ctypes.byref(v)))
     BH = p.B * p.H
