@@ -1,0 +1,116 @@
+"""The seeded input generator does what the stated input recipe says: the
+workload table (shapes, grids, logit scales, tiles, formats, thresholds),
+reproducible per-(b, h) streams independent of threading, Q.K logits at the
+calibrated standard deviation, unit-normal V, a stationary spatio-temporal
+kernel (nearby tokens attend more), and plan-reuse sequences whose
+consecutive steps correlate by rho.  The generator holds none of the
+method's arithmetic; it feeds the oracle and the CUDA path alike."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from latent_gen import get_config, make_qkv
+from latent_gen.configs import LOW_FP8, LOW_NVFP4, LOW_NVFP4_RES
+from latent_gen.generator import grid_positions, make_qkv_steps
+
+
+@pytest.mark.parametrize("name,shape,grid,std,tile,low,tau", [
+    ("tiny", (1, 2, 1024, 64), (4, 16, 16), 3.0, (64, 64), LOW_FP8, (0.7, 0.95)),
+    ("small", (1, 12, 8192, 64), (8, 32, 32), 3.0, (128, 64), LOW_FP8, (0.6, 0.9)),
+    ("480p", (1, 40, 32760, 128), (21, 30, 52), 4.0, (128, 128), LOW_NVFP4, (0.6, 0.9)),
+    ("720p", (1, 24, 118800, 128), (33, 45, 80), 4.0, (128, 128), LOW_NVFP4_RES, (0.5, 0.675, 0.85)),
+    ("480p-fg", (1, 40, 32760, 128), (21, 30, 52), 4.0, (128, 32), LOW_NVFP4, (0.6, 0.9)),
+])
+def test_workload_table(name, shape, grid, std, tile, low, tau):
+    c = get_config(name)
+    assert (c.B, c.H, c.N, c.d) == shape and c.grid == grid
+    assert c.logit_std == std and (c.block_q, c.block_k) == tile
+    assert c.low == low and tuple(c.tau) == tau
+    assert (c.noise, c.n_features, c.seed) == (0.3, 32, 0)
+
+
+def test_sweep_points_share_the_480p_shape():
+    base = get_config("480p")
+    for pct in (0, 30, 50, 70, 90):
+        c = get_config(f"sweep{pct}")
+        assert (c.B, c.H, c.N, c.d, c.grid) == (base.B, base.H, base.N, base.d, base.grid)
+        assert c.low == LOW_FP8
+    # the all-full point's thresholds lie above every cumulative mass
+    assert min(get_config("sweep0").tau) > 1.0
+
+
+def test_raster_order_is_t_major():
+    p = grid_positions((2, 3, 4))
+    assert p.shape == (24, 3)
+    assert tuple(p[0]) == (0, 0, 0) and tuple(p[1]) == (0, 0, 1) and tuple(p[4]) == (0, 1, 0)
+    assert tuple(p[12]) == (1, 0, 0) and tuple(p[23]) == (1, 2, 3)
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    cfg = get_config("tiny")
+    return cfg, make_qkv(cfg)
+
+
+def test_reproducible_and_independent_of_threads(tiny):
+    cfg, (Q, K, V) = tiny
+    assert Q.dtype == torch.bfloat16 and Q.shape == (cfg.B, cfg.H, cfg.N, cfg.d)
+    Q1, K1, V1 = make_qkv(cfg, threads=1)
+    assert torch.equal(Q, Q1) and torch.equal(K, K1) and torch.equal(V, V1)
+    # each (b, h) has its own stream: heads differ, and a head does not
+    # depend on how many heads the layer has
+    assert not torch.equal(Q[0, 0], Q[0, 1])
+    Q2, _, _ = make_qkv(cfg.with_(H=1))
+    assert torch.equal(Q2[0, 0], Q[0, 0])
+    Q3, _, _ = make_qkv(cfg.with_(seed=1))
+    assert not torch.equal(Q3, Q)
+
+
+def test_logit_std_and_value_distribution(tiny):
+    cfg, (Q, K, V) = tiny
+    for h in range(cfg.H):
+        q = Q[0, h].double()
+        k = K[0, h].double()
+        s = (q @ k.T) / math.sqrt(cfg.d)
+        # calibrated on 2^18 sampled pairs of the fp32 values; all N^2 pairs
+        # of the bf16-rounded ones land within a few percent
+        assert abs(s.std().item() / cfg.logit_std - 1.0) < 0.05, s.std().item()
+        v = V[0, h].double()
+        assert abs(v.mean().item()) < 0.02 and abs(v.std().item() - 1.0) < 0.02
+
+
+def test_logits_form_a_stationary_local_kernel(tiny):
+    # Q and K share G, so q(p).k(p') depends on p - p' (up to the noise):
+    # tokens one frame / row / column apart score well above random pairs,
+    # and the same offset scores alike anywhere in the grid
+    cfg, (Q, K, V) = tiny
+    T, Y, X = cfg.grid
+    q = Q[0, 0].double().reshape(T, Y, X, cfg.d)
+    k = K[0, 0].double().reshape(T, Y, X, cfg.d)
+    s = torch.einsum("tyxd,uvwd->tyxuvw", q, k) / math.sqrt(cfg.d)
+    near = s[0, 0, 0, 0, 0, 1].item(), s[0, 0, 0, 0, 1, 0].item(), s[0, 0, 0, 1, 0, 0].item()
+    far_mean = s.mean().item()
+    assert all(x > far_mean + cfg.logit_std for x in near), (near, far_mean)
+    # stationarity: the mean logit at offset (0, 0, 1) is the same in both
+    # halves of the grid, within the noise
+    off = torch.stack([s[t, y, x, t, y, x + 1] for t in range(T) for y in range(Y) for x in range(X - 1)])
+    half = len(off) // 2
+    assert abs(off[:half].mean() - off[half:].mean()).item() < 0.5
+
+
+def test_plan_reuse_steps_correlate_by_rho():
+    cfg = get_config("tiny").with_(H=1)
+    rho = 0.9
+    seq = make_qkv_steps(cfg, 3, rho)
+    assert torch.equal(seq[0][0], make_qkv(cfg)[0])
+    for t in (1, 2):
+        for i in range(3):
+            a = seq[t - 1][i].double().flatten()
+            b = seq[t][i].double().flatten()
+            r = np.corrcoef(a.numpy(), b.numpy())[0, 1]
+            assert abs(r - rho) < 0.02, (t, i, r)
+        # the mix keeps unit variance where the draws have it (V)
+        assert abs(seq[t][2].double().std().item() - 1.0) < 0.02
