@@ -28,8 +28,11 @@
  *    multiple of 16.
  *  - Pointers named *_dev are device pointers; *_host are host pointers (pinned
  *    memory gives asynchronous copies).  The caller owns and allocates every
- *    buffer, including the workspace; the library allocates no memory and keeps
- *    no state between calls (besides cached driver entry points).
+ *    buffer, including the workspace; no call allocates memory.  State the
+ *    library keeps between calls: cached driver entry points, the copy
+ *    streams and events of tiered_attn_layer_from_host (created on its first
+ *    use on a device), and the fixed device array of
+ *    tiered_attn_route_noalloc (part of the module image).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *    Work is enqueued asynchronously on it; only the calls documented as
  *    synchronising wait for the device.
