@@ -70,3 +70,33 @@ def test_header_compiles_as_c_and_as_cpp(tmp_path):
         subprocess.run([exe, std, "-Wall", "-Wextra", "-Werror", "-pedantic", "-I",
                         os.path.join(ROOT, "include"), str(src), "-o", str(tmp_path / "inc")],
                        check=True, capture_output=True)
+
+
+def test_default_tier_costs_agree_between_header_oracle_and_calibration(tmp_path):
+    # the price router's default costs are stated twice, independently: in
+    # the header (what the library uses when tier_cost is all zero) and in the
+    # oracle; the stored price was calibrated with them
+    import json
+
+    from latent_gen import get_config
+    from oracle import route as R
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    names = ["SKIP", "FP8", "NVFP4", "NVFP4_RES", "FULL"]
+    src = tmp_path / "cost.c"
+    src.write_text('#include <stdio.h>\n#include "tiered_attn.h"\nint main(void) {\n' +
+                   "".join(f'  printf("%.17g\\n", (double)TA_TIER_COST_{n});\n' for n in names) +
+                   "  return 0;\n}\n")
+    subprocess.run([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                    str(tmp_path / "cost")], check=True, capture_output=True)
+    out = subprocess.run([str(tmp_path / "cost")], check=True, capture_output=True, text=True).stdout
+    c = dict(zip(names, (float(x) for x in out.split())))
+    for low, low_cost in ((B.TA_LOW_FP8_E4M3, c["FP8"]), (B.TA_LOW_NVFP4, c["NVFP4"]),
+                          (B.TA_LOW_NVFP4_RES, c["NVFP4"])):
+        assert R.default_tier_cost(low) == (c["SKIP"], low_cost, c["NVFP4_RES"], c["FULL"]), low
+    with open(os.path.join(ROOT, "latent_gen", "price.json")) as f:
+        stored = json.load(f)
+    cfg = get_config("480p-price")
+    assert tuple(stored["tier_cost"]) == R.default_tier_cost(cfg.low)
+    assert stored["price"] == cfg.price and not any(cfg.tier_cost)
