@@ -42,6 +42,22 @@ def test_sweep_points_share_the_480p_shape():
     assert min(get_config("sweep0").tau) > 1.0
 
 
+def test_calibrated_workloads_read_their_stored_values():
+    # the thresholds, price and retention written by the oracle's calibration
+    # scripts are the ones the workloads carry
+    import json
+    import os
+    here = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "latent_gen")
+    with open(os.path.join(here, "sweep_tau.json")) as f:
+        points = json.load(f)["points"]
+    assert sorted(points) == ["sweep30", "sweep50", "sweep70", "sweep90"]
+    for name, rec in points.items():
+        assert tuple(get_config(name).tau) == tuple(rec["tau"])
+        assert abs(rec["achieved"]["skip"] - int(name[5:]) / 100) < 1e-3
+    with open(os.path.join(here, "kappa.json")) as f:
+        assert get_config("480p-entropy").kappa == json.load(f)["kappa"]
+
+
 def test_raster_order_is_t_major():
     p = grid_positions((2, 3, 4))
     assert p.shape == (24, 3)
